@@ -173,16 +173,22 @@ def quantize_rtn(w_bits: np.ndarray, symmetric: bool, awq_s: np.ndarray | None =
     return codes, scale16, zero16
 
 
+# Nibble i (bits 4i..4i+3) of packed word w holds the code of input channel
+# 8w + PACK_ORDER[i].  Pairs of nibbles (i, i+4) are then the adjacent
+# channels (2i, 2i+1).
+PACK_ORDER = (0, 2, 4, 6, 1, 3, 5, 7)
+
+
 def pack_codes(codes: np.ndarray) -> np.ndarray:
-    """Pack [N, K] codes into int32 [N, K/8]: code k sits in bits 4*(k%8)..+3
-    of word k/8 (little-endian nibbles).  The pages give sizes only, no layout;
+    """Pack [N, K] codes into int32 [N, K/8], eight codes per word in the
+    nibble order PACK_ORDER.  The pages give storage sizes only, no layout;
     this is the library's canonical layout."""
     c = np.asarray(codes, dtype=np.uint32)
     n, k = c.shape
     c = c.reshape(n, k // 8, 8)
     word = np.zeros((n, k // 8), dtype=np.uint32)
-    for j in range(8):
-        word |= c[:, :, j] << np.uint32(4 * j)
+    for i, j in enumerate(PACK_ORDER):
+        word |= c[:, :, j] << np.uint32(4 * i)
     return word.view(np.int32)
 
 
@@ -191,8 +197,8 @@ def unpack_codes(qweight: np.ndarray) -> np.ndarray:
     w = np.asarray(qweight).view(np.uint32)
     n, kw = w.shape
     out = np.empty((n, kw, 8), dtype=np.uint8)
-    for j in range(8):
-        out[:, :, j] = (w >> np.uint32(4 * j)) & np.uint32(0xF)
+    for i, j in enumerate(PACK_ORDER):
+        out[:, :, j] = (w >> np.uint32(4 * i)) & np.uint32(0xF)
     return out.reshape(n, kw * 8)
 
 

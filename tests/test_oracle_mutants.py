@@ -23,8 +23,8 @@ MUTANTS = [
     ("AWQ s applied the wrong way", "return w - w_hat / np.asarray(s", "return w - w_hat * np.asarray(s"),
     ("AWQ s not applied before quantization",
      "v = w if awq_s is None else w * np.asarray(awq_s, dtype=np.float32)[None, :]", "v = w"),
-    ("nibble order reversed", "word |= c[:, :, j] << np.uint32(4 * j)",
-     "word |= c[:, :, j] << np.uint32(4 * (7 - j))"),
+    ("linear nibble order", "word |= c[:, :, j] << np.uint32(4 * i)",
+     "word |= c[:, :, i] << np.uint32(4 * i)"),
     ("fp16 ties away", "up = (rem > half) | ((rem == half) & ((q & np.uint64(1)) == 1))",
      "up = rem >= half"),
     ("fp16 truncation", "up = (rem > half) | ((rem == half) & ((q & np.uint64(1)) == 1))",

@@ -108,10 +108,18 @@ def test_pack_layout_little_endian_nibbles():
     codes = np.zeros((2, 128), np.uint8)
     codes[0, :8] = [1, 2, 3, 4, 5, 6, 7, 8]
     codes[1, 8:16] = [15, 0, 0, 0, 0, 0, 0, 9]
+    # (channel 8 in nibble 0, channel 15 in nibble 7)
     q = O.pack_codes(codes).view(np.uint32)
     assert q.shape == (2, 16)
-    assert q[0, 0] == 0x87654321 and q[0, 1] == 0
+    # nibbles low->high hold channels 0,2,4,6,1,3,5,7 of the word
+    assert q[0, 0] == 0x86427531 and q[0, 1] == 0
     assert q[1, 1] == 0x9000000F
+    # nibble pair (i, i+4) masked with 0x000F000F gives channels (2i, 2i+1)
+    codes[0, 16:24] = [1, 2, 3, 4, 5, 6, 7, 8]
+    w = int(O.pack_codes(codes).view(np.uint32)[0, 2])
+    for i in range(4):
+        pair = (w >> (4 * i)) & 0x000F000F
+        assert (pair & 0xF, pair >> 16) == (2 * i + 1, 2 * i + 2)
     rng = np.random.default_rng(1)
     c = rng.integers(0, 16, size=(5, 256), dtype=np.uint8)
     assert np.array_equal(O.unpack_codes(O.pack_codes(c)), c)
