@@ -1,0 +1,223 @@
+/*
+ * w4.h -- C ABI of libw4: weight-only int4 group-128 quantization, the W4A16
+ * linear that consumes it, and AWQ alpha/shrink candidate scoring, as
+ * hand-written CUDA kernels for B200 (sm_100a).
+ *
+ * Sources (model-card pages, cited by title and section):
+ *   [rebuttal] "ghostchoir/rebuttal_w4g128_awq_w2": 'Model Details' table
+ *              rows 'Scheme' (weight-only, 4-bit, group size 128, asymmetric
+ *              zero point) and 'Search' (AWQ scale exponent on a 20-point
+ *              grid, clipping as a 10-point global shrink grid); the
+ *              scale-rewrite paragraph (prev_op /= s, W *= s equals
+ *              Q(W diag(s)) diag(1/s)); 'Clipping granularity' (one shrink
+ *              ratio per linear); the table note defining RTN.
+ *   [qwen27b]  "GotoAI-Inc/Qwen3.6-27B-W4A16": opening paragraph (int4, group
+ *              size 128, symmetric, weight-only, activations stay 16-bit).
+ *   [awq-ppl]  "AWQ INT4-g128 WikiText-2 perplexity delta vs fp16, Llama-2
+ *              7B": 'Methodology' (grid size 20 for the alpha search).
+ *   [qsrt]     "malaiwah/GLM-5.2-QSRT-Fruit-Instruct": 'Reproducible runtime'
+ *              (decode-sized batches of at most 16 rows take a separate
+ *              path from prefill).
+ *
+ * Conventions shared by every entry point
+ *   - Device pointers are caller-owned device memory (any allocator).  Host
+ *     pointers are marked "host".  The library never allocates or frees
+ *     memory and keeps no state between calls apart from one device-side
+ *     error word (see w4_device_error).
+ *   - `stream` is a cudaStream_t passed as void*; NULL is the legacy default
+ *     stream.  Launches are asynchronous; outputs are valid once the stream
+ *     has been synchronized.
+ *   - Arguments are validated on the host before anything is launched.  A
+ *     call that returns anything but W4_OK has launched nothing.
+ *   - Every device base pointer must be 16-byte aligned.
+ *   - bf16 / fp16 buffers are passed as raw 16-bit patterns (void* /
+ *     uint16_t*).  Inputs must be finite.
+ *   - No C++ exception crosses the ABI; CUDA failures return W4_ERR_CUDA.
+ *
+ * Packed weight format (canonical; the pages give storage sizes only)
+ *   qweight : int32 [N, K/8].  Word w of row n holds the eight 4-bit codes of
+ *             input channels 8w..8w+7; nibble i (bits 4i..4i+3) holds channel
+ *             8w + {0,2,4,6,1,3,5,7}[i], so nibbles (i, i+4) are the adjacent
+ *             channels (2i, 2i+1).
+ *   scales  : fp16 bits [N, K/128], row-major.
+ *   zeros   : fp16 bits [N, K/128] holding integers 0..15 (asymmetric), or
+ *             absent (symmetric: implicit zero 8).
+ *   Dequantization: w_hat[n,k] = (q[n,k] - zero[n,k/128]) * scale[n,k/128].
+ *   Storage: 0.53125 byte/weight asymmetric, 0.515625 symmetric.
+ */
+#ifndef W4_H
+#define W4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  W4_OK = 0,
+  W4_ERR_INVALID_ARG = 1,    /* NULL pointer where one is required, bad flag */
+  W4_ERR_SHAPE = 2,          /* non-positive size, K not a multiple of 128, ... */
+  W4_ERR_ALIGNMENT = 3,      /* a device pointer not 16-byte aligned */
+  W4_ERR_UNSUPPORTED = 4,    /* group != 128, grid larger than supported, ... */
+  W4_ERR_WORKSPACE = 5,      /* workspace missing or smaller than required */
+  W4_ERR_CUDA = 6,           /* a CUDA runtime call failed (launch, attribute, ...) */
+  W4_ERR_DEVICE_TIMEOUT = 7  /* a kernel gave up on a bounded wait (w4_device_error) */
+} w4_status;
+
+/* Static, NUL-terminated description of a status code. */
+const char* w4_status_string(w4_status status);
+
+/* ABI version of this header (bumped on any incompatible change). */
+#define W4_ABI_VERSION 1
+int w4_abi_version(void);
+
+/*
+ * w4_quantize_pack -- round-to-nearest int4 group-128 quantization and
+ * packing of one linear's weight ([rebuttal] 'Scheme'; [qwen27b]).
+ *
+ * w_bf16    device, bf16 [N, K] row-major (K contiguous): the weight W.
+ * N, K      output and input features; N >= 1, K >= 128, K % 128 == 0.
+ * group     must be 128.
+ * symmetric 0: asymmetric with zero point; 1: symmetric.
+ * awq_s     device, float32 [K], or NULL.  When given, the weight quantized
+ *           is v = W * diag(s) (per input channel, binary32 multiply),
+ *           i.e. the Q(W diag(s)) of [rebuttal]'s scale-rewrite paragraph.
+ *           The caller folds 1/s into the op that produces x.
+ * shrink    clipping shrink ratio r in (0, 1] ([rebuttal] 'Clipping
+ *           granularity'); 1.0 is no clipping.
+ * qweight   device, int32 [N, K/8] out.
+ * scales_f16 device, fp16 bits [N, K/128] out.
+ * zeros_f16 device, fp16 bits [N, K/128] out; must be NULL iff symmetric.
+ *
+ * Per group G of 128 consecutive channels of one row, in IEEE binary32 with
+ * round-to-nearest-even and no fused multiply-add:
+ *   asymmetric: mx = r*max v, mn = r*min v,
+ *               scale = fp16_rn(max(mx - mn, 1e-5) / 15),
+ *               zero  = clamp(rint(-mn / scale), 0, 15);
+ *   symmetric:  scale = fp16_rn(max(r*max|v|, 1e-5) / 7), zero = 8;
+ *   code = clamp(rint(v / scale) + zero, 0, 15)   (scale = the stored fp16
+ *          value, rint ties to even, v/scale correctly rounded).
+ * Bit-exact with the CPU oracle.  Returns W4_OK or a validation / CUDA error.
+ */
+w4_status w4_quantize_pack(const void* w_bf16, int64_t N, int64_t K, int group,
+                           int symmetric, const float* awq_s, float shrink,
+                           int32_t* qweight, uint16_t* scales_f16, uint16_t* zeros_f16,
+                           void* stream);
+
+/*
+ * w4a16_linear -- y = x . dequant(Wq)^T with bf16 activations and a bf16
+ * result ([qwen27b]: activations stay 16-bit; [qsrt] 'Reproducible runtime':
+ * decode-sized row counts take their own path).  No bias.
+ *
+ * x_bf16    device, bf16 [M, K] row-major.
+ * M         token rows, 1 <= M <= 2^31-1.
+ * qweight, scales_f16, zeros_f16  the packed weight (zeros NULL: symmetric).
+ * N, K      as for w4_quantize_pack.
+ * group     must be 128.
+ * y_bf16    device, bf16 [M, N] row-major out (accumulated in binary32,
+ *           rounded once to bf16).
+ * flags     bitwise OR of W4_LINEAR_* below (0 for defaults).
+ *
+ * M <= 16 runs the decode GEMV (tensor-core mma over register-dequantized
+ * weight fragments, HBM-bound); larger M runs the prefill GEMM (tcgen05 with
+ * TMEM accumulators, weight tiles dequantized into shared memory).
+ */
+#define W4_LINEAR_FORCE_GEMV 0x1u  /* decode kernel at any M <= 64 */
+#define W4_LINEAR_FORCE_GEMM 0x2u  /* prefill kernel at any M */
+#define W4_LINEAR_PDL 0x4u         /* programmatic dependent launch: the
+                                      kernel may start before the previous
+                                      kernel on the stream ends and waits for
+                                      it before touching global memory */
+#define W4_LINEAR_STATIC_WEIGHTS 0x8u /* with W4_LINEAR_PDL: the caller
+                                      guarantees qweight/scales/zeros are not
+                                      written by preceding work still in
+                                      flight, so the kernel may start streaming
+                                      them before the dependency wait */
+w4_status w4a16_linear(const void* x_bf16, int64_t M, const int32_t* qweight,
+                       const uint16_t* scales_f16, const uint16_t* zeros_f16,
+                       int64_t N, int64_t K, int group, void* y_bf16,
+                       unsigned flags, void* stream);
+
+/*
+ * w4_awq_scales -- AWQ per-input-channel scales ([rebuttal] 'Search': AWQ
+ * scale exponent grid; [awq-ppl] 'Methodology': grid of 20 alphas).
+ *
+ *   stat_j = (sum_m |x_mj|) / M   (binary64, fixed summation order m = 0..M-1)
+ *   s[i, j] = (float) pow(max(stat_j, 1e-8), alpha_i)   (binary64 pow)
+ *
+ * x_bf16   device, bf16 [M, K];  M >= 1, K >= 1.
+ * alphas   host, float32 [n_alpha], 1 <= n_alpha <= 64.
+ * s_out    device, float32 [n_alpha, K] out.
+ */
+w4_status w4_awq_scales(const void* x_bf16, int64_t M, int64_t K, const float* alphas,
+                        int n_alpha, float* s_out, void* stream);
+
+/*
+ * awq_score_grid -- batched AWQ candidate scoring over the alpha x shrink
+ * grid ([rebuttal] 'Search' and the scale-rewrite paragraph: a candidate is
+ * simulated by swapping only the linear's weight for
+ * Q(W diag(s)) diag(1/s)).  For every (alpha_i, shrink_j):
+ *
+ *   s = w4_awq_scales(x, alpha_i),  What = dequant(Q_r(W diag(s))) diag(1/s),
+ *   SSE[seg, i, j] = || x . (W - What)^T ||_F^2 over the rows of W in seg.
+ *
+ * The candidate's codes are bit-identical to w4_quantize_pack(W, s, shrink).
+ * The error product runs on tcgen05 tensor cores in fp16 in the s-domain,
+ * (x/s) . (W s - w_hat)^T, accumulated in binary32 and squared and summed in
+ * binary64; requires |x/s| < 65504.
+ *
+ * x_bf16       device, bf16 [M, K] calibration activations.
+ * w_bf16       device, bf16 [N, K] weight of one linear, or of several
+ *              linears that share x concatenated along N (q,k,v; gate,up).
+ * group        must be 128;  symmetric as for w4_quantize_pack.
+ * alphas       host, float32 [n_alpha], 1 <= n_alpha <= 64.
+ * shrinks      host, float32 [n_shrink], 1 <= n_shrink <= 64, each in (0,1].
+ * seg_offsets  host, int64 [n_seg + 1] with 0 = off[0] < ... < off[n_seg] = N,
+ *              interior offsets multiples of 16; or NULL with n_seg = 1.
+ * n_seg        1..16 linears sharing x.
+ * sse_out      device, float64 [n_seg, n_alpha, n_shrink] out.
+ * argmin_out   device, int32 [n_seg + 1, 4] out.  Row s < n_seg:
+ *              {joint flat argmin (alpha-major), alpha* at shrink 1.0,
+ *               shrink* at that alpha*, shrink* at the group's alpha*};
+ *              row n_seg: {joint argmin of the summed table, the group's
+ *              alpha* (summed table at shrink 1.0), -1, -1}.  "Shrink 1.0" is
+ *              the first shrink equal to 1.0f, else column 0.  Equal minima
+ *              resolve to the lowest index.
+ * workspace    device scratch of at least w4_awq_workspace_bytes(...) bytes,
+ *              256-byte aligned; contents on entry are ignored.
+ */
+size_t w4_awq_workspace_bytes(int64_t M, int64_t N, int64_t K, int n_alpha, int n_shrink,
+                              int n_seg);
+w4_status awq_score_grid(const void* x_bf16, int64_t M, const void* w_bf16, int64_t N,
+                         int64_t K, int group, int symmetric, const float* alphas,
+                         int n_alpha, const float* shrinks, int n_shrink,
+                         const int64_t* seg_offsets, int n_seg, double* sse_out,
+                         int32_t* argmin_out, void* workspace, size_t workspace_bytes,
+                         void* stream);
+
+/*
+ * w4_device_error -- reads (and with clear != 0 resets) the library's device
+ * error word.  Every wait inside the tcgen05 kernels is bounded (about one
+ * second); a kernel that gives up records it here and returns early, leaving
+ * its outputs undefined but the CUDA context usable.  Synchronize the streams
+ * that ran library kernels first.  Returns W4_OK, W4_ERR_DEVICE_TIMEOUT or
+ * W4_ERR_CUDA; *code_out (may be NULL) receives the raw word (0 = none).
+ */
+w4_status w4_device_error(int clear, uint32_t* code_out);
+
+/*
+ * w4_selftest_bounded_wait -- launches one CTA that waits on a shared-memory
+ * barrier nobody arrives at, with the given limit in nanoseconds
+ * (1e6..2e9), then gives up, records the timeout in the device error word and
+ * returns.  Exercises the failure path of the bounded waits without faulting
+ * or hanging the GPU.
+ */
+w4_status w4_selftest_bounded_wait(uint64_t limit_ns, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* W4_H */

@@ -1,0 +1,98 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports
+every function include/w4.h declares, and rejects bad arguments with the
+documented status codes before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import weight_only_int4_quantize_b200 as w4
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "w4.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    if not os.path.exists(w4.LIB_PATH):
+        from weight_only_int4_quantize_b200 import build
+        build.build()
+    return w4.lib()
+
+
+def _declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\**\s+\**(\w+)\s*\(", src, flags=re.M)))
+
+
+def test_exports_every_declared_function(L):
+    names = _declared_functions()
+    assert {"w4_quantize_pack", "w4a16_linear", "awq_score_grid", "w4_awq_scales",
+            "w4_awq_workspace_bytes", "w4_status_string", "w4_device_error"} <= set(names)
+    for n in names:
+        assert hasattr(L, n), f"libw4.so does not export {n}"
+
+
+def test_status_strings_and_version(L):
+    for code in range(8):
+        assert L.w4_status_string(code)
+    assert L.w4_abi_version() == 1
+
+
+A = 0x10000  # an aligned fake device address: validation runs before any device call
+B = 0x20000
+
+
+def test_quantize_validation(L):
+    q = L.w4_quantize_pack
+    assert q(None, 4, 128, 128, 0, None, 1.0, A, A, A, None) == 1       # NULL weight
+    assert q(A, 4, 128, 128, 0, None, 1.0, A, A, None, None) == 1       # asym needs zeros
+    assert q(A, 4, 128, 128, 1, None, 1.0, A, A, A, None) == 1          # sym forbids zeros
+    assert q(A, 4, 128, 128, 0, None, 0.0, A, A, A, None) == 1          # shrink out of range
+    assert q(A, 4, 128, 128, 0, None, 1.5, A, A, A, None) == 1
+    assert q(A, 4, 128, 64, 0, None, 1.0, A, A, A, None) == 4           # group != 128
+    assert q(A, 4, 100, 128, 0, None, 1.0, A, A, A, None) == 2          # K % 128
+    assert q(A, 0, 128, 128, 0, None, 1.0, A, A, A, None) == 2          # N < 1
+    assert q(A + 2, 4, 128, 128, 0, None, 1.0, A, A, A, None) == 3      # misaligned
+    assert q(A, 4, 128, 128, 0, A + 4, 1.0, A, A, A, None) == 3         # misaligned s
+
+
+def test_linear_validation(L):
+    f = L.w4a16_linear
+    assert f(None, 1, A, A, None, 8, 128, 128, B, 0, None) == 1
+    assert f(A, 1, A, A, None, 8, 128, 128, B, 0x100, None) == 1        # unknown flag
+    assert f(A, 1, A, A, None, 8, 128, 128, B, 0x3, None) == 1          # both forced paths
+    assert f(A, 0, A, A, None, 8, 128, 128, B, 0, None) == 2
+    assert f(A, 1, A, A, None, 8, 130, 128, B, 0, None) == 2
+    assert f(A, 1, A, A, None, 8, 128, 32, B, 0, None) == 4
+    assert f(A, 100, A, A, None, 8, 128, 128, B, 0x1, None) == 4        # GEMV beyond 64 rows
+    assert f(A, 1, A, A, None, 8, 128, 128, B + 8, 0, None) == 3
+
+
+def test_awq_validation(L):
+    f = L.awq_score_grid
+    al = (ctypes.c_float * 2)(0.0, 0.5)
+    sh = (ctypes.c_float * 2)(1.0, 0.9)
+    bad_sh = (ctypes.c_float * 2)(1.0, 1.2)
+    seg_bad = (ctypes.c_int64 * 3)(0, 100, 256)   # interior offset not a multiple of 16
+    seg_ok = (ctypes.c_int64 * 3)(0, 128, 256)
+    need = L.w4_awq_workspace_bytes(64, 256, 256, 2, 2, 2)
+    assert need > 0
+    base = (A, 64, B, 256, 256, 128, 0, al, 2, sh, 2)
+    assert f(*base, None, 1, A, A, A, need, None) != 5  # reaches the device (no GPU here) or OK
+    assert f(*base, seg_bad, 2, A, A, A, need, None) == 2
+    assert f(*base, None, 2, A, A, A, need, None) == 1            # n_seg > 1 needs offsets
+    assert f(*base, seg_ok, 2, A, A, A, 16, None) == 5            # workspace too small
+    assert f(*base, seg_ok, 2, A, A, A + 16, need, None) == 3     # workspace not 256-aligned
+    assert f(A, 64, B, 256, 256, 128, 0, al, 2, bad_sh, 2, None, 1, A, A, A, need, None) == 1
+    assert f(A, 64, B, 256, 256, 128, 0, al, 0, sh, 2, None, 1, A, A, A, need, None) == 4
+    assert L.w4_selftest_bounded_wait(10, None) == 1              # limit below 1 ms
+
+
+def test_binding_fails_loudly_without_library(monkeypatch):
+    monkeypatch.setattr(w4, "_LIB", None)
+    monkeypatch.setattr(w4, "LIB_PATH", "/nonexistent/libw4.so")
+    with pytest.raises(RuntimeError, match="no CPU fallback"):
+        w4.lib()

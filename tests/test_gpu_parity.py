@@ -1,0 +1,273 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle on
+identical seeded inputs.
+
+Bars (written here, checked element by element):
+  * quantize + pack: codes, fp16 scales and fp16 zeros bit-exact;
+  * AWQ scales s: bit-exact;
+  * linear: max|y_gpu - y_ref| / max|y_ref| <= 5e-3 against the binary64
+    oracle over the identical dequantized weights;
+  * AWQ scoring: SSE within SSE_RTOL relative, argmins identical unless the
+    oracle's own values are within ARGMIN_TIE_RTOL of each other (a near tie:
+    then any index of the tied set is correct and the test says so).
+"""
+import numpy as np
+import pytest
+import torch
+
+import weight_only_int4_quantize_b200 as w4
+from oracle import w4_oracle as O
+from weight_only_int4_quantize_b200 import synth
+
+pytestmark = [pytest.mark.gpu,
+              pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA GPU")]
+
+DEV = "cuda:0"
+Y_RTOL = 5e-3           # linear: max-normalized error bound
+SSE_RTOL = 2e-4         # AWQ: fp16 tensor-core operands, binary64 sums
+ARGMIN_TIE_RTOL = 2e-5  # oracle values closer than this count as tied
+
+
+def u16(t):
+    return t.cpu().numpy().view(np.uint16)
+
+
+def quantize_both(w_cpu, sym, s=None, r=1.0):
+    s_dev = None if s is None else torch.from_numpy(np.ascontiguousarray(s)).to(DEV)
+    qw, sc, zr = w4.quantize_pack(w_cpu.to(DEV), sym, s_dev, r)
+    torch.cuda.synchronize()
+    ref = O.quantize_pack(synth.bits(w_cpu), sym, s, r)
+    return (qw, sc, zr), ref
+
+
+def assert_quant_equal(gpu, ref, sym):
+    qw, sc, zr = gpu
+    oq, os_, oz = ref
+    assert np.array_equal(qw.cpu().numpy(), oq), "packed codes differ"
+    assert np.array_equal(u16(sc), os_), "scales differ"
+    if sym:
+        assert zr is None and oz is None
+    else:
+        assert np.array_equal(u16(zr), oz), "zeros differ"
+
+
+def max_rel_err(y_gpu, y_ref):
+    y = y_gpu.float().cpu().numpy().astype(np.float64)
+    return float(np.max(np.abs(y - y_ref)) / np.max(np.abs(y_ref)))
+
+
+# ------------------------------------------------------------ quantize ----
+
+@pytest.mark.parametrize("sym", [False, True])
+def test_quantize_single_linear_2048_outliers(sym):
+    w = synth.normal_weight(2048, 2048, 0.02, seed=0, n_outliers=8, outlier_scale=20.0)
+    gpu, ref = quantize_both(w, sym)
+    assert_quant_equal(gpu, ref, sym)
+
+
+@pytest.mark.parametrize("n,k", [(1, 128), (3, 384), (17, 256), (1000, 1152), (6144, 2048)])
+@pytest.mark.parametrize("sym", [False, True])
+@pytest.mark.parametrize("r", [1.0, 0.7])
+def test_quantize_shapes_shrink(n, k, sym, r):
+    w = synth.normal_weight(n, k, 0.02, seed=n * 7 + k, n_outliers=min(8, k // 16),
+                            outlier_scale=20.0)
+    gpu, ref = quantize_both(w, sym, None, r)
+    assert_quant_equal(gpu, ref, sym)
+
+
+@pytest.mark.parametrize("sym", [False, True])
+@pytest.mark.parametrize("alpha", [0.0, 0.5, 0.95])
+def test_quantize_with_awq_scale(sym, alpha):
+    x = synth.student_t_calibration(256, 2048, seed=5)
+    w = synth.normal_weight(1024, 2048, 0.02, seed=6)
+    s = O.awq_scales(O.awq_channel_stat(synth.bits(x)), [alpha])[0]
+    gpu, ref = quantize_both(w, sym, s, 0.85)
+    assert_quant_equal(gpu, ref, sym)
+    if alpha == 0.0:  # s == 1 reduces to plain RTN, byte for byte
+        plain, _ = quantize_both(w, sym, None, 0.85)
+        for a, b in zip(gpu, plain):
+            assert (a is None and b is None) or torch.equal(a, b)
+
+
+def test_quantize_shrink_one_is_no_clip():
+    w = synth.normal_weight(512, 1024, 0.02, seed=8, n_outliers=8, outlier_scale=20.0)
+    for sym in (False, True):
+        a, _ = quantize_both(w, sym, None, 1.0)
+        s1 = np.ones(1024, np.float32)
+        b, _ = quantize_both(w, sym, s1, 1.0)
+        for p, q in zip(a, b):
+            assert (p is None and q is None) or torch.equal(p, q)
+
+
+def _near_tie_inputs(sym, groups=64, rows=8, seed=3):
+    """Weights and per-channel scales whose products v = w*s put v/scale
+    within a few ulp of a half-integer tie (exactly on it, just above and
+    just below), so the division-free rounding path must defer to the exact
+    division.  w is a power of two per row, so v*2^j keeps the quotients."""
+    rng = np.random.default_rng(seed)
+    k = 128 * groups
+    s = np.empty(k, np.float32)
+    for g in range(groups):
+        # a random fp16 scale with a full mantissa
+        sc = np.float32(np.float16(rng.uniform(0.01, 0.1)))
+        base = g * 128
+        if sym:
+            s[base] = np.float32(7) * sc        # absmax -> scale = sc exactly
+            m = rng.integers(-7, 7, 127)  # |m + 1/2| < 7 keeps absmax = 7 * scale
+        else:
+            s[base] = np.float32(0.0)            # min 0 -> zero 0
+            s[base + 1] = np.float32(15) * sc    # max -> scale = sc exactly
+            m = rng.integers(0, 15, 127)
+        for i, mm in enumerate(m):
+            j = base + 1 + i + (0 if sym else 1)
+            if j >= base + 128:
+                break
+            t = np.float32((mm + 0.5) * np.float64(sc))
+            u = t.view(np.uint32) + np.uint32(rng.integers(-3, 4) & 0xFFFFFFFF)
+            s[j] = u.view(np.float32) if t != 0 else t
+    rowscale = (2.0 ** (np.arange(rows) % 5 - 2)).astype(np.float32)
+    w = torch.from_numpy(np.repeat(rowscale[:, None], k, axis=1)).to(torch.bfloat16)
+    return w, s
+
+
+@pytest.mark.parametrize("sym", [False, True])
+def test_quantize_near_ties_exact(sym):
+    w, s = _near_tie_inputs(sym)
+    gpu, ref = quantize_both(w, sym, s, 1.0)
+    assert_quant_equal(gpu, ref, sym)
+
+
+# -------------------------------------------------------------- linear ----
+
+def linear_case(m, n, k, sym, seed, flags=0, std=0.02, n_out=0, out_scale=1.0, rows=None):
+    w = synth.normal_weight(n, k, std, seed=seed, n_outliers=n_out, outlier_scale=out_scale)
+    x = synth.normal_activations(m, k, seed=seed + 1)
+    qw, sc, zr = w4.quantize_pack(w.to(DEV), sym)
+    y = w4.w4a16_linear(x.to(DEV), qw, sc, zr, flags=flags)
+    torch.cuda.synchronize()
+    codes = O.unpack_codes(qw.cpu().numpy())
+    # the oracle dequantizes its OWN quantization (bit-equality is tested above)
+    oc, os_, oz = O.quantize_rtn(synth.bits(w), sym)
+    assert np.array_equal(codes, oc)
+    what = O.dequantize(oc, os_, oz)
+    xb = synth.bits(x)
+    if rows is None:
+        y_ref = O.linear(xb, what)
+        return max_rel_err(y, y_ref)
+    y_ref = O.linear_rows(xb, what, rows)
+    return max_rel_err(y[torch.as_tensor(rows, device=DEV)], y_ref)
+
+
+@pytest.mark.parametrize("m", [1, 2, 3, 5, 8, 9, 15, 16])
+@pytest.mark.parametrize("sym", [False, True])
+def test_gemv_parity_ragged(m, sym):
+    assert linear_case(m, 1000, 1024, sym, seed=100 + m) <= Y_RTOL
+
+
+@pytest.mark.parametrize("m", [1, 16])
+def test_gemv_single_linear_2048_outliers(m):
+    assert linear_case(m, 2048, 2048, False, seed=0, n_out=8, out_scale=20.0) <= Y_RTOL
+
+
+@pytest.mark.parametrize("m", [17, 40, 64])
+def test_gemv_forced_chunks(m):
+    assert linear_case(m, 520, 640, False, seed=200 + m, flags=w4.LINEAR_FORCE_GEMV) <= Y_RTOL
+
+
+@pytest.mark.parametrize("m,n,k", [(1, 256, 128), (17, 256, 256), (64, 1000, 640), (128, 256, 4096),
+                                   (200, 520, 1024), (300, 4096, 512)])
+@pytest.mark.parametrize("sym", [False, True])
+def test_gemm_parity_ragged(m, n, k, sym):
+    assert linear_case(m, n, k, sym, seed=300 + m + n, flags=w4.LINEAR_FORCE_GEMM) <= Y_RTOL
+
+
+@pytest.mark.parametrize("k,n", [(4096, 4096), (4096, 11008), (11008, 4096)])
+@pytest.mark.parametrize("m", [512, 2048])
+def test_gemm_llama2_7b_shapes(k, n, m):
+    rows = None if m == 512 else np.sort(np.random.default_rng(m + n).choice(m, 256, replace=False))
+    assert linear_case(m, n, k, True, seed=400 + n, rows=rows) <= Y_RTOL
+
+
+@pytest.mark.parametrize("k,n", [(5120, 17408), (17408, 5120), (5120, 10240)])
+@pytest.mark.parametrize("m", [1, 8, 64, 512, 4096])
+def test_linear_27b_shapes(k, n, m):
+    rows = None if m <= 512 else np.sort(np.random.default_rng(m + n).choice(m, 128, replace=False))
+    err = linear_case(m, n, k, True, seed=500 + n, std=0.015, n_out=k // 100, out_scale=10.0,
+                      rows=rows)
+    assert err <= Y_RTOL
+
+
+# ----------------------------------------------------------------- AWQ ----
+
+def test_awq_scales_bit_exact():
+    x = synth.student_t_calibration(2048, 2048, seed=11)
+    alphas = synth.alpha_grid(20)
+    s = w4.awq_scales(x.to(DEV), alphas)
+    torch.cuda.synchronize()
+    ref = O.awq_scales(O.awq_channel_stat(synth.bits(x)), alphas)
+    assert np.array_equal(s.cpu().numpy().view(np.uint32), ref.view(np.uint32))
+
+
+def _within_band(idx, values, what):
+    v = np.asarray(values, dtype=np.float64).ravel()
+    band = np.flatnonzero(v <= v.min() * (1.0 + ARGMIN_TIE_RTOL))
+    assert idx in band, f"{what}: GPU picked {idx}, oracle band {band.tolist()}"
+    if len(band) > 1:
+        print(f"near tie in {what}: {band.tolist()} (gap {O.relative_gap(v):.2e})")
+    return len(band) == 1
+
+
+def check_awq(x, w, alphas, shrinks, sym, seg=None):
+    sse, arg = w4.awq_score_grid(x.to(DEV), w.to(DEV), alphas, shrinks, sym, seg_offsets=seg)
+    torch.cuda.synchronize()
+    sse = sse.cpu().numpy()
+    arg = arg.cpu().numpy()
+    ref, ref_arg = O.awq_score_grid(synth.bits(x), synth.bits(w), alphas, shrinks, sym, seg)
+    rel = np.max(np.abs(sse - ref) / ref)
+    assert rel <= SSE_RTOL, f"SSE relative error {rel:.3e}"
+    c1 = O.no_clip_column(shrinks)
+    n_seg = ref.shape[0]
+    total = ref.sum(axis=0)
+    for s_ in range(n_seg):
+        t = ref[s_]
+        _within_band(arg[s_, 0], t, f"seg {s_} joint")
+        _within_band(arg[s_, 1], t[:, c1], f"seg {s_} alpha*")
+        _within_band(arg[s_, 2], t[arg[s_, 1]], f"seg {s_} shrink*")
+        _within_band(arg[s_, 3], t[arg[n_seg, 1]], f"seg {s_} shrink* at group alpha")
+    _within_band(arg[n_seg, 0], total, "group joint")
+    _within_band(arg[n_seg, 1], total[:, c1], "group alpha*")
+    assert arg[n_seg, 2] == -1 and arg[n_seg, 3] == -1
+    return rel, ref_arg, arg
+
+
+@pytest.mark.parametrize("sym", [False, True])
+def test_awq_grid_small_full_grid(sym):
+    x = synth.student_t_calibration(256, 512, seed=21)
+    w = synth.normal_weight(384, 512, 0.02, seed=22, n_outliers=4, outlier_scale=20.0)
+    check_awq(x, w, synth.alpha_grid(20), synth.shrink_grid(10), sym)
+
+
+def test_awq_grid_segments_ragged_tokens():
+    x = synth.student_t_calibration(200, 640, seed=31)   # M not a multiple of 128
+    w = synth.normal_weight(800, 640, 0.02, seed=32)      # three linears sharing x
+    check_awq(x, w, synth.alpha_grid(8), synth.shrink_grid(4), False, seg=[0, 256, 528, 800])
+
+
+def test_awq_grid_qwen_k_proj_full_size():
+    """One Qwen3-1.7B k_proj (2048 -> 1024) on 2048 heavy-tailed calibration
+    tokens, the full 20 x 10 grid."""
+    x = synth.student_t_calibration(2048, 2048, seed=41)
+    w = synth.normal_weight(1024, 2048, 0.02, seed=42)
+    check_awq(x, w, synth.alpha_grid(20), synth.shrink_grid(10), False)
+
+
+# ------------------------------------------------------ failure path ----
+
+def test_bounded_wait_reports_and_context_survives():
+    w4.device_error(clear=True)
+    w4.selftest_bounded_wait(20_000_000)  # 20 ms
+    torch.cuda.synchronize()
+    code = w4.device_error(clear=True)
+    assert code & 1 and (code >> 16) == 7
+    assert w4.device_error(clear=True) == 0
+    # the context is still usable
+    assert linear_case(4, 256, 256, False, seed=9) <= Y_RTOL

@@ -1,0 +1,226 @@
+"""weight_only_int4_quantize_b200: int4 group-128 weight-only quantization, the
+W4A16 linear and AWQ candidate scoring on B200 (sm_100a).
+
+This module is a thin ctypes binding over the C ABI of ``libw4.so``
+(include/w4.h): it checks tensor devices and dtypes, allocates outputs with
+torch and passes raw pointers and the current CUDA stream.  Every step of the
+computation runs in the library's CUDA kernels; there is no CPU fallback, and
+any call fails loudly if the library has not been built
+(``python -m weight_only_int4_quantize_b200.build``).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+__all__ = [
+    "W4Error", "lib", "quantize_pack", "w4a16_linear", "awq_scales", "awq_score_grid",
+    "awq_workspace_bytes", "device_error", "selftest_bounded_wait",
+    "LINEAR_FORCE_GEMV", "LINEAR_FORCE_GEMM", "LINEAR_PDL", "LINEAR_STATIC_WEIGHTS",
+]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libw4.so")
+
+LINEAR_FORCE_GEMV = 0x1
+LINEAR_FORCE_GEMM = 0x2
+LINEAR_PDL = 0x4
+LINEAR_STATIC_WEIGHTS = 0x8
+
+_STATUS = {
+    0: "W4_OK", 1: "W4_ERR_INVALID_ARG", 2: "W4_ERR_SHAPE", 3: "W4_ERR_ALIGNMENT",
+    4: "W4_ERR_UNSUPPORTED", 5: "W4_ERR_WORKSPACE", 6: "W4_ERR_CUDA", 7: "W4_ERR_DEVICE_TIMEOUT",
+}
+
+
+class W4Error(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        self.name = _STATUS.get(status, str(status))
+        msg = lib().w4_status_string(status).decode() if _LIB is not None else self.name
+        super().__init__(f"{where}: {self.name} ({msg})")
+
+
+_LIB: Optional[ctypes.CDLL] = None
+
+_c = ctypes
+_p = ctypes.c_void_p
+_i64 = ctypes.c_int64
+
+
+def _declare(L: ctypes.CDLL) -> None:
+    L.w4_status_string.restype = ctypes.c_char_p
+    L.w4_status_string.argtypes = [ctypes.c_int]
+    L.w4_abi_version.restype = ctypes.c_int
+    L.w4_abi_version.argtypes = []
+    L.w4_quantize_pack.restype = ctypes.c_int
+    L.w4_quantize_pack.argtypes = [_p, _i64, _i64, ctypes.c_int, ctypes.c_int, _p, ctypes.c_float,
+                                   _p, _p, _p, _p]
+    L.w4a16_linear.restype = ctypes.c_int
+    L.w4a16_linear.argtypes = [_p, _i64, _p, _p, _p, _i64, _i64, ctypes.c_int, _p,
+                               ctypes.c_uint, _p]
+    L.w4_awq_scales.restype = ctypes.c_int
+    L.w4_awq_scales.argtypes = [_p, _i64, _i64, _p, ctypes.c_int, _p, _p]
+    L.w4_awq_workspace_bytes.restype = ctypes.c_size_t
+    L.w4_awq_workspace_bytes.argtypes = [_i64, _i64, _i64, ctypes.c_int, ctypes.c_int,
+                                         ctypes.c_int]
+    L.awq_score_grid.restype = ctypes.c_int
+    L.awq_score_grid.argtypes = [_p, _i64, _p, _i64, _i64, ctypes.c_int, ctypes.c_int, _p,
+                                 ctypes.c_int, _p, ctypes.c_int, _p, ctypes.c_int, _p, _p, _p,
+                                 ctypes.c_size_t, _p]
+    L.w4_device_error.restype = ctypes.c_int
+    L.w4_device_error.argtypes = [ctypes.c_int, _p]
+    L.w4_selftest_bounded_wait.restype = ctypes.c_int
+    L.w4_selftest_bounded_wait.argtypes = [ctypes.c_uint64, _p]
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libw4.so (raises if it has not been built)."""
+    global _LIB
+    if _LIB is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"{LIB_PATH} is missing: build it with "
+                "`python -m weight_only_int4_quantize_b200.build` (no CPU fallback exists)")
+        L = ctypes.CDLL(LIB_PATH)
+        _declare(L)
+        _LIB = L
+    return _LIB
+
+
+def _check(status: int, where: str) -> None:
+    if status != 0:
+        raise W4Error(status, where)
+
+
+def _torch():
+    import torch
+    return torch
+
+
+def _stream(device) -> int:
+    torch = _torch()
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def _cuda(t, dtype, name):
+    torch = _torch()
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t
+
+
+def quantize_pack(w, symmetric: bool, awq_s=None, shrink: float = 1.0, group: int = 128):
+    """RTN int4 g128 quantize+pack of a bf16 [N, K] weight on its device.
+
+    Returns (qweight int32 [N, K/8], scales fp16-bits int16 [N, K/128],
+    zeros fp16-bits int16 [N, K/128] or None when symmetric)."""
+    torch = _torch()
+    _cuda(w, torch.bfloat16, "w")
+    n, k = w.shape
+    if awq_s is not None:
+        _cuda(awq_s, torch.float32, "awq_s")
+    qw = torch.empty((n, k // 8), dtype=torch.int32, device=w.device)
+    sc = torch.empty((n, k // group), dtype=torch.int16, device=w.device)
+    zr = None if symmetric else torch.empty((n, k // group), dtype=torch.int16, device=w.device)
+    with torch.cuda.device(w.device):
+        st = lib().w4_quantize_pack(w.data_ptr(), n, k, group, int(bool(symmetric)),
+                                    None if awq_s is None else awq_s.data_ptr(),
+                                    float(shrink), qw.data_ptr(), sc.data_ptr(),
+                                    None if zr is None else zr.data_ptr(), _stream(w.device))
+    _check(st, "w4_quantize_pack")
+    return qw, sc, zr
+
+
+def w4a16_linear(x, qweight, scales, zeros=None, flags: int = 0, group: int = 128, out=None):
+    """y = x . dequant(Wq)^T, bf16 [M, K] -> bf16 [M, N]."""
+    torch = _torch()
+    _cuda(x, torch.bfloat16, "x")
+    _cuda(qweight, torch.int32, "qweight")
+    _cuda(scales, torch.int16, "scales")
+    if zeros is not None:
+        _cuda(zeros, torch.int16, "zeros")
+    m, k = x.shape
+    n = qweight.shape[0]
+    if qweight.shape[1] * 8 != k:
+        raise ValueError("qweight does not match x's K")
+    y = out if out is not None else torch.empty((m, n), dtype=torch.bfloat16, device=x.device)
+    with torch.cuda.device(x.device):
+        st = lib().w4a16_linear(x.data_ptr(), m, qweight.data_ptr(), scales.data_ptr(),
+                                None if zeros is None else zeros.data_ptr(), n, k, group,
+                                y.data_ptr(), int(flags), _stream(x.device))
+    _check(st, "w4a16_linear")
+    return y
+
+
+def awq_scales(x, alphas: Sequence[float]):
+    """s [n_alpha, K] float32 = max(mean|x|, 1e-8) ** alpha per input channel."""
+    torch = _torch()
+    import numpy as np
+    _cuda(x, torch.bfloat16, "x")
+    m, k = x.shape
+    a = np.ascontiguousarray(np.asarray(alphas, dtype=np.float32))
+    s = torch.empty((len(a), k), dtype=torch.float32, device=x.device)
+    with torch.cuda.device(x.device):
+        st = lib().w4_awq_scales(x.data_ptr(), m, k, a.ctypes.data, len(a), s.data_ptr(),
+                                 _stream(x.device))
+    _check(st, "w4_awq_scales")
+    return s
+
+
+def awq_workspace_bytes(m: int, n: int, k: int, n_alpha: int, n_shrink: int, n_seg: int = 1) -> int:
+    return int(lib().w4_awq_workspace_bytes(m, n, k, n_alpha, n_shrink, n_seg))
+
+
+def awq_score_grid(x, w, alphas, shrinks, symmetric: bool, seg_offsets=None, workspace=None,
+                   group: int = 128):
+    """SSE table [n_seg, n_alpha, n_shrink] (float64) and argmins [n_seg+1, 4]
+    (int32) of every (alpha, shrink) candidate, on the tensors' device."""
+    torch = _torch()
+    import numpy as np
+    _cuda(x, torch.bfloat16, "x")
+    _cuda(w, torch.bfloat16, "w")
+    m, k = x.shape
+    n = w.shape[0]
+    a = np.ascontiguousarray(np.asarray(alphas, dtype=np.float32))
+    r = np.ascontiguousarray(np.asarray(shrinks, dtype=np.float32))
+    if seg_offsets is None:
+        seg = None
+        n_seg = 1
+    else:
+        seg = np.ascontiguousarray(np.asarray(seg_offsets, dtype=np.int64))
+        n_seg = len(seg) - 1
+    need = awq_workspace_bytes(m, n, k, len(a), len(r), n_seg)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
+    sse = torch.empty((n_seg, len(a), len(r)), dtype=torch.float64, device=x.device)
+    arg = torch.empty((n_seg + 1, 4), dtype=torch.int32, device=x.device)
+    with torch.cuda.device(x.device):
+        st = lib().awq_score_grid(x.data_ptr(), m, w.data_ptr(), n, k, group,
+                                  int(bool(symmetric)), a.ctypes.data, len(a), r.ctypes.data,
+                                  len(r), None if seg is None else seg.ctypes.data, n_seg,
+                                  sse.data_ptr(), arg.data_ptr(), workspace.data_ptr(),
+                                  workspace.numel() * workspace.element_size(),
+                                  _stream(x.device))
+    _check(st, "awq_score_grid")
+    return sse, arg
+
+
+def device_error(clear: bool = True) -> int:
+    """The library's device error word (0 = no kernel gave up on a wait)."""
+    code = ctypes.c_uint32(0)
+    st = lib().w4_device_error(int(bool(clear)), ctypes.byref(code))
+    if st not in (0, 7):
+        _check(st, "w4_device_error")
+    return int(code.value)
+
+
+def selftest_bounded_wait(limit_ns: int = 20_000_000) -> None:
+    """Launches the bounded-wait self-test kernel on the current stream."""
+    torch = _torch()
+    _check(lib().w4_selftest_bounded_wait(int(limit_ns), _stream(torch.cuda.current_device())),
+           "w4_selftest_bounded_wait")

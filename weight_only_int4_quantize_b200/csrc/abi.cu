@@ -1,0 +1,277 @@
+// extern "C" entry points of libw4 (declared in include/w4.h): host-side
+// argument validation, path selection and workspace layout.  Nothing is
+// launched unless every check passes; the library allocates nothing.
+#include <cmath>
+#include <cstring>
+
+#include "w4.h"
+#include "w4_common.cuh"
+#include "w4_kernels.h"
+
+namespace w4 {
+
+// The device error word (one instance per device that loads the library).
+__device__ unsigned int g_w4_device_error;
+
+namespace {
+
+constexpr unsigned kKernelIdSelftest = 7;
+
+__global__ void selftest_wait_kernel(unsigned long long limit_ns, unsigned* err) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  // Nobody arrives on this barrier: the bounded wait must expire and report.
+  if (threadIdx.x == 0) {
+    mbar_wait(smem_u32(&bar), 0, &abort_flag, err, kKernelIdSelftest, limit_ns);
+  }
+  __syncthreads();
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+w4_status cuda_status(cudaError_t e) { return e == cudaSuccess ? W4_OK : W4_ERR_CUDA; }
+
+w4_status device_info(int* num_sms, unsigned** err_ptr) {
+  static int sms[64] = {};
+  static unsigned* errp[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return W4_ERR_CUDA;
+  if (dev < 0 || dev >= 64) return W4_ERR_UNSUPPORTED;
+  if (sms[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return W4_ERR_CUDA;
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_w4_device_error) != cudaSuccess) return W4_ERR_CUDA;
+    errp[dev] = static_cast<unsigned*>(p);
+    sms[dev] = n;
+  }
+  *num_sms = sms[dev];
+  if (err_ptr) *err_ptr = errp[dev];
+  return W4_OK;
+}
+
+bool valid_k(int64_t K) { return K >= 128 && K % 128 == 0 && K <= (int64_t{1} << 30); }
+
+// Workspace of awq_score_grid: every region 256-byte aligned.
+struct AwqWs {
+  size_t s, a, e, partials, total;
+};
+
+size_t round256(size_t b) { return (b + 255) & ~size_t{255}; }
+
+AwqWs awq_layout(int64_t M, int64_t N, int64_t K, int n_alpha, int n_shrink, int n_seg) {
+  AwqWs w;
+  w.s = 0;
+  w.a = w.s + round256(sizeof(float) * n_alpha * K);
+  w.e = w.a + round256(sizeof(uint16_t) * M * K);
+  w.partials = w.e + round256(sizeof(uint16_t) * static_cast<size_t>(n_shrink) * N * K);
+  const size_t tiles = static_cast<size_t>(sumsq_tiles(static_cast<int>(M), static_cast<int>(N)));
+  w.total = w.partials + round256(sizeof(double) * n_alpha * n_shrink * n_seg * tiles);
+  return w;
+}
+
+}  // namespace
+}  // namespace w4
+
+using namespace w4;
+
+extern "C" {
+
+const char* w4_status_string(w4_status s) {
+  switch (s) {
+    case W4_OK: return "ok";
+    case W4_ERR_INVALID_ARG: return "invalid argument";
+    case W4_ERR_SHAPE: return "invalid shape";
+    case W4_ERR_ALIGNMENT: return "device pointer not 16-byte aligned";
+    case W4_ERR_UNSUPPORTED: return "unsupported configuration";
+    case W4_ERR_WORKSPACE: return "workspace missing or too small";
+    case W4_ERR_CUDA: return "CUDA runtime error";
+    case W4_ERR_DEVICE_TIMEOUT: return "a kernel gave up on a bounded wait";
+  }
+  return "unknown status";
+}
+
+int w4_abi_version(void) { return W4_ABI_VERSION; }
+
+w4_status w4_quantize_pack(const void* w_bf16, int64_t N, int64_t K, int group, int symmetric,
+                           const float* awq_s, float shrink, int32_t* qweight,
+                           uint16_t* scales_f16, uint16_t* zeros_f16, void* stream) {
+  if (!w_bf16 || !qweight || !scales_f16) return W4_ERR_INVALID_ARG;
+  if ((symmetric != 0) != (zeros_f16 == nullptr)) return W4_ERR_INVALID_ARG;
+  if (!(shrink > 0.0f && shrink <= 1.0f)) return W4_ERR_INVALID_ARG;
+  if (group != 128) return W4_ERR_UNSUPPORTED;
+  if (N < 1 || !valid_k(K) || N > (int64_t{1} << 40) / K) return W4_ERR_SHAPE;
+  if (!aligned16(w_bf16) || !aligned16(qweight) || !aligned16(scales_f16) ||
+      (zeros_f16 && !aligned16(zeros_f16)) || (awq_s && !aligned16(awq_s)))
+    return W4_ERR_ALIGNMENT;
+  int sms = 0;
+  w4_status st = device_info(&sms, nullptr);
+  if (st != W4_OK) return st;
+  return cuda_status(launch_quantize_pack(w_bf16, N, K, symmetric != 0, awq_s, shrink, qweight,
+                                          scales_f16, zeros_f16,
+                                          static_cast<cudaStream_t>(stream), sms));
+}
+
+w4_status w4a16_linear(const void* x_bf16, int64_t M, const int32_t* qweight,
+                       const uint16_t* scales_f16, const uint16_t* zeros_f16, int64_t N,
+                       int64_t K, int group, void* y_bf16, unsigned flags, void* stream) {
+  if (!x_bf16 || !qweight || !scales_f16 || !y_bf16) return W4_ERR_INVALID_ARG;
+  const unsigned known = W4_LINEAR_FORCE_GEMV | W4_LINEAR_FORCE_GEMM | W4_LINEAR_PDL |
+                         W4_LINEAR_STATIC_WEIGHTS;
+  if (flags & ~known) return W4_ERR_INVALID_ARG;
+  if ((flags & W4_LINEAR_FORCE_GEMV) && (flags & W4_LINEAR_FORCE_GEMM)) return W4_ERR_INVALID_ARG;
+  if (group != 128) return W4_ERR_UNSUPPORTED;
+  if (M < 1 || N < 1 || !valid_k(K) || M > 0x7FFFFFFF || N > 0x7FFFFFFF) return W4_ERR_SHAPE;
+  if (!aligned16(x_bf16) || !aligned16(qweight) || !aligned16(scales_f16) ||
+      (zeros_f16 && !aligned16(zeros_f16)) || !aligned16(y_bf16))
+    return W4_ERR_ALIGNMENT;
+  const bool gemv = (flags & W4_LINEAR_FORCE_GEMV) || (M <= 16 && !(flags & W4_LINEAR_FORCE_GEMM));
+  if (gemv && M > 64) return W4_ERR_UNSUPPORTED;
+  if (!gemv && (M + 127) / 128 > 65535) return W4_ERR_UNSUPPORTED;
+  int sms = 0;
+  unsigned* err = nullptr;
+  w4_status st = device_info(&sms, &err);
+  if (st != W4_OK) return st;
+  const bool pdl = (flags & W4_LINEAR_PDL) != 0;
+  const bool stat = (flags & W4_LINEAR_STATIC_WEIGHTS) != 0;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (gemv)
+    return cuda_status(launch_gemv(x_bf16, static_cast<int>(M), qweight, scales_f16, zeros_f16,
+                                   static_cast<int>(N), static_cast<int>(K), y_bf16, pdl, stat, s,
+                                   sms));
+  return cuda_status(launch_prefill_gemm(x_bf16, static_cast<int>(M), qweight, scales_f16,
+                                         zeros_f16, static_cast<int>(N), static_cast<int>(K),
+                                         y_bf16, pdl, stat, s, err));
+}
+
+w4_status w4_awq_scales(const void* x_bf16, int64_t M, int64_t K, const float* alphas,
+                        int n_alpha, float* s_out, void* stream) {
+  if (!x_bf16 || !alphas || !s_out) return W4_ERR_INVALID_ARG;
+  if (n_alpha < 1 || n_alpha > kMaxGrid) return W4_ERR_UNSUPPORTED;
+  if (M < 1 || K < 1 || M > (int64_t{1} << 31) || K > (int64_t{1} << 31)) return W4_ERR_SHAPE;
+  if (!aligned16(x_bf16) || !aligned16(s_out)) return W4_ERR_ALIGNMENT;
+  AlphaList al;
+  al.n = n_alpha;
+  for (int i = 0; i < n_alpha; ++i) {
+    if (!std::isfinite(alphas[i])) return W4_ERR_INVALID_ARG;
+    al.v[i] = alphas[i];
+  }
+  int sms = 0;
+  w4_status st = device_info(&sms, nullptr);
+  if (st != W4_OK) return st;
+  return cuda_status(launch_awq_scales(x_bf16, M, K, al, s_out, static_cast<cudaStream_t>(stream)));
+}
+
+size_t w4_awq_workspace_bytes(int64_t M, int64_t N, int64_t K, int n_alpha, int n_shrink,
+                              int n_seg) {
+  if (M < 1 || N < 1 || K < 1 || n_alpha < 1 || n_shrink < 1 || n_seg < 1) return 0;
+  return awq_layout(M, N, K, n_alpha, n_shrink, n_seg).total;
+}
+
+w4_status awq_score_grid(const void* x_bf16, int64_t M, const void* w_bf16, int64_t N, int64_t K,
+                         int group, int symmetric, const float* alphas, int n_alpha,
+                         const float* shrinks, int n_shrink, const int64_t* seg_offsets,
+                         int n_seg, double* sse_out, int32_t* argmin_out, void* workspace,
+                         size_t workspace_bytes, void* stream) {
+  if (!x_bf16 || !w_bf16 || !alphas || !shrinks || !sse_out || !argmin_out)
+    return W4_ERR_INVALID_ARG;
+  if (group != 128) return W4_ERR_UNSUPPORTED;
+  if (n_alpha < 1 || n_alpha > kMaxGrid || n_shrink < 1 || n_shrink > kMaxGrid)
+    return W4_ERR_UNSUPPORTED;
+  if (n_seg < 1 || n_seg > 16) return W4_ERR_UNSUPPORTED;
+  if (M < 1 || N < 1 || !valid_k(K) || M > (int64_t{1} << 24) || N > (int64_t{1} << 24))
+    return W4_ERR_SHAPE;
+  if (seg_offsets == nullptr && n_seg != 1) return W4_ERR_INVALID_ARG;
+  int seg[17];
+  seg[0] = 0;
+  seg[n_seg] = static_cast<int>(N);
+  if (seg_offsets) {
+    if (seg_offsets[0] != 0 || seg_offsets[n_seg] != N) return W4_ERR_SHAPE;
+    for (int i = 1; i < n_seg; ++i) {
+      if (seg_offsets[i] <= seg_offsets[i - 1] || seg_offsets[i] % 16 != 0) return W4_ERR_SHAPE;
+      seg[i] = static_cast<int>(seg_offsets[i]);
+    }
+    if (seg_offsets[n_seg] <= seg_offsets[n_seg - 1]) return W4_ERR_SHAPE;
+  }
+  AlphaList al;
+  ShrinkList sl;
+  al.n = n_alpha;
+  sl.n = n_shrink;
+  for (int i = 0; i < n_alpha; ++i) {
+    if (!std::isfinite(alphas[i])) return W4_ERR_INVALID_ARG;
+    al.v[i] = alphas[i];
+  }
+  int c1 = 0;
+  bool have1 = false;
+  for (int j = 0; j < n_shrink; ++j) {
+    if (!(shrinks[j] > 0.0f && shrinks[j] <= 1.0f)) return W4_ERR_INVALID_ARG;
+    sl.v[j] = shrinks[j];
+    if (!have1 && shrinks[j] == 1.0f) {
+      c1 = j;
+      have1 = true;
+    }
+  }
+  if (!aligned16(x_bf16) || !aligned16(w_bf16) || !aligned16(sse_out) || !aligned16(argmin_out))
+    return W4_ERR_ALIGNMENT;
+  const AwqWs L = awq_layout(M, N, K, n_alpha, n_shrink, n_seg);
+  if (!workspace || workspace_bytes < L.total) return W4_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return W4_ERR_ALIGNMENT;
+
+  int sms = 0;
+  unsigned* err = nullptr;
+  w4_status st = device_info(&sms, &err);
+  if (st != W4_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  float* s_all = reinterpret_cast<float*>(ws + L.s);
+  void* a_buf = ws + L.a;
+  void* e_buf = ws + L.e;
+  double* partials = reinterpret_cast<double*>(ws + L.partials);
+  const int tiles = sumsq_tiles(static_cast<int>(M), static_cast<int>(N));
+
+  cudaError_t e = launch_awq_scales(x_bf16, M, K, al, s_all, s);
+  for (int i = 0; i < n_alpha && e == cudaSuccess; ++i) {
+    const float* si = s_all + static_cast<size_t>(i) * K;
+    e = launch_awq_xs(x_bf16, si, M, K, a_buf, s, sms);
+    if (e == cudaSuccess) e = launch_awq_err(w_bf16, si, N, K, symmetric != 0, sl, e_buf, s, sms);
+    if (e == cudaSuccess)
+      e = launch_sumsq_gemm(a_buf, static_cast<int>(M), e_buf, static_cast<int>(N),
+                            static_cast<int>(K), n_shrink,
+                            partials + static_cast<size_t>(i) * n_shrink * n_seg * tiles, n_seg,
+                            seg, s, err);
+  }
+  if (e == cudaSuccess) e = launch_awq_reduce(partials, n_alpha * n_shrink, n_seg, tiles, sse_out, s);
+  if (e == cudaSuccess) e = launch_awq_argmin(sse_out, n_seg, n_alpha, n_shrink, c1, argmin_out, s);
+  return cuda_status(e);
+}
+
+w4_status w4_device_error(int clear, uint32_t* code_out) {
+  unsigned v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_w4_device_error, sizeof(v)) != cudaSuccess) return W4_ERR_CUDA;
+  if (clear) {
+    const unsigned zero = 0;
+    if (cudaMemcpyToSymbol(g_w4_device_error, &zero, sizeof(zero)) != cudaSuccess)
+      return W4_ERR_CUDA;
+  }
+  if (code_out) *code_out = v;
+  return v ? W4_ERR_DEVICE_TIMEOUT : W4_OK;
+}
+
+w4_status w4_selftest_bounded_wait(uint64_t limit_ns, void* stream) {
+  if (limit_ns < 1000000ull || limit_ns > 2000000000ull) return W4_ERR_INVALID_ARG;
+  int sms = 0;
+  unsigned* err = nullptr;
+  w4_status st = device_info(&sms, &err);
+  if (st != W4_OK) return st;
+  selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(limit_ns, err);
+  return cuda_status(cudaGetLastError());
+}
+
+}  // extern "C"

@@ -1,0 +1,498 @@
+// tcgen05 GEMM core for sm_100a: D[M, N] = A[M, K] . B[N, K]^T with both
+// operands K-major in 128-byte-swizzled shared memory and the fp32
+// accumulator in tensor memory.  One CTA computes a 128 x 256 tile.
+//
+// Warp roles (10 warps):
+//   warp 0      TMA producer (A tiles; also B tiles when B comes from TMA)
+//   warp 1      TMEM allocation and the single-thread MMA issuer
+//   warps 2..9  B producers when B is a packed int4 weight: they stream the
+//               codes and scales from global memory, dequantize to bf16 in
+//               registers and write the swizzled tile; afterwards all eight
+//               run the epilogue (tcgen05.ld -> bf16 store, or sum of squares)
+//
+// Used by
+//   - the W4A16 prefill linear: A = x (bf16, TMA), B = dequant(Wq) (bf16),
+//     epilogue stores y in bf16;
+//   - AWQ candidate scoring: A = x / s (fp16, TMA), B = W s - w_hat (fp16,
+//     TMA, one candidate per grid z), epilogue writes per-tile sums of y^2
+//     in binary64 (deterministic order).
+//
+// Every mbarrier wait is bounded (w4_common.cuh); a CTA that gives up sets
+// the device error word, drains its own TMA loads and MMAs, frees its TMEM
+// and returns.  No TMA multicast.
+#include <cudaTypedefs.h>
+
+#include "w4_common.cuh"
+#include "w4_kernels.h"
+
+namespace w4 {
+
+namespace {
+
+constexpr int BM = 128;
+constexpr int BN = 256;
+constexpr int BK = 64;
+constexpr int kStages = 4;
+constexpr int kThreads = 320;
+constexpr int kProducerWarps = 8;
+constexpr uint32_t kTileABytes = BM * BK * 2;  // 16 KB
+constexpr uint32_t kTileBBytes = BN * BK * 2;  // 32 KB
+constexpr uint32_t kTmemCols = 256;
+
+enum : int { kBDequant = 0, kBTma = 1 };
+enum : int { kEpiStoreBf16 = 0, kEpiSumSquares = 1 };
+
+constexpr unsigned kKernelIdGemm = 2;
+
+struct SmemLayout {
+  // offsets from a 1024-byte aligned base
+  static constexpr uint32_t a = 0;
+  static constexpr uint32_t b = a + kStages * kTileABytes;
+  static constexpr uint32_t bars = b + kStages * kTileBBytes;
+  // full_a[S], full_b[S], empty[S], acc_full, done
+  static constexpr uint32_t misc = bars + (3 * kStages + 2) * 8;
+  static constexpr uint32_t total = misc + 64 + 16 * 16 * 8;  // + chunk sums
+};
+constexpr size_t kGemmSmemBytes = SmemLayout::total + 1024;
+
+struct SumSqArgs {
+  double* partials;     // [n_cand][n_seg][tiles]
+  int n_seg;
+  int seg_off[17];      // column (N) boundaries, multiples of 16 inside
+  int tiles;            // m_tiles * n_tiles
+};
+
+__device__ __forceinline__ void tma_load_3d(uint32_t smem_dst, const CUtensorMap* map, int c0,
+                                            int c1, int c2, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(bar)
+      : "memory");
+}
+
+__device__ __forceinline__ uint32_t bf16x2_sub(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+__device__ __forceinline__ uint32_t bf16x2_mul(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+__device__ __forceinline__ uint32_t bf16x2_fma(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t r;
+  asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(c));
+  return r;
+}
+__device__ __forceinline__ uint32_t bf16_pair(float v) {
+  const uint32_t h = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+  return h | (h << 16);
+}
+
+// Group constants for the exact bf16 dequantization of one row's group:
+// scale = hi + lo with hi = bf16(scale) and lo = scale - hi (exact in bf16:
+// the fp16 scale has 11 significant bits).  Then for t = q - z (exact):
+// fma(t, hi, t*lo) rounds t*scale once, i.e. equals bf16_rn((q - z)*scale).
+struct DqConst {
+  uint32_t zz;  // (128 + z) in both halves
+  uint32_t hi;
+  uint32_t lo;
+};
+
+__device__ __forceinline__ DqConst dq_const(float sc, float z) {
+  DqConst c;
+  const float hi = __bfloat162float(__float2bfloat16_rn(sc));
+  c.hi = bf16_pair(hi);
+  c.lo = bf16_pair(sc - hi);
+  c.zz = bf16_pair(128.0f + z);
+  return c;
+}
+
+// One packed word (8 codes, nibble order 0,2,4,6,1,3,5,7) -> 8 bf16 in
+// channel order (16 bytes).
+__device__ __forceinline__ uint4 dq_word(uint32_t v, const DqConst& c) {
+  uint32_t o[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t b = ((v >> (4 * i)) & 0x000F000Fu) | 0x43004300u;
+    const uint32_t t = bf16x2_sub(b, c.zz);
+    o[i] = bf16x2_fma(t, c.hi, bf16x2_mul(t, c.lo));
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v) {
+  asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y),
+               "r"(v.z), "r"(v.w)
+               : "memory");
+}
+
+template <int BSRC, int EPI, bool SYM>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_a,
+                   const __grid_constant__ CUtensorMap tmap_b,  // kBTma only
+                   const uint32_t* __restrict__ qw, const uint16_t* __restrict__ scales,
+                   const uint16_t* __restrict__ zeros,          // kBDequant only
+                   __nv_bfloat16* __restrict__ y,               // kEpiStoreBf16 only
+                   const __grid_constant__ SumSqArgs ss,        // kEpiSumSquares only
+                   int M, int N, int K, int pdl_static, unsigned* err) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  const uint32_t base = (raw_addr + 1023u) & ~1023u;
+  uint8_t* base_ptr = smem_raw + (base - raw_addr);
+
+  const uint32_t sA = base + SmemLayout::a;
+  const uint32_t sB = base + SmemLayout::b;
+  const uint32_t bar0 = base + SmemLayout::bars;
+  auto full_a = [&](int s) { return bar0 + 8u * s; };
+  auto full_b = [&](int s) { return bar0 + 8u * (kStages + s); };
+  auto empty = [&](int s) { return bar0 + 8u * (2 * kStages + s); };
+  const uint32_t acc_full = bar0 + 8u * (3 * kStages);
+  const uint32_t done_bar = acc_full + 8u;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(base_ptr + SmemLayout::misc);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base_ptr + SmemLayout::misc + 8);
+  double* chunk_sums = reinterpret_cast<double*>(base_ptr + SmemLayout::misc + 64);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int n0 = blockIdx.x * BN;
+  const int m0 = blockIdx.y * BM;
+  const int cand = blockIdx.z;
+  const int num_kb = K / BK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(full_a(s), 1);
+      mbar_init(full_b(s), BSRC == kBDequant ? kProducerWarps : 1);
+      mbar_init(empty(s), 1);
+    }
+    mbar_init(acc_full, 1);
+    mbar_init(done_bar, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmap_a);
+    if (BSRC == kBTma) tma_prefetch_desc(&tmap_b);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA --
+    if (lane == 0) {
+      pdl_wait();
+      int kb_stop = 0;  // loads for k-blocks [0, kb_stop) were issued
+      for (int kb = 0; kb < num_kb; ++kb) {
+        const int s = kb % kStages;
+        const uint32_t ph = (kb / kStages) & 1u;
+        if (!mbar_wait(empty(s), ph ^ 1u, abort_flag, err, kKernelIdGemm)) break;
+        if (BSRC == kBTma) {
+          mbar_arrive_expect_tx(full_a(s), kTileABytes + kTileBBytes);
+          tma_load_2d(sA + s * kTileABytes, &tmap_a, kb * BK, m0, full_a(s));
+          tma_load_3d(sB + s * kTileBBytes, &tmap_b, kb * BK, n0, cand, full_a(s));
+        } else {
+          mbar_arrive_expect_tx(full_a(s), kTileABytes);
+          tma_load_2d(sA + s * kTileABytes, &tmap_a, kb * BK, m0, full_a(s));
+        }
+        kb_stop = kb + 1;
+      }
+      if (*abort_flag) {
+        // Drain this CTA's own loads before leaving: the last issued k-block
+        // of each stage is the only one that can still be in flight.
+        for (int kb = kb_stop - kStages; kb < kb_stop; ++kb) {
+          if (kb < 0) continue;
+          volatile int dummy = 0;
+          mbar_wait(full_a(kb % kStages), (kb / kStages) & 1u, &dummy, err, kKernelIdGemm,
+                    kWaitLimitNs / 4);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA --
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_f16(BM, BN, EPI == kEpiStoreBf16);
+      bool issued = false;
+      for (int kb = 0; kb < num_kb; ++kb) {
+        const int s = kb % kStages;
+        const uint32_t ph = (kb / kStages) & 1u;
+        if (!mbar_wait(full_a(s), ph, abort_flag, err, kKernelIdGemm)) break;
+        if (BSRC == kBDequant && !mbar_wait(full_b(s), ph, abort_flag, err, kKernelIdGemm)) break;
+        tc_fence_after();
+        const uint64_t da = sdesc_k_sw128(sA + s * kTileABytes);
+        const uint64_t db = sdesc_k_sw128(sB + s * kTileBBytes);
+#pragma unroll
+        for (int kk = 0; kk < BK / 16; ++kk) {
+          // +32 bytes along K inside the swizzle atom = +2 in the address field
+          umma_f16(tmem_base, da + 2ull * kk, db + 2ull * kk, idesc, (kb | kk) != 0);
+        }
+        issued = true;
+        umma_commit(empty(s));
+      }
+      if (!*abort_flag) {
+        umma_commit(acc_full);
+      } else if (issued) {
+        umma_commit(done_bar);  // wait for in-flight MMAs before TMEM is freed
+        volatile int dummy = 0;
+        mbar_wait(done_bar, 0, &dummy, err, kKernelIdGemm, kWaitLimitNs / 4);
+      }
+    }
+  } else {
+    const int pt = threadIdx.x - 64;  // 0..255
+    // ------------------------------------------------- B producers ----
+    if (BSRC == kBDequant) {
+      // Thread pt owns rows r = it*128 + pt/2 (it = 0, 1) and half (pt & 1)
+      // of each row's 64-channel stage slice: 4 packed words -> 4 chunks.
+      const int half = pt & 1;
+      const int G = K >> 7;
+      const size_t row_words = static_cast<size_t>(K) >> 3;
+      int rows[2];
+      bool valid[2];
+      const uint32_t* qrow[2];
+#pragma unroll
+      for (int it = 0; it < 2; ++it) {
+        rows[it] = it * 128 + (pt >> 1);
+        valid[it] = (n0 + rows[it]) < N;
+        qrow[it] = qw + static_cast<size_t>(valid[it] ? n0 + rows[it] : 0) * row_words + 4 * half;
+      }
+      if (pdl_static == 0) pdl_wait();
+      DqConst dc[2];
+      int cur_group = -1;
+      for (int kb = 0; kb < num_kb; ++kb) {
+        const int s = kb % kStages;
+        const uint32_t ph = (kb / kStages) & 1u;
+        uint4 raw[2];
+#pragma unroll
+        for (int it = 0; it < 2; ++it)
+          raw[it] = valid[it] ? __ldg(reinterpret_cast<const uint4*>(qrow[it] + kb * 8))
+                              : make_uint4(0, 0, 0, 0);
+        const int grp = kb >> 1;
+        if (grp != cur_group) {
+          cur_group = grp;
+#pragma unroll
+          for (int it = 0; it < 2; ++it) {
+            float sc = 0.f, z = 8.f;
+            if (valid[it]) {
+              const size_t gi = static_cast<size_t>(n0 + rows[it]) * G + grp;
+              sc = __half2float(__ushort_as_half(scales[gi]));
+              if (!SYM) z = __half2float(__ushort_as_half(zeros[gi]));
+            }
+            dc[it] = dq_const(sc, z);
+          }
+        }
+        if (!mbar_wait(empty(s), ph ^ 1u, abort_flag, err, kKernelIdGemm)) break;
+        const uint32_t tile = sB + s * kTileBBytes;
+#pragma unroll
+        for (int it = 0; it < 2; ++it) {
+          const uint32_t w4[4] = {raw[it].x, raw[it].y, raw[it].z, raw[it].w};
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            st_shared_v4(tile + sw128_offset(rows[it], 4 * half + j), dq_word(w4[j], dc[it]));
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(full_b(s));
+      }
+      if (pdl_static != 0) pdl_wait();
+    }
+
+    if (BSRC == kBTma) pdl_wait();
+
+    // --------------------------------------------------------- epilogue --
+    const int q = warp & 3;         // TMEM lane quarter of this warp
+    const int ch = (warp - 2) >> 2;  // column half: 0 -> 0..127, 1 -> 128..255
+    const bool ok = mbar_wait(acc_full, 0, abort_flag, err, kKernelIdGemm);
+    tc_fence_after();
+    if (ok) {
+      const int m = m0 + 32 * q + lane;
+      if (EPI == kEpiStoreBf16) {
+        for (int c = 0; c < 8; ++c) {
+          const int col = 128 * ch + 16 * c;
+          uint32_t r[16];
+          tmem_ld_32x32b_x16(tmem_base + (static_cast<uint32_t>(32 * q) << 16) + col, r);
+          tmem_ld_wait();
+          const int n = n0 + col;
+          if (m < M && n < N) {
+            __nv_bfloat16* dst = y + static_cast<size_t>(m) * N + n;
+            uint32_t p[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const __nv_bfloat162 b2 =
+                  __floats2bfloat162_rn(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+              p[i] = *reinterpret_cast<const uint32_t*>(&b2);
+            }
+            if (n + 16 <= N && (N & 7) == 0) {
+              uint4* d4 = reinterpret_cast<uint4*>(dst);
+              d4[0] = make_uint4(p[0], p[1], p[2], p[3]);
+              d4[1] = make_uint4(p[4], p[5], p[6], p[7]);
+            } else {
+              for (int i = 0; i < 16 && n + i < N; ++i)
+                dst[i] = __float2bfloat16_rn(__uint_as_float(r[i]));
+            }
+          }
+        }
+      } else {
+        // Sum of squares per 16-column chunk: thread -> fixed-order shuffle
+        // tree over the 32 rows of this warp -> shared -> fixed order over
+        // the 4 warps of this column half -> per-segment sums.
+        for (int c = 0; c < 8; ++c) {
+          const int col = 128 * ch + 16 * c;
+          uint32_t r[16];
+          tmem_ld_32x32b_x16(tmem_base + (static_cast<uint32_t>(32 * q) << 16) + col, r);
+          tmem_ld_wait();
+          double acc = 0.0;
+          if (m < M) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const double v = static_cast<double>(__uint_as_float(r[i]));
+              if (n0 + col + i < N) acc = fma(v, v, acc);
+            }
+          }
+#pragma unroll
+          for (int o = 16; o; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+          if (lane == 0) chunk_sums[(8 * ch + c) * 4 + q] = acc;
+        }
+      }
+    }
+    if (EPI == kEpiSumSquares) {
+      asm volatile("bar.sync 1, 256;" ::: "memory");  // the eight epilogue warps
+      if (pt < 16) {
+        const int chunk = pt;  // 16-column chunk of the tile
+        const double v = ((chunk_sums[chunk * 4 + 0] + chunk_sums[chunk * 4 + 1]) +
+                          chunk_sums[chunk * 4 + 2]) + chunk_sums[chunk * 4 + 3];
+        chunk_sums[64 + chunk] = v;
+      }
+      asm volatile("bar.sync 1, 256;" ::: "memory");
+      if (pt < ss.n_seg && !*abort_flag) {
+        double sum = 0.0;
+        for (int chunk = 0; chunk < 16; ++chunk) {
+          const int c0 = n0 + 16 * chunk;
+          if (c0 >= ss.seg_off[pt] && c0 < ss.seg_off[pt + 1]) sum += chunk_sums[64 + chunk];
+        }
+        const int tile = blockIdx.y * gridDim.x + blockIdx.x;
+        ss.partials[(static_cast<size_t>(cand) * ss.n_seg + pt) * ss.tiles + tile] = sum;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (threadIdx.x == 0) pdl_launch_dependents();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+CUresult encode_tmap(CUtensorMap* map, CUtensorMapDataType dt, int rank, const uint64_t* dims,
+                     const uint64_t* strides_bytes, const uint32_t* box, const void* base) {
+  static PFN_cuTensorMapEncodeTiled fn = nullptr;
+  if (!fn) {
+    cudaDriverEntryPointQueryResult q;
+    void* p = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || !p)
+      return CUDA_ERROR_NOT_FOUND;
+    fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled>(p);
+  }
+  uint32_t estr[3] = {1, 1, 1};
+  return fn(map, dt, rank, const_cast<void*>(base), dims, strides_bytes, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+}
+
+template <typename Kern>
+cudaError_t launch_gemm(Kern kern, dim3 grid, bool pdl, cudaStream_t stream,
+                        const CUtensorMap& ta, const CUtensorMap& tb, const uint32_t* qw,
+                        const uint16_t* sc, const uint16_t* z, __nv_bfloat16* y,
+                        const SumSqArgs& ss, int M, int N, int K, int pdl_static,
+                        unsigned* err) {
+  // The opt-in shared-memory size is a per-device function attribute; set it
+  // once per device and kernel instantiation.
+  static unsigned long long attr_done = 0;  // bit d: device d
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev >= 64 || !(__atomic_load_n(&attr_done, __ATOMIC_ACQUIRE) & (1ull << dev))) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(kGemmSmemBytes));
+    if (e != cudaSuccess) return e;
+    if (dev < 64) __atomic_fetch_or(&attr_done, 1ull << dev, __ATOMIC_RELEASE);
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = kGemmSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  if (pdl) {
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+  }
+  return cudaLaunchKernelEx(&cfg, kern, ta, tb, qw, sc, z, y, ss, M, N, K, pdl_static, err);
+}
+
+}  // namespace
+
+cudaError_t launch_prefill_gemm(const void* x, int M, const int32_t* qw, const uint16_t* sc,
+                                const uint16_t* z, int N, int K, void* y, bool pdl,
+                                bool static_w, cudaStream_t stream, unsigned* err) {
+  CUtensorMap ta, tb;
+  const uint64_t dims[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(M)};
+  const uint64_t str[1] = {static_cast<uint64_t>(K) * 2};
+  const uint32_t box[2] = {BK, BM};
+  if (encode_tmap(&ta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, dims, str, box, x) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+  tb = ta;  // unused by the dequant variant
+  SumSqArgs ss = {};
+  dim3 grid((N + BN - 1) / BN, (M + BM - 1) / BM, 1);
+  const uint32_t* q = reinterpret_cast<const uint32_t*>(qw);
+  __nv_bfloat16* yp = static_cast<__nv_bfloat16*>(y);
+  const int ps = (pdl && static_w) ? 1 : 0;
+  if (z == nullptr)
+    return launch_gemm(gemm_tc_kernel<kBDequant, kEpiStoreBf16, true>, grid, pdl, stream, ta, tb,
+                       q, sc, z, yp, ss, M, N, K, ps, err);
+  return launch_gemm(gemm_tc_kernel<kBDequant, kEpiStoreBf16, false>, grid, pdl, stream, ta, tb,
+                     q, sc, z, yp, ss, M, N, K, ps, err);
+}
+
+cudaError_t launch_sumsq_gemm(const void* a_f16, int M, const void* b_f16, int N, int K,
+                              int n_cand, double* partials, int n_seg, const int* seg_off,
+                              cudaStream_t stream, unsigned* err) {
+  CUtensorMap ta, tb;
+  const uint64_t da[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(M)};
+  const uint64_t sa[1] = {static_cast<uint64_t>(K) * 2};
+  const uint32_t ba[2] = {BK, BM};
+  if (encode_tmap(&ta, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, da, sa, ba, a_f16) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+  const uint64_t db[3] = {static_cast<uint64_t>(K), static_cast<uint64_t>(N),
+                          static_cast<uint64_t>(n_cand)};
+  const uint64_t sb[2] = {static_cast<uint64_t>(K) * 2, static_cast<uint64_t>(K) * 2 * N};
+  const uint32_t bb[3] = {BK, BN, 1};
+  if (encode_tmap(&tb, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, db, sb, bb, b_f16) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+  SumSqArgs ss = {};
+  ss.partials = partials;
+  ss.n_seg = n_seg;
+  for (int i = 0; i <= n_seg; ++i) ss.seg_off[i] = seg_off[i];
+  dim3 grid((N + BN - 1) / BN, (M + BM - 1) / BM, n_cand);
+  ss.tiles = grid.x * grid.y;
+  return launch_gemm(gemm_tc_kernel<kBTma, kEpiSumSquares, false>, grid, false, stream, ta, tb,
+                     nullptr, nullptr, nullptr, nullptr, ss, M, N, K, 0, err);
+}
+
+int sumsq_tiles(int M, int N) { return ((N + BN - 1) / BN) * ((M + BM - 1) / BM); }
+
+}  // namespace w4
