@@ -69,6 +69,11 @@ typedef enum {
 /* Static, NUL-terminated description of a status code. */
 const char* w4_status_string(w4_status status);
 
+/* Description of the last W4_ERR_CUDA returned on the calling host thread
+ * (the failing step and the CUDA error name); empty if none.  Static storage
+ * of the library, valid until the next call on that thread. */
+const char* w4_last_error(void);
+
 /* ABI version of this header (bumped on any incompatible change). */
 #define W4_ABI_VERSION 1
 int w4_abi_version(void);

@@ -122,8 +122,8 @@ def _near_tie_inputs(sym, groups=64, rows=8, seed=3):
             if j >= base + 128:
                 break
             t = np.float32((mm + 0.5) * np.float64(sc))
-            u = t.view(np.uint32) + np.uint32(rng.integers(-3, 4) & 0xFFFFFFFF)
-            s[j] = u.view(np.float32) if t != 0 else t
+            u = (int(t.view(np.uint32)) + int(rng.integers(-3, 4))) & 0xFFFFFFFF
+            s[j] = np.uint32(u).view(np.float32)
     rowscale = (2.0 ** (np.arange(rows) % 5 - 2)).astype(np.float32)
     w = torch.from_numpy(np.repeat(rowscale[:, None], k, axis=1)).to(torch.bfloat16)
     return w, s

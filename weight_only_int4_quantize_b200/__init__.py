@@ -38,6 +38,8 @@ class W4Error(RuntimeError):
         self.status = status
         self.name = _STATUS.get(status, str(status))
         msg = lib().w4_status_string(status).decode() if _LIB is not None else self.name
+        if status == 6 and _LIB is not None:
+            msg += "; " + lib().w4_last_error().decode()
         super().__init__(f"{where}: {self.name} ({msg})")
 
 
@@ -51,6 +53,8 @@ _i64 = ctypes.c_int64
 def _declare(L: ctypes.CDLL) -> None:
     L.w4_status_string.restype = ctypes.c_char_p
     L.w4_status_string.argtypes = [ctypes.c_int]
+    L.w4_last_error.restype = ctypes.c_char_p
+    L.w4_last_error.argtypes = []
     L.w4_abi_version.restype = ctypes.c_int
     L.w4_abi_version.argtypes = []
     L.w4_quantize_pack.restype = ctypes.c_int

@@ -2,6 +2,7 @@
 // argument validation, path selection and workspace layout.  Nothing is
 // launched unless every check passes; the library allocates nothing.
 #include <cmath>
+#include <cstdio>
 #include <cstring>
 
 #include "w4.h"
@@ -35,20 +36,30 @@ __global__ void selftest_wait_kernel(unsigned long long limit_ns, unsigned* err)
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-w4_status cuda_status(cudaError_t e) { return e == cudaSuccess ? W4_OK : W4_ERR_CUDA; }
+// Description of the last W4_ERR_CUDA of this host thread.
+thread_local char g_last_error[256] = "";
+
+w4_status cuda_status(cudaError_t e, const char* step = "launch") {
+  if (e == cudaSuccess) return W4_OK;
+  snprintf(g_last_error, sizeof(g_last_error), "%s: %s (%s)", step, cudaGetErrorName(e),
+           cudaGetErrorString(e));
+  return W4_ERR_CUDA;
+}
 
 w4_status device_info(int* num_sms, unsigned** err_ptr) {
   static int sms[64] = {};
   static unsigned* errp[64] = {};
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return W4_ERR_CUDA;
+  cudaError_t ge = cudaGetDevice(&dev);
+  if (ge != cudaSuccess) return cuda_status(ge, "cudaGetDevice");
   if (dev < 0 || dev >= 64) return W4_ERR_UNSUPPORTED;
   if (sms[dev] == 0) {
     int n = 0;
-    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-      return W4_ERR_CUDA;
+    cudaError_t e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return cuda_status(e, "SM count");
     void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_w4_device_error) != cudaSuccess) return W4_ERR_CUDA;
+    e = cudaGetSymbolAddress(&p, g_w4_device_error);
+    if (e != cudaSuccess) return cuda_status(e, "error word address");
     errp[dev] = static_cast<unsigned*>(p);
     sms[dev] = n;
   }
@@ -100,6 +111,8 @@ const char* w4_status_string(w4_status s) {
 
 int w4_abi_version(void) { return W4_ABI_VERSION; }
 
+const char* w4_last_error(void) { return g_last_error; }
+
 w4_status w4_quantize_pack(const void* w_bf16, int64_t N, int64_t K, int group, int symmetric,
                            const float* awq_s, float shrink, int32_t* qweight,
                            uint16_t* scales_f16, uint16_t* zeros_f16, void* stream) {
@@ -116,7 +129,8 @@ w4_status w4_quantize_pack(const void* w_bf16, int64_t N, int64_t K, int group, 
   if (st != W4_OK) return st;
   return cuda_status(launch_quantize_pack(w_bf16, N, K, symmetric != 0, awq_s, shrink, qweight,
                                           scales_f16, zeros_f16,
-                                          static_cast<cudaStream_t>(stream), sms));
+                                          static_cast<cudaStream_t>(stream), sms),
+                     "quantize+pack launch");
 }
 
 w4_status w4a16_linear(const void* x_bf16, int64_t M, const int32_t* qweight,
@@ -145,10 +159,12 @@ w4_status w4a16_linear(const void* x_bf16, int64_t M, const int32_t* qweight,
   if (gemv)
     return cuda_status(launch_gemv(x_bf16, static_cast<int>(M), qweight, scales_f16, zeros_f16,
                                    static_cast<int>(N), static_cast<int>(K), y_bf16, pdl, stat, s,
-                                   sms));
+                                   sms),
+                       "decode GEMV launch");
   return cuda_status(launch_prefill_gemm(x_bf16, static_cast<int>(M), qweight, scales_f16,
                                          zeros_f16, static_cast<int>(N), static_cast<int>(K),
-                                         y_bf16, pdl, stat, s, err));
+                                         y_bf16, pdl, stat, s, err),
+                     "prefill tcgen05 GEMM launch");
 }
 
 w4_status w4_awq_scales(const void* x_bf16, int64_t M, int64_t K, const float* alphas,
@@ -237,28 +253,35 @@ w4_status awq_score_grid(const void* x_bf16, int64_t M, const void* w_bf16, int6
   const int tiles = sumsq_tiles(static_cast<int>(M), static_cast<int>(N));
 
   cudaError_t e = launch_awq_scales(x_bf16, M, K, al, s_all, s);
-  for (int i = 0; i < n_alpha && e == cudaSuccess; ++i) {
+  if (e != cudaSuccess) return cuda_status(e, "awq scales");
+  for (int i = 0; i < n_alpha; ++i) {
     const float* si = s_all + static_cast<size_t>(i) * K;
     e = launch_awq_xs(x_bf16, si, M, K, a_buf, s, sms);
-    if (e == cudaSuccess) e = launch_awq_err(w_bf16, si, N, K, symmetric != 0, sl, e_buf, s, sms);
-    if (e == cudaSuccess)
-      e = launch_sumsq_gemm(a_buf, static_cast<int>(M), e_buf, static_cast<int>(N),
-                            static_cast<int>(K), n_shrink,
-                            partials + static_cast<size_t>(i) * n_shrink * n_seg * tiles, n_seg,
-                            seg, s, err);
+    if (e != cudaSuccess) return cuda_status(e, "awq x/s operand");
+    e = launch_awq_err(w_bf16, si, N, K, symmetric != 0, sl, e_buf, s, sms);
+    if (e != cudaSuccess) return cuda_status(e, "awq error operand");
+    e = launch_sumsq_gemm(a_buf, static_cast<int>(M), e_buf, static_cast<int>(N),
+                          static_cast<int>(K), n_shrink,
+                          partials + static_cast<size_t>(i) * n_shrink * n_seg * tiles, n_seg, seg,
+                          s, err);
+    if (e != cudaSuccess) return cuda_status(e, "awq tcgen05 sum-of-squares GEMM");
   }
-  if (e == cudaSuccess) e = launch_awq_reduce(partials, n_alpha * n_shrink, n_seg, tiles, sse_out, s);
-  if (e == cudaSuccess) e = launch_awq_argmin(sse_out, n_seg, n_alpha, n_shrink, c1, argmin_out, s);
-  return cuda_status(e);
+  e = launch_awq_reduce(partials, n_alpha * n_shrink, n_seg, tiles, sse_out, s);
+  if (e != cudaSuccess) return cuda_status(e, "awq reduce");
+  return cuda_status(launch_awq_argmin(sse_out, n_seg, n_alpha, n_shrink, c1, argmin_out, s),
+                     "awq argmin");
 }
 
 w4_status w4_device_error(int clear, uint32_t* code_out) {
   unsigned v = 0;
-  if (cudaMemcpyFromSymbol(&v, g_w4_device_error, sizeof(v)) != cudaSuccess) return W4_ERR_CUDA;
+  w4_status st = cuda_status(cudaMemcpyFromSymbol(&v, g_w4_device_error, sizeof(v)),
+                             "read device error word");
+  if (st != W4_OK) return st;
   if (clear) {
     const unsigned zero = 0;
-    if (cudaMemcpyToSymbol(g_w4_device_error, &zero, sizeof(zero)) != cudaSuccess)
-      return W4_ERR_CUDA;
+    st = cuda_status(cudaMemcpyToSymbol(g_w4_device_error, &zero, sizeof(zero)),
+                     "clear device error word");
+    if (st != W4_OK) return st;
   }
   if (code_out) *code_out = v;
   return v ? W4_ERR_DEVICE_TIMEOUT : W4_OK;

@@ -411,8 +411,10 @@ CUresult encode_tmap(CUtensorMap* map, CUtensorMapDataType dt, int rank, const u
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
 }
 
-template <typename Kern>
-cudaError_t launch_gemm(Kern kern, dim3 grid, bool pdl, cudaStream_t stream,
+// One instantiation per kernel (the cache below must be per kernel, and
+// every instantiation of gemm_tc_kernel has the same function type).
+template <auto kern>
+cudaError_t launch_gemm(dim3 grid, bool pdl, cudaStream_t stream,
                         const CUtensorMap& ta, const CUtensorMap& tb, const uint32_t* qw,
                         const uint16_t* sc, const uint16_t* z, __nv_bfloat16* y,
                         const SumSqArgs& ss, int M, int N, int K, int pdl_static,
@@ -462,9 +464,9 @@ cudaError_t launch_prefill_gemm(const void* x, int M, const int32_t* qw, const u
   __nv_bfloat16* yp = static_cast<__nv_bfloat16*>(y);
   const int ps = (pdl && static_w) ? 1 : 0;
   if (z == nullptr)
-    return launch_gemm(gemm_tc_kernel<kBDequant, kEpiStoreBf16, true>, grid, pdl, stream, ta, tb,
+    return launch_gemm<gemm_tc_kernel<kBDequant, kEpiStoreBf16, true>>(grid, pdl, stream, ta, tb,
                        q, sc, z, yp, ss, M, N, K, ps, err);
-  return launch_gemm(gemm_tc_kernel<kBDequant, kEpiStoreBf16, false>, grid, pdl, stream, ta, tb,
+  return launch_gemm<gemm_tc_kernel<kBDequant, kEpiStoreBf16, false>>(grid, pdl, stream, ta, tb,
                      q, sc, z, yp, ss, M, N, K, ps, err);
 }
 
@@ -489,7 +491,7 @@ cudaError_t launch_sumsq_gemm(const void* a_f16, int M, const void* b_f16, int N
   for (int i = 0; i <= n_seg; ++i) ss.seg_off[i] = seg_off[i];
   dim3 grid((N + BN - 1) / BN, (M + BM - 1) / BM, n_cand);
   ss.tiles = grid.x * grid.y;
-  return launch_gemm(gemm_tc_kernel<kBTma, kEpiSumSquares, false>, grid, false, stream, ta, tb,
+  return launch_gemm<gemm_tc_kernel<kBTma, kEpiSumSquares, false>>(grid, false, stream, ta, tb,
                      nullptr, nullptr, nullptr, nullptr, ss, M, N, K, 0, err);
 }
 
