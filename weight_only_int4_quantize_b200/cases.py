@@ -1,0 +1,107 @@
+"""Runs one library call on a named shape, for profilers (ncu) and quick
+timing.  Inputs are seeded and generated on the device.
+
+    python -m weight_only_int4_quantize_b200.cases quantize --n 17408 --k 5120 [--sym]
+    python -m weight_only_int4_quantize_b200.cases linear --m 8 --n 17408 --k 5120 [--sym] [--gemm]
+    python -m weight_only_int4_quantize_b200.cases awq --m 2048 --n 1024 --k 2048 --na 20 --nr 10
+
+Each case captures --iters launches in one CUDA graph (so host launch
+overhead does not count), replays it once to warm up, times one replay with
+CUDA events and prints the mean time per launch and the algorithmic
+throughput.  Back-to-back launches of one linear re-read the same weights:
+for weights smaller than L2 this measures L2, not HBM.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+
+import torch
+
+import weight_only_int4_quantize_b200 as w4
+from weight_only_int4_quantize_b200 import synth
+
+
+def _weights(n, k, seed, std=0.02):
+    g = torch.Generator(device="cuda")
+    g.manual_seed(seed)
+    return (torch.randn(n, k, generator=g, device="cuda") * std).to(torch.bfloat16)
+
+
+def _time(fn, iters, graph=True):
+    """Mean device time per call: `iters` calls captured in one CUDA graph
+    (no host launch overhead between them), replayed after a warm replay."""
+    fn()
+    torch.cuda.synchronize()
+    if graph:
+        g = torch.cuda.CUDAGraph()
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            with torch.cuda.graph(g, stream=s):
+                for _ in range(iters):
+                    fn()
+        torch.cuda.current_stream().wait_stream(s)
+        run = g.replay
+        run()
+    else:
+        def run():
+            for _ in range(iters):
+                fn()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    run()
+    b.record()
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / iters
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("case", choices=["quantize", "linear", "awq"])
+    ap.add_argument("--m", type=int, default=8)
+    ap.add_argument("--n", type=int, default=4096)
+    ap.add_argument("--k", type=int, default=4096)
+    ap.add_argument("--sym", action="store_true")
+    ap.add_argument("--gemm", action="store_true", help="force the tcgen05 prefill kernel")
+    ap.add_argument("--gemv", action="store_true", help="force the decode kernel")
+    ap.add_argument("--na", type=int, default=20)
+    ap.add_argument("--nr", type=int, default=10)
+    ap.add_argument("--iters", type=int, default=3)
+    ap.add_argument("--pdl", action="store_true", help="programmatic dependent launch + static weights")
+    ap.add_argument("--eager", action="store_true", help="time eager launches instead of a graph")
+    a = ap.parse_args()
+    w = _weights(a.n, a.k, 1)
+    out = {"case": a.case, "m": a.m, "n": a.n, "k": a.k, "sym": a.sym}
+    if a.case == "quantize":
+        ms = _time(lambda: w4.quantize_pack(w, a.sym), a.iters, not a.eager)
+        b = a.n * a.k * (2.5 + (2 if a.sym else 4) / 128)
+        out.update(ms=ms, gbs=b / ms / 1e6)
+    elif a.case == "linear":
+        qw, sc, zr = w4.quantize_pack(w, a.sym)
+        del w
+        g = torch.Generator(device="cuda")
+        g.manual_seed(2)
+        x = torch.randn(a.m, a.k, generator=g, device="cuda").to(torch.bfloat16)
+        y = torch.empty(a.m, a.n, dtype=torch.bfloat16, device="cuda")
+        flags = (w4.LINEAR_FORCE_GEMM if a.gemm else 0) | (w4.LINEAR_FORCE_GEMV if a.gemv else 0)
+        if a.pdl:
+            flags |= w4.LINEAR_PDL | w4.LINEAR_STATIC_WEIGHTS
+        ms = _time(lambda: w4.w4a16_linear(x, qw, sc, zr, flags=flags, out=y), a.iters, not a.eager)
+        b = a.n * a.k * (0.5 + (2 if a.sym else 4) / 128) + 2 * a.m * (a.k + a.n)
+        out.update(ms=ms, gbs=b / ms / 1e6, tflops=2.0 * a.m * a.n * a.k / ms / 1e9)
+    else:
+        g = torch.Generator(device="cuda")
+        g.manual_seed(3)
+        x = (torch.randn(a.m, a.k, generator=g, device="cuda")).to(torch.bfloat16)
+        al, sh = synth.alpha_grid(a.na), synth.shrink_grid(a.nr)
+        ws = torch.empty(w4.awq_workspace_bytes(a.m, a.n, a.k, a.na, a.nr), dtype=torch.uint8,
+                         device="cuda")
+        ms = _time(lambda: w4.awq_score_grid(x, w, al, sh, a.sym, workspace=ws), a.iters, False)
+        out.update(ms=ms, tflops=2.0 * a.m * a.n * a.k * a.na * a.nr / ms / 1e9)
+    print(json.dumps(out))
+
+
+if __name__ == "__main__":
+    main()

@@ -38,6 +38,7 @@ constexpr int kProducerWarps = 8;
 constexpr uint32_t kTileABytes = BM * BK * 2;  // 16 KB
 constexpr uint32_t kTileBBytes = BN * BK * 2;  // 32 KB
 constexpr uint32_t kTmemCols = 256;
+constexpr int kLoadAhead = 4;  // stages of packed codes in flight per producer thread
 
 enum : int { kBDequant = 0, kBTma = 1 };
 enum : int { kEpiStoreBf16 = 0, kEpiSumSquares = 1 };
@@ -251,55 +252,74 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (BSRC == kBDequant) {
       // Thread pt owns rows r = it*128 + pt/2 (it = 0, 1) and half (pt & 1)
       // of each row's 64-channel stage slice: 4 packed words -> 4 chunks.
+      // A register ring keeps kLoadAhead stages of codes (and their group's
+      // scale/zero) in flight ahead of the stage being written.
       const int half = pt & 1;
       const int G = K >> 7;
       const size_t row_words = static_cast<size_t>(K) >> 3;
       int rows[2];
       bool valid[2];
       const uint32_t* qrow[2];
+      const uint16_t* srow[2];
+      const uint16_t* zrow[2];
 #pragma unroll
       for (int it = 0; it < 2; ++it) {
         rows[it] = it * 128 + (pt >> 1);
         valid[it] = (n0 + rows[it]) < N;
-        qrow[it] = qw + static_cast<size_t>(valid[it] ? n0 + rows[it] : 0) * row_words + 4 * half;
+        const size_t row = static_cast<size_t>(valid[it] ? n0 + rows[it] : 0);
+        qrow[it] = qw + row * row_words + 4 * half;
+        srow[it] = scales + row * G;
+        zrow[it] = SYM ? nullptr : zeros + row * G;
       }
-      if (pdl_static == 0) pdl_wait();
-      DqConst dc[2];
-      int cur_group = -1;
-      for (int kb = 0; kb < num_kb; ++kb) {
-        const int s = kb % kStages;
-        const uint32_t ph = (kb / kStages) & 1u;
-        uint4 raw[2];
-#pragma unroll
-        for (int it = 0; it < 2; ++it)
-          raw[it] = valid[it] ? __ldg(reinterpret_cast<const uint4*>(qrow[it] + kb * 8))
-                              : make_uint4(0, 0, 0, 0);
-        const int grp = kb >> 1;
-        if (grp != cur_group) {
-          cur_group = grp;
-#pragma unroll
-          for (int it = 0; it < 2; ++it) {
-            float sc = 0.f, z = 8.f;
-            if (valid[it]) {
-              const size_t gi = static_cast<size_t>(n0 + rows[it]) * G + grp;
-              sc = __half2float(__ushort_as_half(scales[gi]));
-              if (!SYM) z = __half2float(__ushort_as_half(zeros[gi]));
-            }
-            dc[it] = dq_const(sc, z);
-          }
-        }
-        if (!mbar_wait(empty(s), ph ^ 1u, abort_flag, err, kKernelIdGemm)) break;
-        const uint32_t tile = sB + s * kTileBBytes;
+      uint4 ring[kLoadAhead][2];
+      uint32_t ring_sz[kLoadAhead][2];
+      auto fetch = [&](int kb, uint4 (&q)[2], uint32_t (&sz)[2]) {
 #pragma unroll
         for (int it = 0; it < 2; ++it) {
-          const uint32_t w4[4] = {raw[it].x, raw[it].y, raw[it].z, raw[it].w};
-#pragma unroll
-          for (int j = 0; j < 4; ++j)
-            st_shared_v4(tile + sw128_offset(rows[it], 4 * half + j), dq_word(w4[j], dc[it]));
+          q[it] = make_uint4(0, 0, 0, 0);
+          sz[it] = 0x48000000u;  // scale 0, zero 8
+          if (valid[it] && kb < num_kb) {
+            q[it] = __ldg(reinterpret_cast<const uint4*>(qrow[it] + kb * 8));
+            sz[it] = srow[it][kb >> 1];
+            sz[it] |= SYM ? 0x48000000u : (static_cast<uint32_t>(zrow[it][kb >> 1]) << 16);
+          }
         }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(full_b(s));
+      };
+      if (pdl_static == 0) pdl_wait();
+#pragma unroll
+      for (int d = 0; d < kLoadAhead; ++d) fetch(d, ring[d], ring_sz[d]);
+      bool stop = false;
+      for (int kb0 = 0; kb0 < num_kb && !stop; kb0 += kLoadAhead) {
+#pragma unroll
+        for (int d = 0; d < kLoadAhead; ++d) {
+          const int kb = kb0 + d;
+          if (kb >= num_kb) break;
+          const int s = kb % kStages;
+          const uint32_t ph = (kb / kStages) & 1u;
+          const uint4 cur[2] = {ring[d][0], ring[d][1]};
+          const uint32_t csz[2] = {ring_sz[d][0], ring_sz[d][1]};
+          fetch(kb + kLoadAhead, ring[d], ring_sz[d]);
+          DqConst dc[2];
+#pragma unroll
+          for (int it = 0; it < 2; ++it)
+            dc[it] = dq_const(__half2float(__ushort_as_half(static_cast<uint16_t>(csz[it] & 0xFFFFu))),
+                              __half2float(__ushort_as_half(static_cast<uint16_t>(csz[it] >> 16))));
+          if (!mbar_wait(empty(s), ph ^ 1u, abort_flag, err, kKernelIdGemm)) {
+            stop = true;
+            break;
+          }
+          const uint32_t tile = sB + s * kTileBBytes;
+#pragma unroll
+          for (int it = 0; it < 2; ++it) {
+            const uint32_t w4[4] = {cur[it].x, cur[it].y, cur[it].z, cur[it].w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              st_shared_v4(tile + sw128_offset(rows[it], 4 * half + j), dq_word(w4[j], dc[it]));
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(full_b(s));
+        }
       }
       if (pdl_static != 0) pdl_wait();
     }

@@ -1,23 +1,31 @@
 // Decode W4A16 GEMV: y[M, N] = x[M, K] . dequant(Wq)^T for M <= 16 (up to 64
-// with W4_LINEAR_FORCE_GEMV).  HBM-bound on the packed weight stream
-// (0.53125 B/weight asymmetric, 0.515625 symmetric).
+// with W4_LINEAR_FORCE_GEMV, in chunks of 16 tokens).  HBM-bound on the
+// packed weight stream (0.53125 B/weight asymmetric, 0.515625 symmetric).
 //
-// Each warp owns a 16-row weight tile and one K slice.  A lane loads 16
-// bytes (32 codes) of two rows per 128-channel group straight into
-// registers, dequantizes them to exact bf16 integers (q - zero) with one
-// mask/OR and one packed subtract per pair (the canonical nibble order puts
-// adjacent channels in nibbles i and i+4), and feeds them as the A fragment
-// of mma.m16n8k16 (rows = weights, columns = tokens).  The fp32 group result
-// is multiplied by the group scale and accumulated.  The K dimension is
-// split over the CTAs of a thread-block cluster; partial sums are reduced in
-// rank order through distributed shared memory by the rank-0 CTA (no global
-// scratch, deterministic).
+// A CTA owns 64 weight rows and one K slice (the K dimension is split over
+// the CTAs of a thread-block cluster).  One producer thread streams the
+// slice through a ring of shared-memory stages with TMA, one 128-channel
+// group per stage: the 64 x 64-byte tile of packed codes plus the matching
+// x tile (tokens x 128 channels, 128-byte swizzled).  Four consumer warps
+// take the groups in turn; for its group a warp turns all four 16-row tiles
+// into exact bf16 values 128 + q in registers (one mask/OR per pair of codes:
+// the canonical nibble order puts adjacent channels in nibbles i and i+4),
+// runs mma.m16n8k16 against the x fragments (rows = weights, columns =
+// tokens), removes (128 + zero) * sum_k x_k with one extra mma of all-ones
+// rows per group (shared by the four tiles) and adds scale * result to fp32
+// accumulators.  Partial sums are reduced across the four warps in shared
+// memory and across the cluster in rank order through distributed shared
+// memory (no global scratch; deterministic).
 //
 // Inside one group the mma's 16 reduction slots map to channels as follows:
-// lane t (= lane % 4) covers channels 32t..32t+31 of the group, step s
-// (0..7) uses channels 32t+4s..32t+4s+3, so the x operand of step s is the
-// two consecutive bf16 pairs at that offset and needs no permutation.
+// lane t (= lane % 4) covers channels 32t..32t+31 of the group and step s
+// (0..7) uses channels 32t+4s..32t+4s+3, so the x operand of step s is two
+// consecutive bf16 pairs and needs no permutation.
+//
+// Every wait is bounded; a CTA that gives up records it in the device error
+// word, drains its own TMA loads and returns.  No TMA multicast.
 #include <cooperative_groups.h>
+#include <cudaTypedefs.h>
 
 #include "w4_common.cuh"
 #include "w4_kernels.h"
@@ -28,219 +36,396 @@ namespace w4 {
 
 namespace {
 
-constexpr int kGemvWarps = 4;
-constexpr int kGemvRows = 16 * kGemvWarps;  // weight rows per CTA
-constexpr int kGemvUnroll = 4;              // groups of weights in flight
+constexpr int kRows = 64;                 // weight rows per CTA
+constexpr int kConsumerWarps = 4;
+constexpr int kThreads = 32 * (kConsumerWarps + 1);
+constexpr int kMaxSliceGroups = 40;       // groups per CTA slice (scale table)
+constexpr uint32_t kOnes = 0x3F803F80u;    // bf16x2 (1.0, 1.0)
+constexpr uint32_t kWTileBytes = kRows * 64;
+constexpr unsigned kKernelIdGemv = 1;
 
-__device__ __forceinline__ uint4 ld_weights(const uint32_t* p) {
+// Shared-memory layout of one CTA (identical on host and device).  The
+// ring holds min(max stages, groups of the slice) stages, so small slices
+// leave room for more CTAs per SM (and for the next kernel under PDL).
+struct GemvLayout {
+  uint32_t x_half, stage, ring, sz, red, part, bars, misc, total;
+  int stages;
+};
+
+__host__ __device__ inline GemvLayout gemv_layout(int nt, int gs_max) {
+  GemvLayout L;
+  const int tokens = 8 * nt;
+  L.x_half = tokens * 128;                      // tokens x 64 channels, bf16
+  L.stage = kWTileBytes + 2 * L.x_half;         // multiple of 1024
+  const int max_stages = 4;                     // 24-32 KB in flight per CTA
+  L.stages = gs_max < max_stages ? (gs_max < 1 ? 1 : gs_max) : max_stages;
+  L.ring = 0;
+  L.sz = L.ring + L.stages * L.stage;            // [64][gs_max] (scale | zero << 16)
+  L.red = L.sz + ((kRows * gs_max * 4 + 15) & ~15u);  // [4][tokens][64] f32
+  L.part = L.red + kConsumerWarps * tokens * kRows * 4;  // [tokens][64] f32
+  L.bars = L.part + tokens * kRows * 4;          // full[S], empty[S]
+  L.misc = L.bars + 2 * L.stages * 8;
+  L.total = L.misc + 16 + 1024;                  // + alignment slack
+  return L;
+}
+
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
   uint4 r;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
                : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
-               : "l"(p));
+               : "r"(addr));
   return r;
 }
 
-__device__ __forceinline__ uint4 ld_x(const __nv_bfloat16* p) {
-  return __ldg(reinterpret_cast<const uint4*>(p));
+// bf16x2 (128 + q_lo, 128 + q_hi) from the nibble pair at bits 0..3 / 16..19
+// of u (exact: bf16 has unit spacing on [128, 256)).
+__device__ __forceinline__ uint32_t code_pair(uint32_t u) {
+  return (u & 0x000F000Fu) | 0x43004300u;
 }
 
-// bf16x2 (q_lo - z, q_hi - z) from the nibble pair at bits 0..3 / 16..19 of u.
-__device__ __forceinline__ uint32_t dq_pair(uint32_t u, uint32_t zz) {
-  const uint32_t b = (u & 0x000F000Fu) | 0x43004300u;  // (128 + q) in each bf16 half
-  uint32_t r;
-  asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(b), "r"(zz));
-  return r;
-}
-
+// A pure register operation (not volatile), so the compiler may interleave
+// independent mma chains.
 __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
                                                uint32_t b1) {
-  asm volatile(
+  asm(
       "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
       "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-// bf16x2 with both halves equal to 128 + z (exact for integer z in 0..15).
-__device__ __forceinline__ uint32_t zz_of(float z) {
-  const uint32_t h = __bfloat16_as_ushort(__float2bfloat16_rn(128.0f + z));
-  return h | (h << 16);
+
+__device__ __forceinline__ void named_bar_consumers() {
+  asm volatile("bar.sync 1, %0;" ::"n"(32 * kConsumerWarps) : "memory");
 }
 
 template <int NT, bool SYM>
-__global__ void __launch_bounds__(kGemvWarps * 32)
-    gemv_w4a16_kernel(const __nv_bfloat16* __restrict__ x, const uint32_t* __restrict__ qw,
+__global__ void __launch_bounds__(kThreads, NT == 1 ? 4 : 2)
+    gemv_w4a16_kernel(const __grid_constant__ CUtensorMap tmap_w,   // uint8 [N, K/2], box 64x64
+                      const __grid_constant__ CUtensorMap tmap_x,   // bf16 [M, K], box 64 x tokens, SW128
                       const uint16_t* __restrict__ scales, const uint16_t* __restrict__ zeros,
                       __nv_bfloat16* __restrict__ y, int M, int N, int K, int ksplit,
-                      int static_weights) {
-  __shared__ float part[NT * 8][kGemvRows];  // [token][row] partial sums of this CTA
+                      int gs_max, int static_weights, unsigned* err) {
+  constexpr int kTokens = 8 * NT;
+  const GemvLayout L = gemv_layout(NT, gs_max);
+  const int S = L.stages;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  const uint32_t base = (raw_addr + 1023u) & ~1023u;
+  uint8_t* bp = smem_raw + (base - raw_addr);
+  uint32_t* s_sz = reinterpret_cast<uint32_t*>(bp + L.sz);
+  float* red = reinterpret_cast<float*>(bp + L.red);
+  float* part = reinterpret_cast<float*>(bp + L.part);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bp + L.misc);
+  const uint32_t bar0 = base + L.bars;
+  auto full = [&](int s) { return bar0 + 8u * s; };
+  auto empty = [&](int s) { return bar0 + 8u * (S + s); };
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int g = lane >> 2;
-  const int t = lane & 3;
   const int G = K >> 7;
-  const int row_blk = blockIdx.x * kGemvRows;
-  const int ra = row_blk + warp * 16 + g;  // rows of the A fragment
-  const int rb = ra + 8;
-  const bool va = ra < N, vb = rb < N;
+  const int row0 = blockIdx.x * kRows;
   const int rank = blockIdx.y;
   const int g_per = (G + ksplit - 1) / ksplit;
   const int g_begin = min(G, rank * g_per);
-  const int g_end = min(G, g_begin + g_per);
-  const size_t row_words = static_cast<size_t>(K) >> 3;
-  const uint32_t* qa = qw + static_cast<size_t>(va ? ra : 0) * row_words + 4 * t;
-  const uint32_t* qb = qw + static_cast<size_t>(vb ? rb : 0) * row_words + 4 * t;
+  const int gs = min(G, g_begin + g_per) - g_begin;
 
-  float acc[NT][4];
-#pragma unroll
-  for (int n = 0; n < NT; ++n)
-#pragma unroll
-    for (int i = 0; i < 4; ++i) acc[n][i] = 0.f;
-
-  uint4 wa[kGemvUnroll], wb[kGemvUnroll];
-  auto load_chunk = [&](int gr0) {
-#pragma unroll
-    for (int u = 0; u < kGemvUnroll; ++u) {
-      const int gr = gr0 + u;
-      wa[u] = make_uint4(0, 0, 0, 0);
-      wb[u] = make_uint4(0, 0, 0, 0);
-      if (gr < g_end) {
-        if (va) wa[u] = ld_weights(qa + static_cast<size_t>(gr) * 16);
-        if (vb) wb[u] = ld_weights(qb + static_cast<size_t>(gr) * 16);
-      }
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(full(s), 1);
+      mbar_init(empty(s), 1);
     }
-  };
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  // Dependents may launch now: their weight prefetch overlaps this kernel.
+  pdl_launch_dependents();
 
-  // With static weights the first chunk streams in before the dependency
-  // wait of a programmatic dependent launch; x and y are only touched after.
-  if (static_weights) load_chunk(g_begin);
-  pdl_wait();
-  if (!static_weights) load_chunk(g_begin);
-
-  for (int gr0 = g_begin; gr0 < g_end; gr0 += kGemvUnroll) {
-    if (gr0 != g_begin) load_chunk(gr0);
-#pragma unroll
-    for (int u = 0; u < kGemvUnroll; ++u) {
-      const int gr = gr0 + u;
-      if (gr >= g_end) break;
-      float sa = 0.f, sb = 0.f, za = 8.f, zb = 8.f;
-      if (va) {
-        sa = __half2float(__ushort_as_half(scales[static_cast<size_t>(ra) * G + gr]));
-        if (!SYM) za = __half2float(__ushort_as_half(zeros[static_cast<size_t>(ra) * G + gr]));
+  if (warp == kConsumerWarps) {
+    // ------------------------------------------------------- producer ----
+    if (lane == 0) {
+      tma_prefetch_desc(&tmap_w);
+      tma_prefetch_desc(&tmap_x);
+      const uint32_t stage_tx = L.stage;
+      // Stages whose weight tile was issued before the dependency wait.
+      const int pre = static_weights ? min(gs, S) : 0;
+      for (int i = 0; i < pre; ++i) {
+        const uint32_t st = base + L.ring + i * L.stage;
+        mbar_arrive_expect_tx(full(i), stage_tx);
+        tma_load_2d(st, &tmap_w, (g_begin + i) * 64, row0, full(i));
       }
-      if (vb) {
-        sb = __half2float(__ushort_as_half(scales[static_cast<size_t>(rb) * G + gr]));
-        if (!SYM) zb = __half2float(__ushort_as_half(zeros[static_cast<size_t>(rb) * G + gr]));
+      pdl_wait();
+      int issued = 0;
+      for (int i = 0; i < gs; ++i) {
+        const int s = i % S;
+        const uint32_t st = base + L.ring + s * L.stage;
+        const int gr = g_begin + i;
+        if (i >= pre) {
+          if (!mbar_wait(empty(s), ((i / S) & 1u) ^ 1u, abort_flag, err, kKernelIdGemv))
+            break;
+          mbar_arrive_expect_tx(full(s), stage_tx);
+          tma_load_2d(st, &tmap_w, gr * 64, row0, full(s));
+        }
+        tma_load_2d(st + kWTileBytes, &tmap_x, gr * 128, 0, full(s));
+        tma_load_2d(st + kWTileBytes + L.x_half, &tmap_x, gr * 128 + 64, 0, full(s));
+        issued = i + 1;
       }
-      const uint32_t zza = zz_of(za), zzb = zz_of(zb);
-      // x fragments: token 8n + g, channels 32t .. 32t+31 of the group.
-      uint4 xv[NT][4];
-#pragma unroll
-      for (int n = 0; n < NT; ++n) {
-        const int m = 8 * n + g;
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          xv[n][j] = make_uint4(0, 0, 0, 0);
-          if (m < M) xv[n][j] = ld_x(x + static_cast<size_t>(m) * K + gr * 128 + 32 * t + 8 * j);
+      if (*abort_flag) {  // drain this CTA's own loads before leaving
+        for (int i = max(0, issued - S); i < issued; ++i) {
+          volatile int dummy = 0;
+          mbar_wait(full(i % S), (i / S) & 1u, &dummy, err, kKernelIdGemv,
+                    kWaitLimitNs / 4);
         }
       }
-      const uint32_t va4[4] = {wa[u].x, wa[u].y, wa[u].z, wa[u].w};
-      const uint32_t vb4[4] = {wb[u].x, wb[u].y, wb[u].z, wb[u].w};
-      float c[NT][4];
+    }
+  } else {
+    // ------------------------------------------------------- consumers ---
+    const int g = lane >> 2;
+    const int t = lane & 3;
+    // (scale | zero << 16) of this CTA's rows and groups into shared memory.
+    // Thread j owns row j / 2 and every other group of it; all its loads are
+    // issued before any is used, so the table costs one memory latency.
+    if (!static_weights) pdl_wait();
+    {
+      const int r = threadIdx.x >> 1;
+      const int row = row0 + r;
+      const bool rv = row < N;
+      const size_t gbase = static_cast<size_t>(rv ? row : 0) * G + g_begin;
+      uint32_t sv[kMaxSliceGroups / 2], zv[kMaxSliceGroups / 2];
+#pragma unroll
+      for (int j = 0; j < kMaxSliceGroups / 2; ++j) {
+        const int q = 2 * j + (threadIdx.x & 1);
+        sv[j] = 0u;
+        zv[j] = 0x4800u;  // zero 8 (symmetric)
+        if (rv && q < gs) {
+          sv[j] = __ldg(scales + gbase + q);
+          if (!SYM) zv[j] = __ldg(zeros + gbase + q);
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < kMaxSliceGroups / 2; ++j) {
+        const int q = 2 * j + (threadIdx.x & 1);
+        if (q < gs) s_sz[r * gs_max + q] = sv[j] | (zv[j] << 16);
+      }
+    }
+    named_bar_consumers();
+
+    float acc[4][NT][4];
+#pragma unroll
+    for (int rt = 0; rt < 4; ++rt)
 #pragma unroll
       for (int n = 0; n < NT; ++n)
 #pragma unroll
-        for (int i = 0; i < 4; ++i) c[n][i] = 0.f;
+        for (int i = 0; i < 4; ++i) acc[rt][n][i] = 0.f;
+
+    for (int i = warp; i < gs; i += kConsumerWarps) {
+      const int s = i % S;
+      if (!mbar_wait(full(s), (i / S) & 1u, abort_flag, err, kKernelIdGemv)) break;
+      const uint32_t st = base + L.ring + s * L.stage;
+      // x fragments: token 8n + g, channels 32t + 8j .. +7 (128B-swizzled halves).
+      uint4 xv[NT][4];
 #pragma unroll
-      for (int s = 0; s < 8; ++s) {
-        const int w = s >> 1;
-        const int sh = 8 * (s & 1);  // pair 2(s&1) -> shift 4*i
-        uint32_t a[4];
-        a[0] = dq_pair(va4[w] >> sh, zza);
-        a[1] = dq_pair(vb4[w] >> sh, zzb);
-        a[2] = dq_pair(va4[w] >> (sh + 4), zza);
-        a[3] = dq_pair(vb4[w] >> (sh + 4), zzb);
+      for (int n = 0; n < NT; ++n)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const uint32_t c = 4 * (t & 1) + j;
+          xv[n][j] = lds128(st + kWTileBytes + (t >> 1) * L.x_half + (8 * n + g) * 128 +
+                            ((c ^ g) << 4));
+        }
+      uint4 wv[4][2];
+#pragma unroll
+      for (int rt = 0; rt < 4; ++rt) {
+        wv[rt][0] = lds128(st + (16 * rt + g) * 64 + 16 * t);
+        wv[rt][1] = lds128(st + (16 * rt + g + 8) * 64 + 16 * t);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(empty(s));  // the stage's data is in registers
+      // Per-token sums of x over the group (an mma against all-ones rows):
+      // sum_k (q - z) x_k = sum_k (128 + q) x_k - (128 + z) sum_k x_k.
+      // Reduction steps outermost, tiles innermost: consecutive mmas belong
+      // to independent accumulator chains.
+      float xs[NT][4];
+      float c[4][NT][4];
+#pragma unroll
+      for (int n = 0; n < NT; ++n)
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          xs[n][k] = 0.f;
+#pragma unroll
+          for (int rt = 0; rt < 4; ++rt) c[rt][n][k] = 0.f;
+        }
+      const uint32_t ones[4] = {kOnes, kOnes, kOnes, kOnes};
+#pragma unroll
+      for (int sp = 0; sp < 8; ++sp) {
+        const int w = sp >> 1;
+        const int sh = 8 * (sp & 1);  // pair 2(sp&1) -> shift 4*pair
+#pragma unroll
+        for (int rt = 0; rt < 4; ++rt) {
+          const uint32_t va = (w == 0 ? wv[rt][0].x : w == 1 ? wv[rt][0].y : w == 2 ? wv[rt][0].z : wv[rt][0].w);
+          const uint32_t vb = (w == 0 ? wv[rt][1].x : w == 1 ? wv[rt][1].y : w == 2 ? wv[rt][1].z : wv[rt][1].w);
+          uint32_t a[4];
+          a[0] = code_pair(va >> sh);
+          a[1] = code_pair(vb >> sh);
+          a[2] = code_pair(va >> (sh + 4));
+          a[3] = code_pair(vb >> (sh + 4));
+#pragma unroll
+          for (int n = 0; n < NT; ++n) {
+            const uint4 xx = xv[n][w];
+            mma_bf16_16816(c[rt][n], a, (sp & 1) ? xx.z : xx.x, (sp & 1) ? xx.w : xx.y);
+          }
+        }
 #pragma unroll
         for (int n = 0; n < NT; ++n) {
           const uint4 xx = xv[n][w];
-          const uint32_t b0 = (s & 1) ? xx.z : xx.x;
-          const uint32_t b1 = (s & 1) ? xx.w : xx.y;
-          mma_bf16_16816(c[n], a, b0, b1);
+          mma_bf16_16816(xs[n], ones, (sp & 1) ? xx.z : xx.x, (sp & 1) ? xx.w : xx.y);
         }
       }
 #pragma unroll
-      for (int n = 0; n < NT; ++n) {
-        acc[n][0] = fmaf(sa, c[n][0], acc[n][0]);
-        acc[n][1] = fmaf(sa, c[n][1], acc[n][1]);
-        acc[n][2] = fmaf(sb, c[n][2], acc[n][2]);
-        acc[n][3] = fmaf(sb, c[n][3], acc[n][3]);
+      for (int rt = 0; rt < 4; ++rt) {
+        const uint32_t sza = s_sz[(16 * rt + g) * gs_max + i];
+        const uint32_t szb = s_sz[(16 * rt + g + 8) * gs_max + i];
+        const float sa = __half2float(__ushort_as_half(static_cast<uint16_t>(sza & 0xFFFFu)));
+        const float sb = __half2float(__ushort_as_half(static_cast<uint16_t>(szb & 0xFFFFu)));
+        const float za = 128.0f + __half2float(__ushort_as_half(static_cast<uint16_t>(sza >> 16)));
+        const float zb = 128.0f + __half2float(__ushort_as_half(static_cast<uint16_t>(szb >> 16)));
+#pragma unroll
+        for (int n = 0; n < NT; ++n) {
+          acc[rt][n][0] = fmaf(sa, fmaf(-za, xs[n][0], c[rt][n][0]), acc[rt][n][0]);
+          acc[rt][n][1] = fmaf(sa, fmaf(-za, xs[n][1], c[rt][n][1]), acc[rt][n][1]);
+          acc[rt][n][2] = fmaf(sb, fmaf(-zb, xs[n][2], c[rt][n][2]), acc[rt][n][2]);
+          acc[rt][n][3] = fmaf(sb, fmaf(-zb, xs[n][3], c[rt][n][3]), acc[rt][n][3]);
+        }
       }
     }
-  }
-
-  // Let the next kernel on the stream begin its prologue.
-  pdl_launch_dependents();
-
-  // Stage this CTA's partial sums: token 8n + 2t + {0,1}, rows ra / rb.
-  const int lr = warp * 16 + g;
+    pdl_wait();  // (no-op when already satisfied) before this CTA writes y
+    // This warp's partial sums: token 8n + 2t + {0,1}, rows 16rt + g (+8).
+    float* rw = red + warp * kTokens * kRows;
 #pragma unroll
-  for (int n = 0; n < NT; ++n) {
-    part[8 * n + 2 * t][lr] = acc[n][0];
-    part[8 * n + 2 * t + 1][lr] = acc[n][1];
-    part[8 * n + 2 * t][lr + 8] = acc[n][2];
-    part[8 * n + 2 * t + 1][lr + 8] = acc[n][3];
+    for (int rt = 0; rt < 4; ++rt)
+#pragma unroll
+      for (int n = 0; n < NT; ++n) {
+        const int r = 16 * rt + g;
+        rw[(8 * n + 2 * t) * kRows + r] = acc[rt][n][0];
+        rw[(8 * n + 2 * t + 1) * kRows + r] = acc[rt][n][1];
+        rw[(8 * n + 2 * t) * kRows + r + 8] = acc[rt][n][2];
+        rw[(8 * n + 2 * t + 1) * kRows + r + 8] = acc[rt][n][3];
+      }
+    named_bar_consumers();
+    for (int e = threadIdx.x; e < kTokens * kRows; e += 32 * kConsumerWarps)
+      part[e] = ((red[e] + red[kTokens * kRows + e]) + red[2 * kTokens * kRows + e]) +
+                red[3 * kTokens * kRows + e];
   }
 
   if (ksplit > 1) {
     cg::cluster_group cluster = cg::this_cluster();
     cluster.sync();
-    if (rank == 0) {
-      for (int e = threadIdx.x; e < NT * 8 * kGemvRows; e += kGemvWarps * 32) {
-        const int m = e / kGemvRows;
-        const int r = e % kGemvRows;
+    if (rank == 0 && warp < kConsumerWarps && !*abort_flag) {
+      for (int e = threadIdx.x; e < kTokens * kRows; e += 32 * kConsumerWarps) {
+        const int m = e / kRows;
+        const int r = e % kRows;
         float sum = 0.f;
-        for (int q = 0; q < ksplit; ++q) {
-          const float* rp = cluster.map_shared_rank(&part[0][0], q);
-          sum += rp[m * kGemvRows + r];
-        }
-        const int n_out = row_blk + r;
+        for (int q = 0; q < ksplit; ++q) sum += cluster.map_shared_rank(part, q)[e];
+        const int n_out = row0 + r;
         if (m < M && n_out < N) y[static_cast<size_t>(m) * N + n_out] = __float2bfloat16_rn(sum);
       }
     }
     cluster.sync();  // peers keep their shared memory alive until rank 0 is done
   } else {
     __syncthreads();
-    for (int e = threadIdx.x; e < NT * 8 * kGemvRows; e += kGemvWarps * 32) {
-      const int m = e / kGemvRows;
-      const int r = e % kGemvRows;
-      const int n_out = row_blk + r;
-      if (m < M && n_out < N)
-        y[static_cast<size_t>(m) * N + n_out] = __float2bfloat16_rn(part[m][r]);
+    if (warp < kConsumerWarps && !*abort_flag) {
+      for (int e = threadIdx.x; e < kTokens * kRows; e += 32 * kConsumerWarps) {
+        const int m = e / kRows;
+        const int r = e % kRows;
+        const int n_out = row0 + r;
+        if (m < M && n_out < N) y[static_cast<size_t>(m) * N + n_out] = __float2bfloat16_rn(part[e]);
+      }
     }
   }
+}
+
+CUresult encode_2d(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uint64_t inner,
+                   uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
+                   CUtensorMapSwizzle swz) {
+  static PFN_cuTensorMapEncodeTiled fn = nullptr;
+  if (!fn) {
+    cudaDriverEntryPointQueryResult q;
+    void* p = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || !p)
+      return CUDA_ERROR_NOT_FOUND;
+    fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled>(p);
+  }
+  const uint64_t dims[2] = {inner, outer};
+  const uint64_t strides[1] = {row_bytes};
+  const uint32_t box[2] = {box_inner, box_outer};
+  const uint32_t estr[2] = {1, 1};
+  return fn(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
 }
 
 template <int NT, bool SYM>
 cudaError_t launch_gemv_t(const void* x, int M, const int32_t* qw, const uint16_t* sc,
                           const uint16_t* z, int N, int K, void* y, bool pdl, bool static_w,
-                          cudaStream_t stream, int num_sms) {
+                          cudaStream_t stream, int num_sms, unsigned* err) {
+  constexpr int kTokens = 8 * NT;
   const int G = K / 128;
-  const int row_blocks = (N + kGemvRows - 1) / kGemvRows;
+  const int row_blocks = (N + kRows - 1) / kRows;
+  auto kern = gemv_w4a16_kernel<NT, SYM>;
+  // Opt in once per device to the largest layout this kernel can use, and
+  // record how many CTAs of it an SM holds.
+  static unsigned long long attr_done = 0;  // bit d: device d
+  static int per_sm[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev >= 64 || !(__atomic_load_n(&attr_done, __ATOMIC_ACQUIRE) & (1ull << dev))) {
+    const int max_smem = static_cast<int>(gemv_layout(NT, kMaxSliceGroups).total);
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, max_smem);
+    if (e != cudaSuccess) return e;
+    int nb = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, kern, kThreads, max_smem);
+    if (e != cudaSuccess) return e;
+    if (dev < 64) {
+      per_sm[dev] = nb < 1 ? 1 : nb;
+      __atomic_fetch_or(&attr_done, 1ull << dev, __ATOMIC_RELEASE);
+    }
+  }
+  const int capacity = num_sms * (dev < 64 ? per_sm[dev] : 1);
+  // Split K over a cluster as far as the grid still fits in one wave and
+  // every CTA keeps at least two groups; the CTA's K slice must fit the
+  // shared scale table.
   int ks = 1;
-  while (ks < 8 && row_blocks * ks < 2 * num_sms && G / (ks * 2) >= 2) ks *= 2;
+  while (ks < 8 && row_blocks * ks * 2 <= capacity && G / (ks * 2) >= 2) ks *= 2;
+  while ((G + ks - 1) / ks > kMaxSliceGroups && ks < 8) ks *= 2;
+  if ((G + ks - 1) / ks > kMaxSliceGroups) return cudaErrorInvalidValue;
+  const int gs_max = (G + ks - 1) / ks;
+  const GemvLayout L = gemv_layout(NT, gs_max);
+
+  CUtensorMap tw, tx;
+  if (encode_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, qw, static_cast<uint64_t>(K) / 2, N,
+                static_cast<uint64_t>(K) / 2, 64, kRows, CU_TENSOR_MAP_SWIZZLE_NONE) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+  if (encode_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, K, M, static_cast<uint64_t>(K) * 2, 64,
+                kTokens, CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(row_blocks, ks, 1);
-  cfg.blockDim = dim3(kGemvWarps * 32, 1, 1);
-  cfg.dynamicSmemBytes = 0;
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = L.total;
   cfg.stream = stream;
   cudaLaunchAttribute attrs[2];
   int na = 0;
-  attrs[na].id = cudaLaunchAttributeClusterDimension;
-  attrs[na].val.clusterDim.x = 1;
-  attrs[na].val.clusterDim.y = ks;
-  attrs[na].val.clusterDim.z = 1;
-  ++na;
+  if (ks > 1) {
+    attrs[na].id = cudaLaunchAttributeClusterDimension;
+    attrs[na].val.clusterDim.x = 1;
+    attrs[na].val.clusterDim.y = ks;
+    attrs[na].val.clusterDim.z = 1;
+    ++na;
+  }
   if (pdl) {
     attrs[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attrs[na].val.programmaticStreamSerializationAllowed = 1;
@@ -248,18 +433,15 @@ cudaError_t launch_gemv_t(const void* x, int M, const int32_t* qw, const uint16_
   }
   cfg.attrs = attrs;
   cfg.numAttrs = na;
-  return cudaLaunchKernelEx(&cfg, gemv_w4a16_kernel<NT, SYM>,
-                            static_cast<const __nv_bfloat16*>(x),
-                            reinterpret_cast<const uint32_t*>(qw), sc, z,
-                            static_cast<__nv_bfloat16*>(y), M, N, K, ks,
-                            static_cast<int>(pdl && static_w));
+  return cudaLaunchKernelEx(&cfg, kern, tw, tx, sc, z, static_cast<__nv_bfloat16*>(y), M, N, K,
+                            ks, gs_max, static_cast<int>(pdl && static_w), err);
 }
 
 }  // namespace
 
 cudaError_t launch_gemv(const void* x, int M, const int32_t* qw, const uint16_t* sc,
                         const uint16_t* z, int N, int K, void* y, bool pdl, bool static_w,
-                        cudaStream_t stream, int num_sms) {
+                        cudaStream_t stream, int num_sms, unsigned* err) {
   const bool sym = (z == nullptr);
   // M <= 64 in chunks of up to 16 tokens (two n-tiles of 8).
   for (int m0 = 0; m0 < M; m0 += 16) {
@@ -268,11 +450,11 @@ cudaError_t launch_gemv(const void* x, int M, const int32_t* qw, const uint16_t*
     void* yc = static_cast<__nv_bfloat16*>(y) + static_cast<size_t>(m0) * N;
     cudaError_t e;
     if (mc <= 8) {
-      e = sym ? launch_gemv_t<1, true>(xc, mc, qw, sc, z, N, K, yc, pdl, static_w, stream, num_sms)
-              : launch_gemv_t<1, false>(xc, mc, qw, sc, z, N, K, yc, pdl, static_w, stream, num_sms);
+      e = sym ? launch_gemv_t<1, true>(xc, mc, qw, sc, z, N, K, yc, pdl, static_w, stream, num_sms, err)
+              : launch_gemv_t<1, false>(xc, mc, qw, sc, z, N, K, yc, pdl, static_w, stream, num_sms, err);
     } else {
-      e = sym ? launch_gemv_t<2, true>(xc, mc, qw, sc, z, N, K, yc, pdl, static_w, stream, num_sms)
-              : launch_gemv_t<2, false>(xc, mc, qw, sc, z, N, K, yc, pdl, static_w, stream, num_sms);
+      e = sym ? launch_gemv_t<2, true>(xc, mc, qw, sc, z, N, K, yc, pdl, static_w, stream, num_sms, err)
+              : launch_gemv_t<2, false>(xc, mc, qw, sc, z, N, K, yc, pdl, static_w, stream, num_sms, err);
     }
     if (e != cudaSuccess) return e;
   }

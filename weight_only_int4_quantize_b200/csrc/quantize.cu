@@ -3,11 +3,10 @@
 //
 // HBM-bound: 2 bytes read and 0.5 + 4/128 (asymmetric) bytes written per
 // weight.  The weight is a sequence of N*K/128 contiguous 256-byte groups;
-// each half warp owns one group per step, each lane one 16-byte vector of 8
-// values, so loads are fully coalesced 16-byte vectors and the 16 packed
-// words of a group are one contiguous 64-byte store.  Group min/max use
-// half-warp shuffles; codes use the division-free exact rounding of
-// quant_group.cuh.
+// a lane quad owns one group per step, each lane 64 contiguous bytes (32
+// values), so a warp reads 2 KB of consecutive memory and the 16 packed
+// words of a group are four contiguous 16-byte stores.  Group min/max use
+// quad shuffles (on packed bf16 pairs when no AWQ scale is applied).
 #include "quant_group.cuh"
 #include "w4_kernels.h"
 
@@ -16,72 +15,216 @@ namespace w4 {
 namespace {
 
 constexpr int kQuantThreads = 256;
-constexpr int kQuantUnroll = 4;  // groups in flight per half warp
 
 __device__ __forceinline__ uint4 ld_stream(const uint4* p) {
   uint4 r;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+  asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
                : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
                : "l"(p));
   return r;
 }
 
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
+  float2 r;
+  asm("mul.rn.f32x2 %0, %1, %2;"
+      : "=l"(*reinterpret_cast<unsigned long long*>(&r))
+      : "l"(*reinterpret_cast<unsigned long long*>(&a)),
+        "l"(*reinterpret_cast<unsigned long long*>(&b)));
+  return r;
+}
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+  float2 r;
+  asm("add.rn.f32x2 %0, %1, %2;"
+      : "=l"(*reinterpret_cast<unsigned long long*>(&r))
+      : "l"(*reinterpret_cast<unsigned long long*>(&a)),
+        "l"(*reinterpret_cast<unsigned long long*>(&b)));
+  return r;
+}
+__device__ __forceinline__ float2 sub2(float2 a, float2 b) {
+  float2 r;
+  asm("sub.rn.f32x2 %0, %1, %2;"
+      : "=l"(*reinterpret_cast<unsigned long long*>(&r))
+      : "l"(*reinterpret_cast<unsigned long long*>(&a)),
+        "l"(*reinterpret_cast<unsigned long long*>(&b)));
+  return r;
+}
+__device__ __forceinline__ uint32_t clamp_codes_s16x2(uint32_t p) {
+  uint32_t r;
+  asm("max.s16x2 %0, %1, %2;" : "=r"(r) : "r"(p), "r"(0u));
+  asm("min.s16x2 %0, %1, %2;" : "=r"(r) : "r"(r), "r"(0x000F000Fu));
+  return r;
+}
+
+// Reduction over the 4 lanes of a lane quad.
+__device__ __forceinline__ float quad_max(float a) {
+  a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 2));
+  return fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 1));
+}
+__device__ __forceinline__ float quad_min(float a) {
+  a = fminf(a, __shfl_xor_sync(0xffffffffu, a, 2));
+  return fminf(a, __shfl_xor_sync(0xffffffffu, a, 1));
+}
+__device__ __forceinline__ uint32_t bmax2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("max.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+__device__ __forceinline__ uint32_t bmin2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("min.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
+// One group = 128 contiguous values held by a lane quad, 32 per lane
+// (channels 32*l4 .. 32*l4+31 of the group, in adjacent pairs).  A warp
+// quantizes eight consecutive groups per iteration.
+//
+// Codes, fast path: with t = v * fl(1/scale) and Mz = 1.5*2^23 + zero,
+// fl(t + Mz) = Mz + rint(t) whenever t is not within 2^-16 of a half-integer
+// tie (so the tie-breaking parity of Mz never matters), and its low 16 bits
+// are rint(t) + zero as a signed 16-bit integer (|t| < 2^14 is checked per
+// group).  Two such codes are packed into one register, clamped to 0..15 with
+// packed 16-bit min/max, and in the canonical nibble order the pair of
+// adjacent channels (2i, 2i+1) belongs in nibbles (i, i+4): one shift by 4i.
+// t lies within 1.5 * 2^-23 * |v/scale| of the exact quotient, so for
+// |t| < 17 a distance above 2^-16 from every tie guarantees
+// rint(fl(v/scale)) == rint(t); for |t| >= 17 the clamp saturates either way.
+// Any lane with a value closer to a tie sends the whole warp through the
+// exact path (correctly rounded division, as in quant_group.cuh).
 template <bool SYM, bool HAS_S>
-__global__ void __launch_bounds__(kQuantThreads)
+__global__ void __launch_bounds__(kQuantThreads, 3)
     quantize_pack_kernel(const uint4* __restrict__ w, const float* __restrict__ s, float shrink,
-                         int64_t n_groups, int64_t groups_per_row, uint32_t* __restrict__ qw,
+                         int64_t n_groups, int64_t groups_per_row, uint4* __restrict__ qw,
                          uint16_t* __restrict__ scales, uint16_t* __restrict__ zeros) {
   const int lane = threadIdx.x & 31;
-  const int half = lane >> 4;
-  const int l16 = lane & 15;
+  const int sub = lane >> 2;  // group of this quad within the warp's eight
+  const int l4 = lane & 3;
   const int64_t warp = (static_cast<int64_t>(blockIdx.x) * kQuantThreads + threadIdx.x) >> 5;
   const int64_t n_warps = (static_cast<int64_t>(gridDim.x) * kQuantThreads) >> 5;
-  // Warp unit u covers groups 2u and 2u+1; the loop bound is warp-uniform.
-  const int64_t n_units = (n_groups + 1) >> 1;
+  const int64_t n_units = (n_groups + 7) >> 3;
+  const float thr = 0.5f - 1.52587890625e-05f;  // 0.5 - 2^-16
 
-  for (int64_t u0 = warp; u0 < n_units; u0 += n_warps * kQuantUnroll) {
-    uint4 raw[kQuantUnroll];
-    int64_t gi[kQuantUnroll];
+  // Software pipeline: the next unit's 64 bytes per lane are in flight while
+  // the current unit is quantized.
+  auto load_unit = [&](int64_t u, uint32_t (&dst)[16]) {
+    const int64_t gi = 8 * u + sub;
+    const uint4* src = w + gi * 16 + l4 * 4;
 #pragma unroll
-    for (int i = 0; i < kQuantUnroll; ++i) {
-      gi[i] = 2 * (u0 + i * n_warps) + half;
-      raw[i] = make_uint4(0, 0, 0, 0);
-      if (gi[i] < n_groups) raw[i] = ld_stream(w + gi[i] * 16 + l16);
+    for (int q = 0; q < 4; ++q) {
+      const uint4 r = (u < n_units && gi < n_groups) ? ld_stream(src + q) : make_uint4(0, 0, 0, 0);
+      dst[4 * q] = r.x; dst[4 * q + 1] = r.y; dst[4 * q + 2] = r.z; dst[4 * q + 3] = r.w;
     }
+  };
+  uint32_t nxt[16];
+  load_unit(warp, nxt);
+  for (int64_t u = warp; u < n_units; u += n_warps) {
+    const int64_t gi = 8 * u + sub;
+    const bool valid = gi < n_groups;
+    uint32_t raw[16];
 #pragma unroll
-    for (int i = 0; i < kQuantUnroll; ++i) {
-      if (u0 + i * n_warps >= n_units) break;  // warp-uniform
-      float v[8];
-      bf16x8_to_f32(raw[i], v);
-      if (HAS_S) {
-        const int64_t k0 = (gi[i] % groups_per_row) * 128 + l16 * 8;
-        const float4 s0 = __ldg(reinterpret_cast<const float4*>(s + k0));
-        const float4 s1 = __ldg(reinterpret_cast<const float4*>(s + k0 + 4));
-        v[0] = __fmul_rn(v[0], s0.x); v[1] = __fmul_rn(v[1], s0.y);
-        v[2] = __fmul_rn(v[2], s0.z); v[3] = __fmul_rn(v[3], s0.w);
-        v[4] = __fmul_rn(v[4], s1.x); v[5] = __fmul_rn(v[5], s1.y);
-        v[6] = __fmul_rn(v[6], s1.z); v[7] = __fmul_rn(v[7], s1.w);
+    for (int p = 0; p < 16; ++p) raw[p] = nxt[p];
+    load_unit(u + n_warps, nxt);
+    float2 v[16];
+#pragma unroll
+    for (int p = 0; p < 16; ++p)
+      v[p] = make_float2(__uint_as_float(raw[p] << 16), __uint_as_float(raw[p] & 0xFFFF0000u));
+    GroupQ g;
+    float amax;
+    if (HAS_S) {
+      const int64_t k0 = (gi % groups_per_row) * 128 + l4 * 32;
+      const float4* sp = reinterpret_cast<const float4*>(s + (valid ? k0 : 0));
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const float4 sv = __ldg(sp + q);
+        v[2 * q] = mul2(v[2 * q], make_float2(sv.x, sv.y));
+        v[2 * q + 1] = mul2(v[2 * q + 1], make_float2(sv.z, sv.w));
       }
-      GroupQ g;
       if (SYM) {
-        float a = fabsf(v[0]);
+        float a = 0.f;
 #pragma unroll
-        for (int j = 1; j < 8; ++j) a = fmaxf(a, fabsf(v[j]));
-        g = group_params<true>(hw_max(a), 0.f, shrink);
+        for (int p = 0; p < 16; ++p) a = fmaxf(a, fmaxf(fabsf(v[p].x), fabsf(v[p].y)));
+        amax = quad_max(a);
+        g = group_params<true>(amax, 0.f, shrink);
       } else {
-        float mx = v[0], mn = v[0];
+        float mx = v[0].x, mn = v[0].x;
 #pragma unroll
-        for (int j = 1; j < 8; ++j) { mx = fmaxf(mx, v[j]); mn = fminf(mn, v[j]); }
-        g = group_params<false>(hw_max(mx), hw_min(mn), shrink);
+        for (int p = 0; p < 16; ++p) {
+          mx = fmaxf(mx, fmaxf(v[p].x, v[p].y));
+          mn = fminf(mn, fminf(v[p].x, v[p].y));
+        }
+        mx = quad_max(mx);
+        mn = quad_min(mn);
+        g = group_params<false>(mx, mn, shrink);
+        amax = fmaxf(fabsf(mx), fabsf(mn));
       }
-      uint32_t word = 0;
+    } else {
+      // Group statistics on the raw bf16 pairs (exact: max/min only compare).
+      uint32_t bx = raw[0], bn = raw[0];
+      if (SYM) {
 #pragma unroll
-      for (int j = 0; j < 8; ++j) word |= code_of(v[j], g) << (4 * nibble_pos(j));
-      if (gi[i] < n_groups) {
-        qw[gi[i] * 16 + l16] = word;
-        if (l16 == 0) {
-          scales[gi[i]] = g.s16;
-          if (!SYM) zeros[gi[i]] = g.z16;
+        for (int p = 0; p < 16; ++p) bx = bmax2(bx, raw[p] & 0x7FFF7FFFu);
+      } else {
+#pragma unroll
+        for (int p = 1; p < 16; ++p) {
+          bx = bmax2(bx, raw[p]);
+          bn = bmin2(bn, raw[p]);
+        }
+      }
+      const float mx = quad_max(fmaxf(__uint_as_float(bx << 16), __uint_as_float(bx & 0xFFFF0000u)));
+      if (SYM) {
+        amax = mx;
+        g = group_params<true>(amax, 0.f, shrink);
+      } else {
+        const float mn =
+            quad_min(fminf(__uint_as_float(bn << 16), __uint_as_float(bn & 0xFFFF0000u)));
+        g = group_params<false>(mx, mn, shrink);
+        amax = fmaxf(fabsf(mx), fabsf(mn));
+      }
+    }
+    // Fast path.
+    const float mz = 12582912.0f + g.zero;  // exact
+    const float2 rcp2 = make_float2(g.rcp, g.rcp);
+    const float2 mz2 = make_float2(mz, mz);
+    float dmax = 0.f;
+    uint32_t word[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+    for (int p = 0; p < 16; ++p) {
+      const float2 t = mul2(v[p], rcp2);
+      const float2 r = add2(t, mz2);
+      const float2 d = sub2(t, sub2(r, mz2));
+      dmax = fmaxf(dmax, fmaxf(fabsf(d.x), fabsf(d.y)));
+      const uint32_t pair = __byte_perm(__float_as_uint(r.x), __float_as_uint(r.y), 0x5410);
+      word[p >> 2] += clamp_codes_s16x2(pair) << (4 * (p & 3));
+    }
+    const bool bad = !(dmax < thr) || !(__fmul_rn(amax, g.rcp) < 16384.0f);
+    if (__any_sync(0xffffffffu, bad)) {
+      // Exact path for the whole warp (rare).
+#pragma unroll
+      for (int p = 0; p < 16; ++p) {
+        if ((p & 3) == 0) word[p >> 2] = 0u;
+        const uint32_t c0 = code_of(v[p].x, g), c1 = code_of(v[p].y, g);
+        word[p >> 2] |= (c0 | (c1 << 16)) << (4 * (p & 3));
+      }
+    }
+    // Scales / zeros of the eight groups: gathered into lanes 0 and 16.
+    const uint32_t sz = static_cast<uint32_t>(g.s16) | (static_cast<uint32_t>(g.z16) << 16);
+    const uint32_t sz1 = __shfl_down_sync(0xffffffffu, sz, 4);
+    const uint32_t sz2 = __shfl_down_sync(0xffffffffu, sz, 8);
+    const uint32_t sz3 = __shfl_down_sync(0xffffffffu, sz, 12);
+    if (valid) qw[gi * 4 + l4] = make_uint4(word[0], word[1], word[2], word[3]);
+    if ((lane & 15) == 0) {
+      const int64_t g0 = gi;  // first of four consecutive groups
+      if (g0 + 3 < n_groups) {
+        *reinterpret_cast<uint2*>(scales + g0) =
+            make_uint2((sz & 0xFFFFu) | (sz1 << 16), (sz2 & 0xFFFFu) | (sz3 << 16));
+        if (!SYM)
+          *reinterpret_cast<uint2*>(zeros + g0) =
+              make_uint2((sz >> 16) | (sz1 & 0xFFFF0000u), (sz2 >> 16) | (sz3 & 0xFFFF0000u));
+      } else {
+        const uint32_t all[4] = {sz, sz1, sz2, sz3};
+        for (int q = 0; q < 4 && g0 + q < n_groups; ++q) {
+          scales[g0 + q] = static_cast<uint16_t>(all[q] & 0xFFFFu);
+          if (!SYM) zeros[g0 + q] = static_cast<uint16_t>(all[q] >> 16);
         }
       }
     }
@@ -94,14 +237,13 @@ cudaError_t launch_quantize_pack(const void* w, int64_t N, int64_t K, bool symme
                                  const float* s, float shrink, int32_t* qweight, uint16_t* scales,
                                  uint16_t* zeros, cudaStream_t stream, int num_sms) {
   const int64_t n_groups = N * (K / 128);
-  const int64_t n_units = (n_groups + 1) / 2;
-  const int64_t warps_needed = (n_units + kQuantUnroll - 1) / kQuantUnroll;
+  const int64_t warps_needed = (n_groups + 7) / 8;
   int64_t blocks = (warps_needed + (kQuantThreads / 32) - 1) / (kQuantThreads / 32);
   const int64_t cap = static_cast<int64_t>(num_sms) * 8;  // 8 x 256 threads per SM
   if (blocks > cap) blocks = cap;
   if (blocks < 1) blocks = 1;
   const uint4* wp = static_cast<const uint4*>(w);
-  uint32_t* qp = reinterpret_cast<uint32_t*>(qweight);
+  uint4* qp = reinterpret_cast<uint4*>(qweight);
   const int64_t gpr = K / 128;
   dim3 grid(static_cast<unsigned>(blocks)), block(kQuantThreads);
   if (symmetric) {

@@ -24,7 +24,7 @@ cudaError_t launch_quantize_pack(const void* w, int64_t N, int64_t K, bool symme
 
 cudaError_t launch_gemv(const void* x, int M, const int32_t* qw, const uint16_t* sc,
                         const uint16_t* z, int N, int K, void* y, bool pdl, bool static_w,
-                        cudaStream_t stream, int num_sms);
+                        cudaStream_t stream, int num_sms, unsigned* err);
 
 cudaError_t launch_prefill_gemm(const void* x, int M, const int32_t* qw, const uint16_t* sc,
                                 const uint16_t* z, int N, int K, void* y, bool pdl,
