@@ -125,12 +125,12 @@ w4_status w4_quantize_pack(const void* w_bf16, int64_t N, int64_t K, int group,
  *           rounded once to bf16).
  * flags     bitwise OR of W4_LINEAR_* below (0 for defaults).
  *
- * M <= 16 (and K <= 40960) runs the decode GEMV (tensor-core mma over
+ * M <= 16 (and K <= 81920) runs the decode GEMV (tensor-core mma over
  * register-dequantized weight fragments, HBM-bound); larger M runs the
  * prefill GEMM (tcgen05 with TMEM accumulators, weight tiles dequantized into
  * shared memory).
  */
-#define W4_LINEAR_FORCE_GEMV 0x1u  /* decode kernel at any M <= 64 (K <= 40960) */
+#define W4_LINEAR_FORCE_GEMV 0x1u  /* decode kernel at any M <= 64 (K <= 81920) */
 #define W4_LINEAR_FORCE_GEMM 0x2u  /* prefill kernel at any M */
 #define W4_LINEAR_PDL 0x4u         /* programmatic dependent launch: the
                                       kernel may start before the previous

@@ -146,9 +146,9 @@ w4_status w4a16_linear(const void* x_bf16, int64_t M, const int32_t* qweight,
   if (!aligned16(x_bf16) || !aligned16(qweight) || !aligned16(scales_f16) ||
       (zeros_f16 && !aligned16(zeros_f16)) || !aligned16(y_bf16))
     return W4_ERR_ALIGNMENT;
-  // The decode kernel keeps a CTA's K slice (at most 8 x 40 groups) in a
+  // The decode kernel keeps a CTA's K slice (at most 8 x 80 groups) in a
   // shared scale table; longer K goes to the prefill kernel.
-  const bool gemv_ok = K <= 8 * 40 * 128;
+  const bool gemv_ok = K <= 8 * 80 * 128;
   const bool gemv = (flags & W4_LINEAR_FORCE_GEMV) ||
                     (M <= 16 && gemv_ok && !(flags & W4_LINEAR_FORCE_GEMM));
   if (gemv && (M > 64 || !gemv_ok)) return W4_ERR_UNSUPPORTED;

@@ -39,7 +39,7 @@ namespace {
 constexpr int kRows = 64;                 // weight rows per CTA
 constexpr int kConsumerWarps = 4;
 constexpr int kThreads = 32 * (kConsumerWarps + 1);
-constexpr int kMaxSliceGroups = 40;       // groups per CTA slice (scale table)
+constexpr int kMaxSliceGroups = 80;       // groups per CTA slice (scale table)
 constexpr uint32_t kOnes = 0x3F803F80u;    // bf16x2 (1.0, 1.0)
 constexpr uint32_t kWTileBytes = kRows * 64;
 constexpr unsigned kKernelIdGemv = 1;
@@ -57,12 +57,18 @@ __host__ __device__ inline GemvLayout gemv_layout(int nt, int gs_max) {
   const int tokens = 8 * nt;
   L.x_half = tokens * 128;                      // tokens x 64 channels, bf16
   L.stage = kWTileBytes + 2 * L.x_half;         // multiple of 1024
-  const int max_stages = 4;                     // 24-32 KB in flight per CTA
+  // Three (two for 16 tokens) stages per consumer warp keep groups in flight
+  // while a warp computes; stage s is only ever consumed by warp s % 4 (the
+  // ring length is a multiple of the warp count whenever a stage is reused).
+  const int max_stages = (nt == 1 ? 3 : 2) * kConsumerWarps;
   L.stages = gs_max < max_stages ? (gs_max < 1 ? 1 : gs_max) : max_stages;
   L.ring = 0;
   L.sz = L.ring + L.stages * L.stage;            // [64][gs_max] (scale | zero << 16)
-  L.red = L.sz + ((kRows * gs_max * 4 + 15) & ~15u);  // [4][tokens][64] f32
-  L.part = L.red + kConsumerWarps * tokens * kRows * 4;  // [tokens][64] f32
+  // The per-warp partial sums reuse the ring once every stage is consumed.
+  L.red = L.ring;                                // [4][tokens][64] f32
+  const uint32_t red_end = L.red + kConsumerWarps * tokens * kRows * 4;
+  L.part = L.sz + ((kRows * gs_max * 4 + 15) & ~15u);  // [tokens][64] f32
+  if (L.part < red_end) L.part = red_end;
   L.bars = L.part + tokens * kRows * 4;          // full[S], empty[S]
   L.misc = L.bars + 2 * L.stages * 8;
   L.total = L.misc + 16 + 1024;                  // + alignment slack
@@ -77,14 +83,53 @@ __device__ __forceinline__ uint4 lds128(uint32_t addr) {
   return r;
 }
 
-// bf16x2 (128 + q_lo, 128 + q_hi) from the nibble pair at bits 0..3 / 16..19
-// of u (exact: bf16 has unit spacing on [128, 256)).
-__device__ __forceinline__ uint32_t code_pair(uint32_t u) {
-  return (u & 0x000F000Fu) | 0x43004300u;
-}
+// One reduction step of one 16-row tile, fused so that the code pairs land
+// directly in the mma's operand registers: for the two packed words va (row
+// g) and vb (row g+8), shifted right by SH, the A fragment is
+//   (x >> SH) & 0x000F000F | 0x43004300   and   (x >> (SH+4)) & ...,
+// i.e. bf16x2 (128 + q) pairs of adjacent channels (exact: bf16 has unit
+// spacing on [128, 256)).
+// One 16-row tile over one 128-channel group, 8 reduction steps, in a single
+// asm block: the code pairs and the running accumulator stay in registers the
+// block owns.  Word j of each row (channels 8j..8j+7 of this lane's 32) feeds
+// steps 2j (pairs at shift 0 and 4) and 2j+1 (shift 8 and 12); the A fragment
+// of a step is (w >> sh) & 0x000F000F | 0x43004300, bf16x2 (128 + q) pairs of
+// adjacent channels (exact: bf16 has unit spacing on [128, 256)).
+// x0..x3: this lane's x fragments (channels 8j..8j+7 as four bf16x2).
+#define W4_TILE_STEP(VA, VB, B0, B1, SH0)                                       \
+  "shr.b32 s0, " VA ", " SH0 ";\n\t"                                            \
+  "shr.b32 s1, " VB ", " SH0 ";\n\t"                                            \
+  "shr.b32 s2, " VA ", " SH0 "+4;\n\t"                                          \
+  "shr.b32 s3, " VB ", " SH0 "+4;\n\t"                                          \
+  "lop3.b32 a0, s0, 0x000F000F, 0x43004300, 0xEA;\n\t"                          \
+  "lop3.b32 a1, s1, 0x000F000F, 0x43004300, 0xEA;\n\t"                          \
+  "lop3.b32 a2, s2, 0x000F000F, 0x43004300, 0xEA;\n\t"                          \
+  "lop3.b32 a3, s3, 0x000F000F, 0x43004300, 0xEA;\n\t"                          \
+  "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {c0, c1, c2, c3}, "      \
+  "{a0, a1, a2, a3}, {" B0 ", " B1 "}, {c0, c1, c2, c3};\n\t"
 
-// A pure register operation (not volatile), so the compiler may interleave
-// independent mma chains.
+__device__ __forceinline__ void tile_group(float (&d)[4], const uint4 wa, const uint4 wb,
+                                           const uint4 (&x)[4]) {
+  asm("{\n\t.reg .b32 a0, a1, a2, a3, s0, s1, s2, s3;\n\t"
+      ".reg .f32 c0, c1, c2, c3;\n\t"
+      "mov.b32 c0, 0;\n\tmov.b32 c1, 0;\n\tmov.b32 c2, 0;\n\tmov.b32 c3, 0;\n\t"
+      W4_TILE_STEP("%4", "%8", "%12", "%13", "0")
+      W4_TILE_STEP("%4", "%8", "%14", "%15", "8")
+      W4_TILE_STEP("%5", "%9", "%16", "%17", "0")
+      W4_TILE_STEP("%5", "%9", "%18", "%19", "8")
+      W4_TILE_STEP("%6", "%10", "%20", "%21", "0")
+      W4_TILE_STEP("%6", "%10", "%22", "%23", "8")
+      W4_TILE_STEP("%7", "%11", "%24", "%25", "0")
+      W4_TILE_STEP("%7", "%11", "%26", "%27", "8")
+      "mov.b32 %0, c0;\n\tmov.b32 %1, c1;\n\tmov.b32 %2, c2;\n\tmov.b32 %3, c3;\n\t}"
+      : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+      : "r"(wa.x), "r"(wa.y), "r"(wa.z), "r"(wa.w), "r"(wb.x), "r"(wb.y), "r"(wb.z), "r"(wb.w),
+        "r"(x[0].x), "r"(x[0].y), "r"(x[0].z), "r"(x[0].w), "r"(x[1].x), "r"(x[1].y), "r"(x[1].z),
+        "r"(x[1].w), "r"(x[2].x), "r"(x[2].y), "r"(x[2].z), "r"(x[2].w), "r"(x[3].x), "r"(x[3].y),
+        "r"(x[3].z), "r"(x[3].w));
+}
+#undef W4_TILE_STEP
+
 __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
                                                uint32_t b1) {
   asm(
@@ -100,7 +145,7 @@ __device__ __forceinline__ void named_bar_consumers() {
 }
 
 template <int NT, bool SYM>
-__global__ void __launch_bounds__(kThreads, NT == 1 ? 4 : 2)
+__global__ void __launch_bounds__(kThreads, 2)
     gemv_w4a16_kernel(const __grid_constant__ CUtensorMap tmap_w,   // uint8 [N, K/2], box 64x64
                       const __grid_constant__ CUtensorMap tmap_x,   // bf16 [M, K], box 64 x tokens, SW128
                       const uint16_t* __restrict__ scales, const uint16_t* __restrict__ zeros,
@@ -187,26 +232,28 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 4 : 2)
     // Thread j owns row j / 2 and every other group of it; all its loads are
     // issued before any is used, so the table costs one memory latency.
     if (!static_weights) pdl_wait();
-    {
+    if (threadIdx.x < 2 * kRows) {
       const int r = threadIdx.x >> 1;
       const int row = row0 + r;
       const bool rv = row < N;
       const size_t gbase = static_cast<size_t>(rv ? row : 0) * G + g_begin;
-      uint32_t sv[kMaxSliceGroups / 2], zv[kMaxSliceGroups / 2];
+      for (int q0 = 0; q0 < gs; q0 += 20) {
+        uint32_t sv[10], zv[10];
 #pragma unroll
-      for (int j = 0; j < kMaxSliceGroups / 2; ++j) {
-        const int q = 2 * j + (threadIdx.x & 1);
-        sv[j] = 0u;
-        zv[j] = 0x4800u;  // zero 8 (symmetric)
-        if (rv && q < gs) {
-          sv[j] = __ldg(scales + gbase + q);
-          if (!SYM) zv[j] = __ldg(zeros + gbase + q);
+        for (int j = 0; j < 10; ++j) {
+          const int q = q0 + 2 * j + (threadIdx.x & 1);
+          sv[j] = 0u;
+          zv[j] = 0x4800u;  // zero 8 (symmetric)
+          if (rv && q < gs) {
+            sv[j] = __ldg(scales + gbase + q);
+            if (!SYM) zv[j] = __ldg(zeros + gbase + q);
+          }
         }
-      }
 #pragma unroll
-      for (int j = 0; j < kMaxSliceGroups / 2; ++j) {
-        const int q = 2 * j + (threadIdx.x & 1);
-        if (q < gs) s_sz[r * gs_max + q] = sv[j] | (zv[j] << 16);
+        for (int j = 0; j < 10; ++j) {
+          const int q = q0 + 2 * j + (threadIdx.x & 1);
+          if (q < gs) s_sz[r * gs_max + q] = sv[j] | (zv[j] << 16);
+        }
       }
     }
     named_bar_consumers();
@@ -250,37 +297,19 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 4 : 2)
 #pragma unroll
       for (int n = 0; n < NT; ++n)
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          xs[n][k] = 0.f;
-#pragma unroll
-          for (int rt = 0; rt < 4; ++rt) c[rt][n][k] = 0.f;
-        }
+        for (int k = 0; k < 4; ++k) xs[n][k] = 0.f;
       const uint32_t ones[4] = {kOnes, kOnes, kOnes, kOnes};
 #pragma unroll
-      for (int sp = 0; sp < 8; ++sp) {
-        const int w = sp >> 1;
-        const int sh = 8 * (sp & 1);  // pair 2(sp&1) -> shift 4*pair
-#pragma unroll
-        for (int rt = 0; rt < 4; ++rt) {
-          const uint32_t va = (w == 0 ? wv[rt][0].x : w == 1 ? wv[rt][0].y : w == 2 ? wv[rt][0].z : wv[rt][0].w);
-          const uint32_t vb = (w == 0 ? wv[rt][1].x : w == 1 ? wv[rt][1].y : w == 2 ? wv[rt][1].z : wv[rt][1].w);
-          uint32_t a[4];
-          a[0] = code_pair(va >> sh);
-          a[1] = code_pair(vb >> sh);
-          a[2] = code_pair(va >> (sh + 4));
-          a[3] = code_pair(vb >> (sh + 4));
-#pragma unroll
-          for (int n = 0; n < NT; ++n) {
-            const uint4 xx = xv[n][w];
-            mma_bf16_16816(c[rt][n], a, (sp & 1) ? xx.z : xx.x, (sp & 1) ? xx.w : xx.y);
-          }
-        }
+      for (int sp = 0; sp < 8; ++sp)
 #pragma unroll
         for (int n = 0; n < NT; ++n) {
-          const uint4 xx = xv[n][w];
+          const uint4 xx = xv[n][sp >> 1];
           mma_bf16_16816(xs[n], ones, (sp & 1) ? xx.z : xx.x, (sp & 1) ? xx.w : xx.y);
         }
-      }
+#pragma unroll
+      for (int rt = 0; rt < 4; ++rt)
+#pragma unroll
+        for (int n = 0; n < NT; ++n) tile_group(c[rt][n], wv[rt][0], wv[rt][1], xv[n]);
 #pragma unroll
       for (int rt = 0; rt < 4; ++rt) {
         const uint32_t sza = s_sz[(16 * rt + g) * gs_max + i];
@@ -300,6 +329,9 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 4 : 2)
     }
     pdl_wait();  // (no-op when already satisfied) before this CTA writes y
     // This warp's partial sums: token 8n + 2t + {0,1}, rows 16rt + g (+8).
+    // (The ring is free: every issued stage has been consumed; after a
+    // timeout the results are undefined anyway.)
+    named_bar_consumers();
     float* rw = red + warp * kTokens * kRows;
 #pragma unroll
     for (int rt = 0; rt < 4; ++rt)
@@ -313,8 +345,12 @@ __global__ void __launch_bounds__(kThreads, NT == 1 ? 4 : 2)
       }
     named_bar_consumers();
     for (int e = threadIdx.x; e < kTokens * kRows; e += 32 * kConsumerWarps)
-      part[e] = ((red[e] + red[kTokens * kRows + e]) + red[2 * kTokens * kRows + e]) +
-                red[3 * kTokens * kRows + e];
+    {
+      float sum = 0.f;
+#pragma unroll
+      for (int q = 0; q < kConsumerWarps; ++q) sum += red[q * kTokens * kRows + e];
+      part[e] = sum;
+    }
   }
 
   if (ksplit > 1) {
