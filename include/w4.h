@@ -112,6 +112,26 @@ w4_status w4_quantize_pack(const void* w_bf16, int64_t N, int64_t K, int group,
                            void* stream);
 
 /*
+ * w4_quantize_pack_batched -- w4_quantize_pack over `count` independent
+ * tensors (for example every linear of a model) in as few launches as
+ * possible (64 tensors per launch).  Each item is validated as
+ * w4_quantize_pack validates its arguments; `symmetric` and `group` apply to
+ * all items; each item has its own optional AWQ scale and shrink ratio.
+ * items: host array.  Results are bit-identical to per-tensor calls.
+ */
+typedef struct {
+  const void* w_bf16;     /* device, bf16 [N, K] */
+  int64_t N, K;
+  const float* awq_s;     /* device, float32 [K], or NULL */
+  float shrink;           /* (0, 1] */
+  int32_t* qweight;       /* device, int32 [N, K/8] out */
+  uint16_t* scales_f16;   /* device, fp16 [N, K/128] out */
+  uint16_t* zeros_f16;    /* device, fp16 [N, K/128] out; NULL iff symmetric */
+} w4_quant_item;
+w4_status w4_quantize_pack_batched(const w4_quant_item* items, int count, int group,
+                                   int symmetric, void* stream);
+
+/*
  * w4a16_linear -- y = x . dequant(Wq)^T with bf16 activations and a bf16
  * result ([qwen27b]: activations stay 16-bit; [qsrt] 'Reproducible runtime':
  * decode-sized row counts take their own path).  No bias.
@@ -145,6 +165,27 @@ w4_status w4a16_linear(const void* x_bf16, int64_t M, const int32_t* qweight,
                        const uint16_t* scales_f16, const uint16_t* zeros_f16,
                        int64_t N, int64_t K, int group, void* y_bf16,
                        unsigned flags, void* stream);
+
+/*
+ * w4a16_linear_batched -- w4a16_linear over `count` independent linears that
+ * share the token count M and the symmetry (all zeros NULL or none), for
+ * example every projection of a decode step whose inputs are ready.  M <= 64
+ * (K <= 81920) runs the decode kernel with up to 32 linears per launch;
+ * larger M runs one prefill GEMM per linear.  flags: W4_LINEAR_PDL and
+ * W4_LINEAR_STATIC_WEIGHTS only.  items: host array.  Each result meets the
+ * same error bound as a per-linear call (the K split of a batch, and so the
+ * binary32 summation order, may differ from a single call's).
+ */
+typedef struct {
+  const void* x_bf16;          /* device, bf16 [M, K] */
+  const int32_t* qweight;      /* device, packed weight */
+  const uint16_t* scales_f16;
+  const uint16_t* zeros_f16;   /* NULL: symmetric */
+  int64_t N, K;
+  void* y_bf16;                /* device, bf16 [M, N] out */
+} w4_linear_item;
+w4_status w4a16_linear_batched(const w4_linear_item* items, int count, int64_t M, int group,
+                               unsigned flags, void* stream);
 
 /*
  * w4_awq_scales -- AWQ per-input-channel scales ([rebuttal] 'Search': AWQ

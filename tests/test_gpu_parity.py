@@ -271,3 +271,46 @@ def test_bounded_wait_reports_and_context_survives():
     assert w4.device_error(clear=True) == 0
     # the context is still usable
     assert linear_case(4, 256, 256, False, seed=9) <= Y_RTOL
+
+
+# ------------------------------------------------------------- batched ----
+
+@pytest.mark.parametrize("sym", [False, True])
+def test_quantize_batched_mixed_tensors(sym):
+    shapes = [(n, k) for _, k, n in synth.QWEN3_1P7B_BLOCK] + [(3, 384), (17, 256)]
+    x = synth.student_t_calibration(64, 2048, seed=71)
+    s2048 = O.awq_scales(O.awq_channel_stat(synth.bits(x)), [0.5])[0]
+    items, refs = [], []
+    for i, (n, k) in enumerate(shapes):
+        w = synth.normal_weight(n, k, 0.02, seed=700 + i, n_outliers=4, outlier_scale=20.0)
+        s = s2048 if (k == 2048 and i % 2 == 0) else None
+        r = (1.0, 0.9, 0.75)[i % 3]
+        qw = torch.empty(n, k // 8, dtype=torch.int32, device=DEV)
+        sc = torch.empty(n, k // 128, dtype=torch.int16, device=DEV)
+        zr = None if sym else torch.empty(n, k // 128, dtype=torch.int16, device=DEV)
+        s_dev = None if s is None else torch.from_numpy(s).to(DEV)
+        items.append((w.to(DEV), s_dev, r, qw, sc, zr))
+        refs.append(O.quantize_pack(synth.bits(w), sym, s, r))
+    w4.quantize_pack_batched(items, sym)
+    torch.cuda.synchronize()
+    for (w_, s_, r_, qw, sc, zr), ref in zip(items, refs):
+        assert_quant_equal((qw, sc, zr), ref, sym)
+
+
+@pytest.mark.parametrize("m", [1, 5, 16, 40])
+@pytest.mark.parametrize("sym", [False, True])
+def test_linear_batched_qwen_block(m, sym):
+    shapes = [(n, k) for _, k, n in synth.QWEN3_1P7B_BLOCK] + [(72, 640)]
+    items, refs = [], []
+    for i, (n, k) in enumerate(shapes):
+        w = synth.normal_weight(n, k, 0.02, seed=800 + i)
+        x = synth.normal_activations(m, k, seed=900 + i)
+        qw, sc, zr = w4.quantize_pack(w.to(DEV), sym)
+        y = torch.empty(m, n, dtype=torch.bfloat16, device=DEV)
+        items.append((x.to(DEV), qw, sc, zr, y))
+        oc, os_, oz = O.quantize_rtn(synth.bits(w), sym)
+        refs.append(O.linear(synth.bits(x), O.dequantize(oc, os_, oz)))
+    w4.w4a16_linear_batched(items, m)
+    torch.cuda.synchronize()
+    for (x, qw, sc, zr, y), ref in zip(items, refs):
+        assert max_rel_err(y, ref) <= Y_RTOL

@@ -15,7 +15,8 @@ import os
 from typing import Optional, Sequence
 
 __all__ = [
-    "W4Error", "lib", "quantize_pack", "w4a16_linear", "awq_scales", "awq_score_grid",
+    "W4Error", "lib", "quantize_pack", "quantize_pack_batched", "w4a16_linear",
+    "w4a16_linear_batched", "awq_scales", "awq_score_grid",
     "awq_workspace_bytes", "device_error", "selftest_bounded_wait",
     "LINEAR_FORCE_GEMV", "LINEAR_FORCE_GEMM", "LINEAR_PDL", "LINEAR_STATIC_WEIGHTS",
 ]
@@ -63,6 +64,10 @@ def _declare(L: ctypes.CDLL) -> None:
     L.w4a16_linear.restype = ctypes.c_int
     L.w4a16_linear.argtypes = [_p, _i64, _p, _p, _p, _i64, _i64, ctypes.c_int, _p,
                                ctypes.c_uint, _p]
+    L.w4_quantize_pack_batched.restype = ctypes.c_int
+    L.w4_quantize_pack_batched.argtypes = [_p, ctypes.c_int, ctypes.c_int, ctypes.c_int, _p]
+    L.w4a16_linear_batched.restype = ctypes.c_int
+    L.w4a16_linear_batched.argtypes = [_p, ctypes.c_int, _i64, ctypes.c_int, ctypes.c_uint, _p]
     L.w4_awq_scales.restype = ctypes.c_int
     L.w4_awq_scales.argtypes = [_p, _i64, _i64, _p, ctypes.c_int, _p, _p]
     L.w4_awq_workspace_bytes.restype = ctypes.c_size_t
@@ -159,6 +164,65 @@ def w4a16_linear(x, qweight, scales, zeros=None, flags: int = 0, group: int = 12
                                 y.data_ptr(), int(flags), _stream(x.device))
     _check(st, "w4a16_linear")
     return y
+
+
+class QuantItem(ctypes.Structure):
+    _fields_ = [("w_bf16", ctypes.c_void_p), ("N", ctypes.c_int64), ("K", ctypes.c_int64),
+                ("awq_s", ctypes.c_void_p), ("shrink", ctypes.c_float),
+                ("qweight", ctypes.c_void_p), ("scales_f16", ctypes.c_void_p),
+                ("zeros_f16", ctypes.c_void_p)]
+
+
+class LinearItem(ctypes.Structure):
+    _fields_ = [("x_bf16", ctypes.c_void_p), ("qweight", ctypes.c_void_p),
+                ("scales_f16", ctypes.c_void_p), ("zeros_f16", ctypes.c_void_p),
+                ("N", ctypes.c_int64), ("K", ctypes.c_int64), ("y_bf16", ctypes.c_void_p)]
+
+
+def quantize_pack_items(items):
+    """ctypes array of QuantItem for w4_quantize_pack_batched from
+    (w, awq_s or None, shrink, qweight, scales, zeros or None) tuples."""
+    arr = (QuantItem * len(items))()
+    for a, (w, s, r, qw, sc, zr) in zip(arr, items):
+        a.w_bf16, a.N, a.K = w.data_ptr(), w.shape[0], w.shape[1]
+        a.awq_s = None if s is None else s.data_ptr()
+        a.shrink = float(r)
+        a.qweight, a.scales_f16 = qw.data_ptr(), sc.data_ptr()
+        a.zeros_f16 = None if zr is None else zr.data_ptr()
+    return arr
+
+
+def quantize_pack_batched(items, symmetric: bool, group: int = 128, stream=None) -> None:
+    """Quantize+pack many tensors in few launches; items are tuples
+    (w, awq_s or None, shrink, qweight, scales, zeros or None) of CUDA tensors
+    (outputs preallocated), or a prepared quantize_pack_items() array."""
+    torch = _torch()
+    arr = items if isinstance(items, ctypes.Array) else quantize_pack_items(items)
+    st = lib().w4_quantize_pack_batched(ctypes.addressof(arr), len(arr), group,
+                                        int(bool(symmetric)),
+                                        stream if stream is not None else _stream(torch.cuda.current_device()))
+    _check(st, "w4_quantize_pack_batched")
+
+
+def linear_items(items):
+    """ctypes array of LinearItem from (x, qweight, scales, zeros or None, y) tuples."""
+    arr = (LinearItem * len(items))()
+    for a, (x, qw, sc, zr, y) in zip(arr, items):
+        a.x_bf16, a.qweight, a.scales_f16 = x.data_ptr(), qw.data_ptr(), sc.data_ptr()
+        a.zeros_f16 = None if zr is None else zr.data_ptr()
+        a.N, a.K, a.y_bf16 = qw.shape[0], x.shape[1], y.data_ptr()
+    return arr
+
+
+def w4a16_linear_batched(items, m: int, flags: int = 0, group: int = 128, stream=None) -> None:
+    """Many independent linears with the same token count m in few launches;
+    items are (x, qweight, scales, zeros or None, y) tuples of CUDA tensors or
+    a prepared linear_items() array."""
+    torch = _torch()
+    arr = items if isinstance(items, ctypes.Array) else linear_items(items)
+    st = lib().w4a16_linear_batched(ctypes.addressof(arr), len(arr), int(m), group, int(flags),
+                                    stream if stream is not None else _stream(torch.cuda.current_device()))
+    _check(st, "w4a16_linear_batched")
 
 
 def awq_scales(x, alphas: Sequence[float]):

@@ -113,25 +113,81 @@ int w4_abi_version(void) { return W4_ABI_VERSION; }
 
 const char* w4_last_error(void) { return g_last_error; }
 
-w4_status w4_quantize_pack(const void* w_bf16, int64_t N, int64_t K, int group, int symmetric,
-                           const float* awq_s, float shrink, int32_t* qweight,
-                           uint16_t* scales_f16, uint16_t* zeros_f16, void* stream) {
+static w4_status check_quant_item(const void* w_bf16, int64_t N, int64_t K, int symmetric,
+                                  const float* awq_s, float shrink, int32_t* qweight,
+                                  uint16_t* scales_f16, uint16_t* zeros_f16) {
   if (!w_bf16 || !qweight || !scales_f16) return W4_ERR_INVALID_ARG;
   if ((symmetric != 0) != (zeros_f16 == nullptr)) return W4_ERR_INVALID_ARG;
   if (!(shrink > 0.0f && shrink <= 1.0f)) return W4_ERR_INVALID_ARG;
-  if (group != 128) return W4_ERR_UNSUPPORTED;
   if (N < 1 || !valid_k(K) || N > (int64_t{1} << 40) / K) return W4_ERR_SHAPE;
   if (!aligned16(w_bf16) || !aligned16(qweight) || !aligned16(scales_f16) ||
       (zeros_f16 && !aligned16(zeros_f16)) || (awq_s && !aligned16(awq_s)))
     return W4_ERR_ALIGNMENT;
+  return W4_OK;
+}
+
+w4_status w4_quantize_pack(const void* w_bf16, int64_t N, int64_t K, int group, int symmetric,
+                           const float* awq_s, float shrink, int32_t* qweight,
+                           uint16_t* scales_f16, uint16_t* zeros_f16, void* stream) {
+  if (group != 128 && w_bf16 && qweight && scales_f16) return W4_ERR_UNSUPPORTED;
+  w4_status st = check_quant_item(w_bf16, N, K, symmetric, awq_s, shrink, qweight, scales_f16,
+                                  zeros_f16);
+  if (st != W4_OK) return st;
+  if (group != 128) return W4_ERR_UNSUPPORTED;
+  int sms = 0;
+  st = device_info(&sms, nullptr);
+  if (st != W4_OK) return st;
+  QuantBatch b;
+  b.count = 0;
+  b.unit_start[0] = 0;
+  quant_batch_add(b, w_bf16, N, K, awq_s, shrink, qweight, scales_f16, zeros_f16);
+  return cuda_status(launch_quantize_pack_batch(b, symmetric != 0,
+                                                static_cast<cudaStream_t>(stream), sms),
+                     "quantize+pack launch");
+}
+
+w4_status w4_quantize_pack_batched(const w4_quant_item* items, int count, int group,
+                                   int symmetric, void* stream) {
+  if (!items || count < 1) return W4_ERR_INVALID_ARG;
+  if (group != 128) return W4_ERR_UNSUPPORTED;
+  for (int i = 0; i < count; ++i) {
+    const w4_quant_item& it = items[i];
+    const w4_status st = check_quant_item(it.w_bf16, it.N, it.K, symmetric, it.awq_s, it.shrink,
+                                          it.qweight, it.scales_f16, it.zeros_f16);
+    if (st != W4_OK) return st;
+  }
   int sms = 0;
   w4_status st = device_info(&sms, nullptr);
   if (st != W4_OK) return st;
-  return cuda_status(launch_quantize_pack(w_bf16, N, K, symmetric != 0, awq_s, shrink, qweight,
-                                          scales_f16, zeros_f16,
-                                          static_cast<cudaStream_t>(stream), sms),
-                     "quantize+pack launch");
+  for (int i0 = 0; i0 < count; i0 += kQuantBatch) {
+    QuantBatch b;
+    b.count = 0;
+    b.unit_start[0] = 0;
+    for (int i = i0; i < count && i < i0 + kQuantBatch; ++i) {
+      const w4_quant_item& it = items[i];
+      quant_batch_add(b, it.w_bf16, it.N, it.K, it.awq_s, it.shrink, it.qweight, it.scales_f16,
+                      it.zeros_f16);
+    }
+    st = cuda_status(launch_quantize_pack_batch(b, symmetric != 0,
+                                                static_cast<cudaStream_t>(stream), sms),
+                     "batched quantize+pack launch");
+    if (st != W4_OK) return st;
+  }
+  return W4_OK;
 }
+
+static w4_status check_linear_item(const void* x_bf16, int64_t M, const int32_t* qweight,
+                                   const uint16_t* scales_f16, const uint16_t* zeros_f16,
+                                   int64_t N, int64_t K, void* y_bf16) {
+  if (!x_bf16 || !qweight || !scales_f16 || !y_bf16) return W4_ERR_INVALID_ARG;
+  if (M < 1 || N < 1 || !valid_k(K) || M > 0x7FFFFFFF || N > 0x7FFFFFFF) return W4_ERR_SHAPE;
+  if (!aligned16(x_bf16) || !aligned16(qweight) || !aligned16(scales_f16) ||
+      (zeros_f16 && !aligned16(zeros_f16)) || !aligned16(y_bf16))
+    return W4_ERR_ALIGNMENT;
+  return W4_OK;
+}
+
+static constexpr int64_t kGemvMaxK = 8 * 80 * 128;  // decode kernel: K slice <= 80 groups x 8
 
 w4_status w4a16_linear(const void* x_bf16, int64_t M, const int32_t* qweight,
                        const uint16_t* scales_f16, const uint16_t* zeros_f16, int64_t N,
@@ -142,20 +198,18 @@ w4_status w4a16_linear(const void* x_bf16, int64_t M, const int32_t* qweight,
   if (flags & ~known) return W4_ERR_INVALID_ARG;
   if ((flags & W4_LINEAR_FORCE_GEMV) && (flags & W4_LINEAR_FORCE_GEMM)) return W4_ERR_INVALID_ARG;
   if (group != 128) return W4_ERR_UNSUPPORTED;
-  if (M < 1 || N < 1 || !valid_k(K) || M > 0x7FFFFFFF || N > 0x7FFFFFFF) return W4_ERR_SHAPE;
-  if (!aligned16(x_bf16) || !aligned16(qweight) || !aligned16(scales_f16) ||
-      (zeros_f16 && !aligned16(zeros_f16)) || !aligned16(y_bf16))
-    return W4_ERR_ALIGNMENT;
+  w4_status st = check_linear_item(x_bf16, M, qweight, scales_f16, zeros_f16, N, K, y_bf16);
+  if (st != W4_OK) return st;
   // The decode kernel keeps a CTA's K slice (at most 8 x 80 groups) in a
   // shared scale table; longer K goes to the prefill kernel.
-  const bool gemv_ok = K <= 8 * 80 * 128;
+  const bool gemv_ok = K <= kGemvMaxK;
   const bool gemv = (flags & W4_LINEAR_FORCE_GEMV) ||
                     (M <= 16 && gemv_ok && !(flags & W4_LINEAR_FORCE_GEMM));
   if (gemv && (M > 64 || !gemv_ok)) return W4_ERR_UNSUPPORTED;
   if (!gemv && (M + 127) / 128 > 65535) return W4_ERR_UNSUPPORTED;
   int sms = 0;
   unsigned* err = nullptr;
-  w4_status st = device_info(&sms, &err);
+  st = device_info(&sms, &err);
   if (st != W4_OK) return st;
   const bool pdl = (flags & W4_LINEAR_PDL) != 0;
   const bool stat = (flags & W4_LINEAR_STATIC_WEIGHTS) != 0;
@@ -169,6 +223,62 @@ w4_status w4a16_linear(const void* x_bf16, int64_t M, const int32_t* qweight,
                                          zeros_f16, static_cast<int>(N), static_cast<int>(K),
                                          y_bf16, pdl, stat, s, err),
                      "prefill tcgen05 GEMM launch");
+}
+
+w4_status w4a16_linear_batched(const w4_linear_item* items, int count, int64_t M, int group,
+                               unsigned flags, void* stream) {
+  if (!items || count < 1) return W4_ERR_INVALID_ARG;
+  const unsigned known = W4_LINEAR_PDL | W4_LINEAR_STATIC_WEIGHTS;
+  if (flags & ~known) return W4_ERR_INVALID_ARG;
+  if (group != 128) return W4_ERR_UNSUPPORTED;
+  const bool sym = items[0].zeros_f16 == nullptr;
+  for (int i = 0; i < count; ++i) {
+    const w4_linear_item& it = items[i];
+    w4_status st = check_linear_item(it.x_bf16, M, it.qweight, it.scales_f16, it.zeros_f16, it.N,
+                                     it.K, it.y_bf16);
+    if (st != W4_OK) return st;
+    if ((it.zeros_f16 == nullptr) != sym) return W4_ERR_INVALID_ARG;
+    if (M <= 64 && it.K > kGemvMaxK) return W4_ERR_UNSUPPORTED;
+  }
+  int sms = 0;
+  unsigned* err = nullptr;
+  w4_status st = device_info(&sms, &err);
+  if (st != W4_OK) return st;
+  const bool pdl = (flags & W4_LINEAR_PDL) != 0;
+  const bool stat = (flags & W4_LINEAR_STATIC_WEIGHTS) != 0;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (M > 64) {  // prefill: one tcgen05 GEMM per linear
+    for (int i = 0; i < count; ++i) {
+      const w4_linear_item& it = items[i];
+      st = cuda_status(launch_prefill_gemm(it.x_bf16, static_cast<int>(M), it.qweight,
+                                           it.scales_f16, it.zeros_f16, static_cast<int>(it.N),
+                                           static_cast<int>(it.K), it.y_bf16, pdl, stat, s, err),
+                       "prefill tcgen05 GEMM launch");
+      if (st != W4_OK) return st;
+    }
+    return W4_OK;
+  }
+  for (int64_t m0 = 0; m0 < M; m0 += 16) {
+    const int mc = static_cast<int>(M - m0 < 16 ? M - m0 : 16);
+    for (int i0 = 0; i0 < count; i0 += kGemvBatch) {
+      GemvBatch b;
+      b.count = 0;
+      b.cta_start[0] = 0;
+      b.M = mc;
+      for (int i = i0; i < count && i < i0 + kGemvBatch; ++i) {
+        const w4_linear_item& it = items[i];
+        const void* xc = static_cast<const uint16_t*>(it.x_bf16) + m0 * it.K;
+        void* yc = static_cast<uint16_t*>(it.y_bf16) + m0 * it.N;
+        st = cuda_status(gemv_batch_add(b, xc, it.qweight, it.scales_f16, it.zeros_f16,
+                                        static_cast<int>(it.N), static_cast<int>(it.K), yc),
+                         "tensor map");
+        if (st != W4_OK) return st;
+      }
+      st = cuda_status(launch_gemv_batch(b, sym, pdl, stat, s, sms, err), "batched decode GEMV launch");
+      if (st != W4_OK) return st;
+    }
+  }
+  return W4_OK;
 }
 
 w4_status w4_awq_scales(const void* x_bf16, int64_t M, int64_t K, const float* alphas,

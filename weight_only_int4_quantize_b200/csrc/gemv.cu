@@ -146,12 +146,24 @@ __device__ __forceinline__ void named_bar_consumers() {
 
 template <int NT, bool SYM>
 __global__ void __launch_bounds__(kThreads, 2)
-    gemv_w4a16_kernel(const __grid_constant__ CUtensorMap tmap_w,   // uint8 [N, K/2], box 64x64
-                      const __grid_constant__ CUtensorMap tmap_x,   // bf16 [M, K], box 64 x tokens, SW128
-                      const uint16_t* __restrict__ scales, const uint16_t* __restrict__ zeros,
-                      __nv_bfloat16* __restrict__ y, int M, int N, int K, int ksplit,
-                      int gs_max, int static_weights, unsigned* err) {
+    gemv_w4a16_kernel(const __grid_constant__ GemvBatch b, int static_weights, unsigned* err) {
   constexpr int kTokens = 8 * NT;
+  // This CTA's linear of the batch and its 64-row block.
+  int item = 0;
+  {
+    int lo = 0, hi = b.count - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (b.cta_start[mid] <= static_cast<int>(blockIdx.x)) lo = mid; else hi = mid - 1;
+    }
+    item = lo;
+  }
+  const CUtensorMap* tmap_w = &b.tw[item];   // uint8 [N, K/2], box 64 x 64
+  const CUtensorMap* tmap_x = &b.tx[item];   // bf16 [M, K], box 64 x tokens, SW128
+  const uint16_t* __restrict__ scales = b.scales[item];
+  const uint16_t* __restrict__ zeros = b.zeros[item];
+  __nv_bfloat16* __restrict__ y = b.y[item];
+  const int M = b.M, N = b.N[item], K = b.K[item], ksplit = b.ksplit, gs_max = b.gs_max;
   const GemvLayout L = gemv_layout(NT, gs_max);
   const int S = L.stages;
   extern __shared__ uint8_t smem_raw[];
@@ -169,7 +181,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int G = K >> 7;
-  const int row0 = blockIdx.x * kRows;
+  const int row0 = (static_cast<int>(blockIdx.x) - b.cta_start[item]) * kRows;
   const int rank = blockIdx.y;
   const int g_per = (G + ksplit - 1) / ksplit;
   const int g_begin = min(G, rank * g_per);
@@ -190,15 +202,15 @@ __global__ void __launch_bounds__(kThreads, 2)
   if (warp == kConsumerWarps) {
     // ------------------------------------------------------- producer ----
     if (lane == 0) {
-      tma_prefetch_desc(&tmap_w);
-      tma_prefetch_desc(&tmap_x);
+      tma_prefetch_desc(tmap_w);
+      tma_prefetch_desc(tmap_x);
       const uint32_t stage_tx = L.stage;
       // Stages whose weight tile was issued before the dependency wait.
       const int pre = static_weights ? min(gs, S) : 0;
       for (int i = 0; i < pre; ++i) {
         const uint32_t st = base + L.ring + i * L.stage;
         mbar_arrive_expect_tx(full(i), stage_tx);
-        tma_load_2d(st, &tmap_w, (g_begin + i) * 64, row0, full(i));
+        tma_load_2d(st, tmap_w, (g_begin + i) * 64, row0, full(i));
       }
       pdl_wait();
       int issued = 0;
@@ -210,10 +222,10 @@ __global__ void __launch_bounds__(kThreads, 2)
           if (!mbar_wait(empty(s), ((i / S) & 1u) ^ 1u, abort_flag, err, kKernelIdGemv))
             break;
           mbar_arrive_expect_tx(full(s), stage_tx);
-          tma_load_2d(st, &tmap_w, gr * 64, row0, full(s));
+          tma_load_2d(st, tmap_w, gr * 64, row0, full(s));
         }
-        tma_load_2d(st + kWTileBytes, &tmap_x, gr * 128, 0, full(s));
-        tma_load_2d(st + kWTileBytes + L.x_half, &tmap_x, gr * 128 + 64, 0, full(s));
+        tma_load_2d(st + kWTileBytes, tmap_x, gr * 128, 0, full(s));
+        tma_load_2d(st + kWTileBytes + L.x_half, tmap_x, gr * 128 + 64, 0, full(s));
         issued = i + 1;
       }
       if (*abort_flag) {  // drain this CTA's own loads before leaving
@@ -403,12 +415,8 @@ CUresult encode_2d(CUtensorMap* map, CUtensorMapDataType dt, const void* base, u
 }
 
 template <int NT, bool SYM>
-cudaError_t launch_gemv_t(const void* x, int M, const int32_t* qw, const uint16_t* sc,
-                          const uint16_t* z, int N, int K, void* y, bool pdl, bool static_w,
-                          cudaStream_t stream, int num_sms, unsigned* err) {
-  constexpr int kTokens = 8 * NT;
-  const int G = K / 128;
-  const int row_blocks = (N + kRows - 1) / kRows;
+cudaError_t launch_gemv_batch_t(GemvBatch& b, bool pdl, bool static_w, cudaStream_t stream,
+                                int num_sms, unsigned* err) {
   auto kern = gemv_w4a16_kernel<NT, SYM>;
   // Opt in once per device to the largest layout this kernel can use, and
   // record how many CTAs of it an SM holds.
@@ -431,22 +439,21 @@ cudaError_t launch_gemv_t(const void* x, int M, const int32_t* qw, const uint16_
   }
   const int capacity = num_sms * (dev < 64 ? per_sm[dev] : 1);
   // Split K over a cluster as far as the grid still fits in one wave and
-  // every CTA keeps at least two groups; the CTA's K slice must fit the
-  // shared scale table.
+  // every CTA of every linear keeps at least two groups; a CTA's K slice
+  // must fit the shared scale table.
+  const int row_blocks = b.cta_start[b.count];
+  int g_min = 1 << 30, g_max = 0;
+  for (int i = 0; i < b.count; ++i) {
+    g_min = b.K[i] / 128 < g_min ? b.K[i] / 128 : g_min;
+    g_max = b.K[i] / 128 > g_max ? b.K[i] / 128 : g_max;
+  }
   int ks = 1;
-  while (ks < 8 && row_blocks * ks * 2 <= capacity && G / (ks * 2) >= 2) ks *= 2;
-  while ((G + ks - 1) / ks > kMaxSliceGroups && ks < 8) ks *= 2;
-  if ((G + ks - 1) / ks > kMaxSliceGroups) return cudaErrorInvalidValue;
-  const int gs_max = (G + ks - 1) / ks;
-  const GemvLayout L = gemv_layout(NT, gs_max);
-
-  CUtensorMap tw, tx;
-  if (encode_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, qw, static_cast<uint64_t>(K) / 2, N,
-                static_cast<uint64_t>(K) / 2, 64, kRows, CU_TENSOR_MAP_SWIZZLE_NONE) != CUDA_SUCCESS)
-    return cudaErrorInvalidValue;
-  if (encode_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, K, M, static_cast<uint64_t>(K) * 2, 64,
-                kTokens, CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS)
-    return cudaErrorInvalidValue;
+  while (ks < 8 && row_blocks * ks * 2 <= capacity && g_min / (ks * 2) >= 2) ks *= 2;
+  while ((g_max + ks - 1) / ks > kMaxSliceGroups && ks < 8) ks *= 2;
+  if ((g_max + ks - 1) / ks > kMaxSliceGroups) return cudaErrorInvalidValue;
+  b.ksplit = ks;
+  b.gs_max = (g_max + ks - 1) / ks;
+  const GemvLayout L = gemv_layout(NT, b.gs_max);
 
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(row_blocks, ks, 1);
@@ -469,29 +476,55 @@ cudaError_t launch_gemv_t(const void* x, int M, const int32_t* qw, const uint16_
   }
   cfg.attrs = attrs;
   cfg.numAttrs = na;
-  return cudaLaunchKernelEx(&cfg, kern, tw, tx, sc, z, static_cast<__nv_bfloat16*>(y), M, N, K,
-                            ks, gs_max, static_cast<int>(pdl && static_w), err);
+  return cudaLaunchKernelEx(&cfg, kern, b, static_cast<int>(pdl && static_w), err);
 }
 
 }  // namespace
 
+// Adds one linear (one chunk of at most 16 tokens) to a batch.
+cudaError_t gemv_batch_add(GemvBatch& b, const void* x, const int32_t* qw, const uint16_t* sc,
+                           const uint16_t* z, int N, int K, void* y) {
+  const int i = b.count;
+  if (encode_2d(&b.tw[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, qw, static_cast<uint64_t>(K) / 2, N,
+                static_cast<uint64_t>(K) / 2, 64, kRows, CU_TENSOR_MAP_SWIZZLE_NONE) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+  if (encode_2d(&b.tx[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, K, b.M,
+                static_cast<uint64_t>(K) * 2, 64, b.M <= 8 ? 8 : 16,
+                CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+  b.scales[i] = sc;
+  b.zeros[i] = z;
+  b.y[i] = static_cast<__nv_bfloat16*>(y);
+  b.N[i] = N;
+  b.K[i] = K;
+  b.cta_start[i + 1] = b.cta_start[i] + (N + kRows - 1) / kRows;
+  b.count = i + 1;
+  return cudaSuccess;
+}
+
+// All items share M (<= 16 tokens) and symmetry.
+cudaError_t launch_gemv_batch(GemvBatch& b, bool symmetric, bool pdl, bool static_w,
+                              cudaStream_t stream, int num_sms, unsigned* err) {
+  if (b.M <= 8)
+    return symmetric ? launch_gemv_batch_t<1, true>(b, pdl, static_w, stream, num_sms, err)
+                     : launch_gemv_batch_t<1, false>(b, pdl, static_w, stream, num_sms, err);
+  return symmetric ? launch_gemv_batch_t<2, true>(b, pdl, static_w, stream, num_sms, err)
+                   : launch_gemv_batch_t<2, false>(b, pdl, static_w, stream, num_sms, err);
+}
+
 cudaError_t launch_gemv(const void* x, int M, const int32_t* qw, const uint16_t* sc,
                         const uint16_t* z, int N, int K, void* y, bool pdl, bool static_w,
                         cudaStream_t stream, int num_sms, unsigned* err) {
-  const bool sym = (z == nullptr);
   // M <= 64 in chunks of up to 16 tokens (two n-tiles of 8).
   for (int m0 = 0; m0 < M; m0 += 16) {
-    const int mc = (M - m0) < 16 ? (M - m0) : 16;
+    GemvBatch b;
+    b.count = 0;
+    b.cta_start[0] = 0;
+    b.M = (M - m0) < 16 ? (M - m0) : 16;
     const void* xc = static_cast<const __nv_bfloat16*>(x) + static_cast<size_t>(m0) * K;
     void* yc = static_cast<__nv_bfloat16*>(y) + static_cast<size_t>(m0) * N;
-    cudaError_t e;
-    if (mc <= 8) {
-      e = sym ? launch_gemv_t<1, true>(xc, mc, qw, sc, z, N, K, yc, pdl, static_w, stream, num_sms, err)
-              : launch_gemv_t<1, false>(xc, mc, qw, sc, z, N, K, yc, pdl, static_w, stream, num_sms, err);
-    } else {
-      e = sym ? launch_gemv_t<2, true>(xc, mc, qw, sc, z, N, K, yc, pdl, static_w, stream, num_sms, err)
-              : launch_gemv_t<2, false>(xc, mc, qw, sc, z, N, K, yc, pdl, static_w, stream, num_sms, err);
-    }
+    cudaError_t e = gemv_batch_add(b, xc, qw, sc, z, N, K, yc);
+    if (e == cudaSuccess) e = launch_gemv_batch(b, z == nullptr, pdl, static_w, stream, num_sms, err);
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;

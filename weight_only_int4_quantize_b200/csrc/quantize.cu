@@ -93,33 +93,54 @@ __device__ __forceinline__ uint32_t bmin2(uint32_t a, uint32_t b) {
 // exact path (correctly rounded division, as in quant_group.cuh).
 template <bool SYM, bool HAS_S>
 __global__ void __launch_bounds__(kQuantThreads, 3)
-    quantize_pack_kernel(const uint4* __restrict__ w, const float* __restrict__ s, float shrink,
-                         int64_t n_groups, int64_t groups_per_row, uint4* __restrict__ qw,
-                         uint16_t* __restrict__ scales, uint16_t* __restrict__ zeros) {
+    quantize_pack_kernel(const __grid_constant__ QuantBatch b) {
   const int lane = threadIdx.x & 31;
   const int sub = lane >> 2;  // group of this quad within the warp's eight
   const int l4 = lane & 3;
   const int64_t warp = (static_cast<int64_t>(blockIdx.x) * kQuantThreads + threadIdx.x) >> 5;
   const int64_t n_warps = (static_cast<int64_t>(gridDim.x) * kQuantThreads) >> 5;
-  const int64_t n_units = (n_groups + 7) >> 3;
+  const int64_t n_units = b.unit_start[b.count];
   const float thr = 0.5f - 1.52587890625e-05f;  // 0.5 - 2^-16
 
+  // Unit u (8 consecutive groups of one tensor) -> its tensor.
+  auto item_of = [&](int64_t u) {
+    int lo = 0, hi = b.count - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (b.unit_start[mid] <= u) lo = mid; else hi = mid - 1;
+    }
+    return lo;
+  };
   // Software pipeline: the next unit's 64 bytes per lane are in flight while
   // the current unit is quantized.
   auto load_unit = [&](int64_t u, uint32_t (&dst)[16]) {
-    const int64_t gi = 8 * u + sub;
-    const uint4* src = w + gi * 16 + l4 * 4;
+    uint4 r[4] = {};
+    if (u < n_units) {
+      const int it = item_of(u);
+      const int64_t gi = 8 * (u - b.unit_start[it]) + sub;
+      if (gi < b.n_groups[it]) {
+        const uint4* src = static_cast<const uint4*>(b.w[it]) + gi * 16 + l4 * 4;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) r[q] = ld_stream(src + q);
+      }
+    }
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-      const uint4 r = (u < n_units && gi < n_groups) ? ld_stream(src + q) : make_uint4(0, 0, 0, 0);
-      dst[4 * q] = r.x; dst[4 * q + 1] = r.y; dst[4 * q + 2] = r.z; dst[4 * q + 3] = r.w;
+      dst[4 * q] = r[q].x; dst[4 * q + 1] = r[q].y; dst[4 * q + 2] = r[q].z; dst[4 * q + 3] = r[q].w;
     }
   };
   uint32_t nxt[16];
   load_unit(warp, nxt);
   for (int64_t u = warp; u < n_units; u += n_warps) {
-    const int64_t gi = 8 * u + sub;
+    const int it = item_of(u);
+    const int64_t n_groups = b.n_groups[it];
+    const int64_t gi = 8 * (u - b.unit_start[it]) + sub;
     const bool valid = gi < n_groups;
+    const float shrink = b.shrink[it];
+    const float* s = b.s[it];
+    uint4* qw = static_cast<uint4*>(b.qw[it]);
+    uint16_t* scales = b.scales[it];
+    uint16_t* zeros = b.zeros[it];
     uint32_t raw[16];
 #pragma unroll
     for (int p = 0; p < 16; ++p) raw[p] = nxt[p];
@@ -131,13 +152,15 @@ __global__ void __launch_bounds__(kQuantThreads, 3)
     GroupQ g;
     float amax;
     if (HAS_S) {
-      const int64_t k0 = (gi % groups_per_row) * 128 + l4 * 32;
-      const float4* sp = reinterpret_cast<const float4*>(s + (valid ? k0 : 0));
+      if (s != nullptr) {
+        const int64_t k0 = (gi % b.groups_per_row[it]) * 128 + l4 * 32;
+        const float4* sp = reinterpret_cast<const float4*>(s + (valid ? k0 : 0));
 #pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        const float4 sv = __ldg(sp + q);
-        v[2 * q] = mul2(v[2 * q], make_float2(sv.x, sv.y));
-        v[2 * q + 1] = mul2(v[2 * q + 1], make_float2(sv.z, sv.w));
+        for (int q = 0; q < 8; ++q) {
+          const float4 sv = __ldg(sp + q);
+          v[2 * q] = mul2(v[2 * q], make_float2(sv.x, sv.y));
+          v[2 * q + 1] = mul2(v[2 * q + 1], make_float2(sv.z, sv.w));
+        }
       }
       if (SYM) {
         float a = 0.f;
@@ -233,27 +256,39 @@ __global__ void __launch_bounds__(kQuantThreads, 3)
 
 }  // namespace
 
-cudaError_t launch_quantize_pack(const void* w, int64_t N, int64_t K, bool symmetric,
-                                 const float* s, float shrink, int32_t* qweight, uint16_t* scales,
-                                 uint16_t* zeros, cudaStream_t stream, int num_sms) {
-  const int64_t n_groups = N * (K / 128);
-  const int64_t warps_needed = (n_groups + 7) / 8;
-  int64_t blocks = (warps_needed + (kQuantThreads / 32) - 1) / (kQuantThreads / 32);
+cudaError_t launch_quantize_pack_batch(const QuantBatch& b, bool symmetric, cudaStream_t stream,
+                                       int num_sms) {
+  const int64_t n_units = b.unit_start[b.count];
+  int64_t blocks = (n_units + (kQuantThreads / 32) - 1) / (kQuantThreads / 32);
   const int64_t cap = static_cast<int64_t>(num_sms) * 8;  // 8 x 256 threads per SM
   if (blocks > cap) blocks = cap;
   if (blocks < 1) blocks = 1;
-  const uint4* wp = static_cast<const uint4*>(w);
-  uint4* qp = reinterpret_cast<uint4*>(qweight);
-  const int64_t gpr = K / 128;
+  bool any_s = false;
+  for (int i = 0; i < b.count; ++i) any_s = any_s || b.s[i] != nullptr;
   dim3 grid(static_cast<unsigned>(blocks)), block(kQuantThreads);
   if (symmetric) {
-    if (s) quantize_pack_kernel<true, true><<<grid, block, 0, stream>>>(wp, s, shrink, n_groups, gpr, qp, scales, zeros);
-    else   quantize_pack_kernel<true, false><<<grid, block, 0, stream>>>(wp, s, shrink, n_groups, gpr, qp, scales, zeros);
+    if (any_s) quantize_pack_kernel<true, true><<<grid, block, 0, stream>>>(b);
+    else       quantize_pack_kernel<true, false><<<grid, block, 0, stream>>>(b);
   } else {
-    if (s) quantize_pack_kernel<false, true><<<grid, block, 0, stream>>>(wp, s, shrink, n_groups, gpr, qp, scales, zeros);
-    else   quantize_pack_kernel<false, false><<<grid, block, 0, stream>>>(wp, s, shrink, n_groups, gpr, qp, scales, zeros);
+    if (any_s) quantize_pack_kernel<false, true><<<grid, block, 0, stream>>>(b);
+    else       quantize_pack_kernel<false, false><<<grid, block, 0, stream>>>(b);
   }
   return cudaGetLastError();
+}
+
+void quant_batch_add(QuantBatch& b, const void* w, int64_t N, int64_t K, const float* s,
+                     float shrink, int32_t* qweight, uint16_t* scales, uint16_t* zeros) {
+  const int i = b.count;
+  b.w[i] = w;
+  b.s[i] = s;
+  b.shrink[i] = shrink;
+  b.qw[i] = qweight;
+  b.scales[i] = scales;
+  b.zeros[i] = zeros;
+  b.n_groups[i] = N * (K / 128);
+  b.groups_per_row[i] = K / 128;
+  b.unit_start[i + 1] = b.unit_start[i] + (b.n_groups[i] + 7) / 8;
+  b.count = i + 1;
 }
 
 }  // namespace w4

@@ -3,6 +3,8 @@
 #pragma once
 
 #include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 namespace w4 {
@@ -18,10 +20,43 @@ struct ShrinkList {
   float v[kMaxGrid];
 };
 
-cudaError_t launch_quantize_pack(const void* w, int64_t N, int64_t K, bool symmetric,
-                                 const float* s, float shrink, int32_t* qweight, uint16_t* scales,
-                                 uint16_t* zeros, cudaStream_t stream, int num_sms);
+// Up to kQuantBatch tensors quantized by one launch (kernel parameter).
+constexpr int kQuantBatch = 64;
+struct QuantBatch {
+  int count;
+  const void* w[kQuantBatch];
+  const float* s[kQuantBatch];
+  float shrink[kQuantBatch];
+  void* qw[kQuantBatch];
+  uint16_t* scales[kQuantBatch];
+  uint16_t* zeros[kQuantBatch];
+  int64_t n_groups[kQuantBatch];
+  int64_t groups_per_row[kQuantBatch];
+  int64_t unit_start[kQuantBatch + 1];  // prefix sums of ceil(groups / 8)
+};
+void quant_batch_add(QuantBatch& b, const void* w, int64_t N, int64_t K, const float* s,
+                     float shrink, int32_t* qweight, uint16_t* scales, uint16_t* zeros);
+cudaError_t launch_quantize_pack_batch(const QuantBatch& b, bool symmetric, cudaStream_t stream,
+                                       int num_sms);
 
+// Up to kGemvBatch independent linears with the same token count (<= 16)
+// decoded by one launch; tensor maps travel in the kernel parameter.
+constexpr int kGemvBatch = 32;
+struct GemvBatch {
+  CUtensorMap tw[kGemvBatch];  // packed codes, uint8 [N, K/2], box 64 x 64
+  CUtensorMap tx[kGemvBatch];  // x, bf16 [M, K], box 64 x tokens, 128B swizzle
+  const uint16_t* scales[kGemvBatch];
+  const uint16_t* zeros[kGemvBatch];
+  __nv_bfloat16* y[kGemvBatch];
+  int N[kGemvBatch];
+  int K[kGemvBatch];
+  int cta_start[kGemvBatch + 1];  // prefix sums of 64-row blocks
+  int count, M, ksplit, gs_max;
+};
+cudaError_t gemv_batch_add(GemvBatch& b, const void* x, const int32_t* qw, const uint16_t* sc,
+                           const uint16_t* z, int N, int K, void* y);
+cudaError_t launch_gemv_batch(GemvBatch& b, bool symmetric, bool pdl, bool static_w,
+                              cudaStream_t stream, int num_sms, unsigned* err);
 cudaError_t launch_gemv(const void* x, int M, const int32_t* qw, const uint16_t* sc,
                         const uint16_t* z, int N, int K, void* y, bool pdl, bool static_w,
                         cudaStream_t stream, int num_sms, unsigned* err);
