@@ -23,7 +23,9 @@
  *   - Device pointers are caller-owned device memory (any allocator).  Host
  *     pointers are marked "host".  The library never allocates or frees
  *     memory and keeps no state between calls apart from one device-side
- *     error word (see w4_device_error).
+ *     error word (see w4_device_error).  The one fixed device array it holds,
+ *     the scratch of awq_score_grid_static_scratch, carries nothing from one
+ *     call to the next.
  *   - `stream` is a cudaStream_t passed as void*; NULL is the legacy default
  *     stream.  Launches are asynchronous; outputs are valid once the stream
  *     has been synchronized.
@@ -243,6 +245,50 @@ w4_status awq_score_grid(const void* x_bf16, int64_t M, const void* w_bf16, int6
                          const int64_t* seg_offsets, int n_seg, double* sse_out,
                          int32_t* argmin_out, void* workspace, size_t workspace_bytes,
                          void* stream);
+
+/*
+ * awq_score_grid_static_scratch -- awq_score_grid without a caller-supplied
+ * workspace: its scratch is a fixed device array inside the library of
+ * W4_AWQ_STATIC_SCRATCH_BYTES (32 MiB).  The pages have no counterpart; the
+ * candidates, SSE table and argmins are those of awq_score_grid
+ * ([rebuttal] 'Search' and the scale-rewrite paragraph), bit-identical for
+ * the same inputs.
+ *
+ * It is for callers that cannot allocate device memory when they score: a
+ * serving process whose caching allocator already holds the free HBM (for
+ * weights and KV cache), so that a fresh cudaMalloc of the workspace fails;
+ * and a caller in the middle of queued asynchronous work, where cudaFree's
+ * implicit device-wide synchronization would stall the pipeline.  The call
+ * allocates nothing (no cudaMalloc, cudaFree or allocating library routine).
+ *
+ * Size limit: a problem whose w4_awq_workspace_bytes(M, N, K, n_alpha,
+ * n_shrink, n_seg) exceeds W4_AWQ_STATIC_SCRATCH_BYTES is refused with
+ * W4_ERR_WORKSPACE, nothing launched; w4_last_error() then names the needed
+ * and available sizes.  Any other invalid argument returns the same status
+ * as awq_score_grid would.
+ *
+ * Set-up: the first call on each device, with that device current, looks up
+ * the scratch's device address (cudaGetSymbolAddress) and caches it; under
+ * CUDA's default lazy module loading this is also when the driver reserves
+ * the 32 MiB on that device.  Make that first call before any stream capture
+ * begins.
+ *
+ * Nothing in the scratch needs to start at zero: every word a kernel of the
+ * call reads is written earlier in the same call, so nothing is cleared.
+ *
+ * Concurrency: there is one scratch per device.  Calls whose work overlaps on
+ * one device (different streams, or several host threads) race on it and
+ * produce undefined results; order them on one stream.
+ *
+ * Arguments as for awq_score_grid, without workspace and workspace_bytes.
+ */
+#define W4_AWQ_STATIC_SCRATCH_BYTES (32u << 20)
+w4_status awq_score_grid_static_scratch(const void* x_bf16, int64_t M, const void* w_bf16,
+                                        int64_t N, int64_t K, int group, int symmetric,
+                                        const float* alphas, int n_alpha,
+                                        const float* shrinks, int n_shrink,
+                                        const int64_t* seg_offsets, int n_seg,
+                                        double* sse_out, int32_t* argmin_out, void* stream);
 
 /*
  * w4_device_error -- reads (and with clear != 0 resets) the library's device

@@ -16,7 +16,7 @@ from typing import Optional, Sequence
 
 __all__ = [
     "W4Error", "lib", "quantize_pack", "quantize_pack_batched", "w4a16_linear",
-    "w4a16_linear_batched", "awq_scales", "awq_score_grid",
+    "w4a16_linear_batched", "awq_scales", "awq_score_grid", "awq_score_grid_static_scratch",
     "awq_workspace_bytes", "device_error", "selftest_bounded_wait",
     "LINEAR_FORCE_GEMV", "LINEAR_FORCE_GEMM", "LINEAR_PDL", "LINEAR_STATIC_WEIGHTS",
 ]
@@ -77,6 +77,10 @@ def _declare(L: ctypes.CDLL) -> None:
     L.awq_score_grid.argtypes = [_p, _i64, _p, _i64, _i64, ctypes.c_int, ctypes.c_int, _p,
                                  ctypes.c_int, _p, ctypes.c_int, _p, ctypes.c_int, _p, _p, _p,
                                  ctypes.c_size_t, _p]
+    L.awq_score_grid_static_scratch.restype = ctypes.c_int
+    L.awq_score_grid_static_scratch.argtypes = [_p, _i64, _p, _i64, _i64, ctypes.c_int,
+                                                ctypes.c_int, _p, ctypes.c_int, _p, ctypes.c_int,
+                                                _p, ctypes.c_int, _p, _p, _p]
     L.w4_device_error.restype = ctypes.c_int
     L.w4_device_error.argtypes = [ctypes.c_int, _p]
     L.w4_selftest_bounded_wait.restype = ctypes.c_int
@@ -276,6 +280,41 @@ def awq_score_grid(x, w, alphas, shrinks, symmetric: bool, seg_offsets=None, wor
                                   _stream(x.device))
     _check(st, "awq_score_grid")
     return sse, arg
+
+
+def awq_score_grid_static_scratch(x, w, alphas, shrinks, symmetric: bool, seg_offsets=None,
+                                  sse_out=None, argmin_out=None, group: int = 128):
+    """awq_score_grid with the library's fixed device scratch instead of a
+    workspace.  The C call allocates nothing; pass preallocated sse_out
+    [n_seg, n_alpha, n_shrink] float64 and argmin_out [n_seg + 1, 4] int32
+    to keep this binding from allocating them."""
+    torch = _torch()
+    import numpy as np
+    _cuda(x, torch.bfloat16, "x")
+    _cuda(w, torch.bfloat16, "w")
+    m, k = x.shape
+    n = w.shape[0]
+    a = np.ascontiguousarray(np.asarray(alphas, dtype=np.float32))
+    r = np.ascontiguousarray(np.asarray(shrinks, dtype=np.float32))
+    seg = None if seg_offsets is None else np.ascontiguousarray(np.asarray(seg_offsets, dtype=np.int64))
+    n_seg = 1 if seg is None else len(seg) - 1
+    if sse_out is None:
+        sse_out = torch.empty((n_seg, len(a), len(r)), dtype=torch.float64, device=x.device)
+    if argmin_out is None:
+        argmin_out = torch.empty((n_seg + 1, 4), dtype=torch.int32, device=x.device)
+    _cuda(sse_out, torch.float64, "sse_out")
+    _cuda(argmin_out, torch.int32, "argmin_out")
+    if tuple(sse_out.shape) != (n_seg, len(a), len(r)) or tuple(argmin_out.shape) != (n_seg + 1, 4):
+        raise ValueError("sse_out / argmin_out have the wrong shape")
+    with torch.cuda.device(x.device):
+        st = lib().awq_score_grid_static_scratch(
+            x.data_ptr(), m, w.data_ptr(), n, k, group, int(bool(symmetric)), a.ctypes.data,
+            len(a), r.ctypes.data, len(r), None if seg is None else seg.ctypes.data, n_seg,
+            sse_out.data_ptr(), argmin_out.data_ptr(), _stream(x.device))
+    if st == 5:  # W4_ERR_WORKSPACE: the problem does not fit the static scratch
+        raise W4Error(st, "awq_score_grid_static_scratch: " + lib().w4_last_error().decode())
+    _check(st, "awq_score_grid_static_scratch")
+    return sse_out, argmin_out
 
 
 def device_error(clear: bool = True) -> int:

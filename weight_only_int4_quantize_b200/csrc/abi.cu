@@ -386,6 +386,37 @@ w4_status awq_score_grid(const void* x_bf16, int64_t M, const void* w_bf16, int6
                      "awq argmin");
 }
 
+// Variant of awq_score_grid for callers that cannot allocate a workspace:
+// the scratch is the library's fixed device array (noalloc.cu).  Nothing here
+// allocates; the only CUDA call before the existing entry point is the
+// once-per-device address lookup.
+w4_status awq_score_grid_static_scratch(const void* x_bf16, int64_t M, const void* w_bf16,
+                                        int64_t N, int64_t K, int group, int symmetric,
+                                        const float* alphas, int n_alpha, const float* shrinks,
+                                        int n_shrink, const int64_t* seg_offsets, int n_seg,
+                                        double* sse_out, int32_t* argmin_out, void* stream) {
+  const size_t need = w4_awq_workspace_bytes(M, N, K, n_alpha, n_shrink, n_seg);
+  if (need > W4_AWQ_STATIC_SCRATCH_BYTES) {
+    // Without a workspace the shared validation reports any earlier argument
+    // error first and launches nothing; W4_ERR_WORKSPACE means only the size.
+    const w4_status st = awq_score_grid(x_bf16, M, w_bf16, N, K, group, symmetric, alphas,
+                                        n_alpha, shrinks, n_shrink, seg_offsets, n_seg, sse_out,
+                                        argmin_out, nullptr, 0, stream);
+    if (st == W4_ERR_WORKSPACE)
+      snprintf(g_last_error, sizeof(g_last_error),
+               "awq_score_grid_static_scratch: the problem needs %zu bytes of scratch, the "
+               "static scratch holds %zu; use awq_score_grid with a workspace",
+               need, static_cast<size_t>(W4_AWQ_STATIC_SCRATCH_BYTES));
+    return st;
+  }
+  void* scratch = nullptr;
+  const w4_status st = cuda_status(awq_static_scratch_address(&scratch), "static scratch address");
+  if (st != W4_OK) return st;
+  return awq_score_grid(x_bf16, M, w_bf16, N, K, group, symmetric, alphas, n_alpha, shrinks,
+                        n_shrink, seg_offsets, n_seg, sse_out, argmin_out, scratch,
+                        W4_AWQ_STATIC_SCRATCH_BYTES, stream);
+}
+
 w4_status w4_device_error(int clear, uint32_t* code_out) {
   unsigned v = 0;
   w4_status st = cuda_status(cudaMemcpyFromSymbol(&v, g_w4_device_error, sizeof(v)),

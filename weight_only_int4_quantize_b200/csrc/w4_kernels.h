@@ -81,5 +81,9 @@ cudaError_t launch_awq_reduce(const double* partials, int n_cand, int n_seg, int
 cudaError_t launch_awq_argmin(const double* sse, int n_seg, int n_a, int n_r, int c1,
                               int32_t* out, cudaStream_t stream);
 
+// Device address of the fixed scratch behind awq_score_grid_static_scratch
+// on the current device (looked up once per device, then cached).
+cudaError_t awq_static_scratch_address(void** ptr);
+
 
 }  // namespace w4
