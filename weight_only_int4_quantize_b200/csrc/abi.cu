@@ -135,14 +135,15 @@ w4_status w4_quantize_pack(const void* w_bf16, int64_t N, int64_t K, int group, 
   if (st != W4_OK) return st;
   if (group != 128) return W4_ERR_UNSUPPORTED;
   int sms = 0;
-  st = device_info(&sms, nullptr);
+  unsigned* err = nullptr;
+  st = device_info(&sms, &err);
   if (st != W4_OK) return st;
   QuantBatch b;
   b.count = 0;
   b.unit_start[0] = 0;
   quant_batch_add(b, w_bf16, N, K, awq_s, shrink, qweight, scales_f16, zeros_f16);
   return cuda_status(launch_quantize_pack_batch(b, symmetric != 0,
-                                                static_cast<cudaStream_t>(stream), sms),
+                                                static_cast<cudaStream_t>(stream), sms, err),
                      "quantize+pack launch");
 }
 
@@ -157,7 +158,8 @@ w4_status w4_quantize_pack_batched(const w4_quant_item* items, int count, int gr
     if (st != W4_OK) return st;
   }
   int sms = 0;
-  w4_status st = device_info(&sms, nullptr);
+  unsigned* err = nullptr;
+  w4_status st = device_info(&sms, &err);
   if (st != W4_OK) return st;
   for (int i0 = 0; i0 < count; i0 += kQuantBatch) {
     QuantBatch b;
@@ -169,7 +171,7 @@ w4_status w4_quantize_pack_batched(const w4_quant_item* items, int count, int gr
                       it.zeros_f16);
     }
     st = cuda_status(launch_quantize_pack_batch(b, symmetric != 0,
-                                                static_cast<cudaStream_t>(stream), sms),
+                                                static_cast<cudaStream_t>(stream), sms, err),
                      "batched quantize+pack launch");
     if (st != W4_OK) return st;
   }

@@ -32,12 +32,12 @@ struct QuantBatch {
   uint16_t* zeros[kQuantBatch];
   int64_t n_groups[kQuantBatch];
   int64_t groups_per_row[kQuantBatch];
-  int64_t unit_start[kQuantBatch + 1];  // prefix sums of ceil(groups / 8)
+  int64_t unit_start[kQuantBatch + 1];  // prefix sums of ceil(groups / 32) (chunks)
 };
 void quant_batch_add(QuantBatch& b, const void* w, int64_t N, int64_t K, const float* s,
                      float shrink, int32_t* qweight, uint16_t* scales, uint16_t* zeros);
 cudaError_t launch_quantize_pack_batch(const QuantBatch& b, bool symmetric, cudaStream_t stream,
-                                       int num_sms);
+                                       int num_sms, unsigned* err);
 
 // Up to kGemvBatch independent linears with the same token count (<= 16)
 // decoded by one launch; tensor maps travel in the kernel parameter.
