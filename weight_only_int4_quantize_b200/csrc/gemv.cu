@@ -56,11 +56,13 @@ __host__ __device__ inline GemvLayout gemv_layout(int nt, int gs_max) {
   GemvLayout L;
   const int tokens = 8 * nt;
   L.x_half = tokens * 128;                      // tokens x 64 channels, bf16
-  L.stage = kWTileBytes + 2 * L.x_half;         // multiple of 1024
-  // Three (two for 16 tokens) stages per consumer warp keep groups in flight
-  // while a warp computes; stage s is only ever consumed by warp s % 4 (the
-  // ring length is a multiple of the warp count whenever a stage is reused).
-  const int max_stages = (nt == 1 ? 3 : 2) * kConsumerWarps;
+  // Up to 8 tokens the stages hold weights only (consumers read x from
+  // global memory, where it stays cached), six per consumer warp; 16 tokens
+  // take the x tile through the stage as well, two stages per warp.  Stage s
+  // is only ever consumed by warp s % 4 (the ring length is a multiple of the
+  // warp count whenever a stage is reused).
+  L.stage = nt == 1 ? kWTileBytes : kWTileBytes + 2 * L.x_half;  // multiple of 1024
+  const int max_stages = (nt == 1 ? 6 : 2) * kConsumerWarps;
   L.stages = gs_max < max_stages ? (gs_max < 1 ? 1 : gs_max) : max_stages;
   L.ring = 0;
   L.sz = L.ring + L.stages * L.stage;            // [64][gs_max] (scale | zero << 16)
@@ -203,7 +205,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     // ------------------------------------------------------- producer ----
     if (lane == 0) {
       tma_prefetch_desc(tmap_w);
-      tma_prefetch_desc(tmap_x);
+      if (NT == 2) tma_prefetch_desc(tmap_x);
       const uint32_t stage_tx = L.stage;
       // Stages whose weight tile was issued before the dependency wait.
       const int pre = static_weights ? min(gs, S) : 0;
@@ -224,8 +226,10 @@ __global__ void __launch_bounds__(kThreads, 2)
           mbar_arrive_expect_tx(full(s), stage_tx);
           tma_load_2d(st, tmap_w, gr * 64, row0, full(s));
         }
-        tma_load_2d(st + kWTileBytes, tmap_x, gr * 128, 0, full(s));
-        tma_load_2d(st + kWTileBytes + L.x_half, tmap_x, gr * 128 + 64, 0, full(s));
+        if (NT == 2) {
+          tma_load_2d(st + kWTileBytes, tmap_x, gr * 128, 0, full(s));
+          tma_load_2d(st + kWTileBytes + L.x_half, tmap_x, gr * 128 + 64, 0, full(s));
+        }
         issued = i + 1;
       }
       if (*abort_flag) {  // drain this CTA's own loads before leaving
@@ -278,20 +282,44 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
         for (int i = 0; i < 4; ++i) acc[rt][n][i] = 0.f;
 
+    // Up to 8 tokens: this lane's x fragment of group i (token g, channels
+    // 32t .. 32t+31 of the group) comes straight from global memory, loaded
+    // one group ahead; tokens beyond M are zero.
+    const __nv_bfloat16* __restrict__ xg = b.xp[item];
+    auto load_xg = [&](int i, uint4 (&dst)[4]) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) dst[j] = make_uint4(0u, 0u, 0u, 0u);
+      if (g < M && i < gs) {
+        const uint4* p = reinterpret_cast<const uint4*>(
+            xg + static_cast<size_t>(g) * K + static_cast<size_t>(g_begin + i) * 128 + 32 * t);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) dst[j] = __ldg(p + j);
+      }
+    };
+    uint4 xnext[4];
+    if (NT == 1) load_xg(warp, xnext);
+
     for (int i = warp; i < gs; i += kConsumerWarps) {
       const int s = i % S;
       if (!mbar_wait(full(s), (i / S) & 1u, abort_flag, err, kKernelIdGemv)) break;
       const uint32_t st = base + L.ring + s * L.stage;
-      // x fragments: token 8n + g, channels 32t + 8j .. +7 (128B-swizzled halves).
+      // x fragments: token 8n + g, channels 32t + 8j .. +7.
       uint4 xv[NT][4];
+      if (NT == 1) {
 #pragma unroll
-      for (int n = 0; n < NT; ++n)
+        for (int j = 0; j < 4; ++j) xv[0][j] = xnext[j];
+        load_xg(i + kConsumerWarps, xnext);
+      } else {
+        // 16 tokens: from the stage's two 128B-swizzled halves.
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const uint32_t c = 4 * (t & 1) + j;
-          xv[n][j] = lds128(st + kWTileBytes + (t >> 1) * L.x_half + (8 * n + g) * 128 +
-                            ((c ^ g) << 4));
-        }
+        for (int n = 0; n < NT; ++n)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const uint32_t c = 4 * (t & 1) + j;
+            xv[n][j] = lds128(st + kWTileBytes + (t >> 1) * L.x_half + (8 * n + g) * 128 +
+                              ((c ^ g) << 4));
+          }
+      }
       uint4 wv[4][2];
 #pragma unroll
       for (int rt = 0; rt < 4; ++rt) {
@@ -492,6 +520,7 @@ cudaError_t gemv_batch_add(GemvBatch& b, const void* x, const int32_t* qw, const
                 static_cast<uint64_t>(K) * 2, 64, b.M <= 8 ? 8 : 16,
                 CU_TENSOR_MAP_SWIZZLE_128B) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
+  b.xp[i] = static_cast<const __nv_bfloat16*>(x);
   b.scales[i] = sc;
   b.zeros[i] = z;
   b.y[i] = static_cast<__nv_bfloat16*>(y);

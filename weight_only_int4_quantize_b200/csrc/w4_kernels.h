@@ -45,6 +45,7 @@ constexpr int kGemvBatch = 32;
 struct GemvBatch {
   CUtensorMap tw[kGemvBatch];  // packed codes, uint8 [N, K/2], box 64 x 64
   CUtensorMap tx[kGemvBatch];  // x, bf16 [M, K], box 64 x tokens, 128B swizzle
+  const __nv_bfloat16* xp[kGemvBatch];  // x, bf16 [M, K] (read directly for <= 8 tokens)
   const uint16_t* scales[kGemvBatch];
   const uint16_t* zeros[kGemvBatch];
   __nv_bfloat16* y[kGemvBatch];
