@@ -4,6 +4,7 @@ timing.  Inputs are seeded and generated on the device.
     python -m weight_only_int4_quantize_b200.cases quantize --n 17408 --k 5120 [--sym]
     python -m weight_only_int4_quantize_b200.cases linear --m 8 --n 17408 --k 5120 [--sym] [--gemm]
     python -m weight_only_int4_quantize_b200.cases awq --m 2048 --n 1024 --k 2048 --na 20 --nr 10
+    python -m weight_only_int4_quantize_b200.cases decode_batch --m 1 --blocks 4
 
 Each case captures --iters launches in one CUDA graph (so host launch
 overhead does not count), replays it once to warm up, times one replay with
@@ -59,7 +60,9 @@ def _time(fn, iters, graph=True):
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("case", choices=["quantize", "linear", "awq"])
+    ap.add_argument("case", choices=["quantize", "linear", "awq", "decode_batch"])
+    ap.add_argument("--blocks", type=int, default=4,
+                    help="decode_batch: Qwen3-1.7B-shaped blocks (7 linears each) in one batch")
     ap.add_argument("--m", type=int, default=8)
     ap.add_argument("--n", type=int, default=4096)
     ap.add_argument("--k", type=int, default=4096)
@@ -91,6 +94,26 @@ def main():
         ms = _time(lambda: w4.w4a16_linear(x, qw, sc, zr, flags=flags, out=y), a.iters, not a.eager)
         b = a.n * a.k * (0.5 + (2 if a.sym else 4) / 128) + 2 * a.m * (a.k + a.n)
         out.update(ms=ms, gbs=b / ms / 1e6, tflops=2.0 * a.m * a.n * a.k / ms / 1e9)
+    elif a.case == "decode_batch":
+        # a.blocks x 7 independent linears at a.m tokens through
+        # w4a16_linear_batched (asymmetric), as one decode step would run them.
+        del w
+        items, byts = [], 0.0
+        for bi in range(a.blocks):
+            for li, (_name, k, n) in enumerate(synth.QWEN3_1P7B_BLOCK):
+                wb = _weights(n, k, 100 + 7 * bi + li)
+                qw, sc, zr = w4.quantize_pack(wb, False)
+                del wb
+                g = torch.Generator(device="cuda")
+                g.manual_seed(200 + 7 * bi + li)
+                x = torch.randn(a.m, k, generator=g, device="cuda").to(torch.bfloat16)
+                y = torch.empty(a.m, n, dtype=torch.bfloat16, device="cuda")
+                items.append((x, qw, sc, zr, y))
+                byts += n * k * (0.5 + 4 / 128) + 2 * a.m * (k + n)
+        arr = w4.linear_items(items)
+        flags = w4.LINEAR_PDL | w4.LINEAR_STATIC_WEIGHTS if a.pdl else 0
+        ms = _time(lambda: w4.w4a16_linear_batched(arr, a.m, flags), a.iters, not a.eager)
+        out.update(ms=ms, gbs=byts / ms / 1e6, linears=len(items))
     else:
         g = torch.Generator(device="cuda")
         g.manual_seed(3)

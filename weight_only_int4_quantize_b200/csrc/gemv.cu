@@ -203,20 +203,27 @@ __global__ void __launch_bounds__(kThreads, 2)
 
   if (warp == kConsumerWarps) {
     // ------------------------------------------------------- producer ----
-    if (lane == 0) {
-      tma_prefetch_desc(tmap_w);
-      if (NT == 2) tma_prefetch_desc(tmap_x);
+    // Lane w < 4 feeds consumer warp w: it refills only the stages that warp
+    // reads (s = w, w + 4, ...), so a slow warp never holds back the others'
+    // loads.
+    if (lane < kConsumerWarps) {
+      if (lane == 0) {
+        tma_prefetch_desc(tmap_w);
+        if (NT == 2) tma_prefetch_desc(tmap_x);
+      }
+      __syncwarp(0xFu);
       const uint32_t stage_tx = L.stage;
       // Stages whose weight tile was issued before the dependency wait.
       const int pre = static_weights ? min(gs, S) : 0;
-      for (int i = 0; i < pre; ++i) {
+      for (int i = lane; i < pre; i += kConsumerWarps) {
         const uint32_t st = base + L.ring + i * L.stage;
         mbar_arrive_expect_tx(full(i), stage_tx);
         tma_load_2d(st, tmap_w, (g_begin + i) * 64, row0, full(i));
       }
       pdl_wait();
-      int issued = 0;
-      for (int i = 0; i < gs; ++i) {
+      int issued = 0;  // groups this lane has issued (its last is issued - 1 ... )
+      int last = -1;
+      for (int i = lane; i < gs; i += kConsumerWarps) {
         const int s = i % S;
         const uint32_t st = base + L.ring + s * L.stage;
         const int gr = g_begin + i;
@@ -230,15 +237,16 @@ __global__ void __launch_bounds__(kThreads, 2)
           tma_load_2d(st + kWTileBytes, tmap_x, gr * 128, 0, full(s));
           tma_load_2d(st + kWTileBytes + L.x_half, tmap_x, gr * 128 + 64, 0, full(s));
         }
-        issued = i + 1;
+        last = i;
+        ++issued;
       }
-      if (*abort_flag) {  // drain this CTA's own loads before leaving
-        for (int i = max(0, issued - S); i < issued; ++i) {
+      if (*abort_flag) {  // drain this lane's own loads before leaving
+        for (int i = last; i >= 0 && i > last - S; i -= kConsumerWarps) {
           volatile int dummy = 0;
-          mbar_wait(full(i % S), (i / S) & 1u, &dummy, err, kKernelIdGemv,
-                    kWaitLimitNs / 4);
+          mbar_wait(full(i % S), (i / S) & 1u, &dummy, err, kKernelIdGemv, kWaitLimitNs / 4);
         }
       }
+      (void)issued;
     }
   } else {
     // ------------------------------------------------------- consumers ---
@@ -296,6 +304,9 @@ __global__ void __launch_bounds__(kThreads, 2)
         for (int j = 0; j < 4; ++j) dst[j] = __ldg(p + j);
       }
     };
+    // x may be written by the preceding kernel: wait for it before the first
+    // direct read (a no-op without programmatic dependent launch).
+    pdl_wait();
     uint4 xnext[4];
     if (NT == 1) load_xg(warp, xnext);
 
