@@ -267,8 +267,20 @@ w4_status w4a16_linear_batched(const w4_linear_item* items, int count, int64_t M
       b.count = 0;
       b.cta_start[0] = 0;
       b.M = mc;
-      for (int i = i0; i < count && i < i0 + kGemvBatch; ++i) {
-        const w4_linear_item& it = items[i];
+      // Longest K first: the launch's longest CTAs start first instead of
+      // trailing at its end (results do not depend on the order).
+      int order[kGemvBatch];
+      const int nb = (count - i0) < kGemvBatch ? (count - i0) : kGemvBatch;
+      for (int j = 0; j < nb; ++j) {
+        int p = j;
+        while (p > 0 && items[i0 + order[p - 1]].K < items[i0 + j].K) {
+          order[p] = order[p - 1];
+          --p;
+        }
+        order[p] = j;
+      }
+      for (int j = 0; j < nb; ++j) {
+        const w4_linear_item& it = items[i0 + order[j]];
         const void* xc = static_cast<const uint16_t*>(it.x_bf16) + m0 * it.K;
         void* yc = static_cast<uint16_t*>(it.y_bf16) + m0 * it.N;
         st = cuda_status(gemv_batch_add(b, xc, it.qweight, it.scales_f16, it.zeros_f16,
