@@ -45,7 +45,28 @@ DECODE_M = (1, 4, 8)
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) over the
+# algorithmic bytes of the same launch, from one ncu capture per kernel (the
+# summaries under profiles/ give the commands), with the digest of the kernel
+# source the capture was taken on.  A changed source reports traffic null.
+TRAFFIC_CAPTURES = {
+    # decode_batch --m 1 --blocks 4: 111.07 MB over 106.92 MB algorithmic
+    "gemv_w4a16": {"source": "gemv.cu", "digest": "fb9e87eb5d8c1cfd", "ratio": 111.07 / 106.92},
+    # quantize 17408 x 5120: 202.90 MB over 225.67 MB (part of the written codes
+    # is still in the write-back L2 when the kernel ends)
+    "quantize_pack": {"source": "quantize.cu", "digest": "fe920be4faac0b8e", "ratio": 202.90 / 225.67},
+}
+
 # --------------------------------------------------------------------------
+
+
+def source_digest(name):
+    import hashlib
+    path = os.path.join(ROOT, "weight_only_int4_quantize_b200", "csrc", name)
+    try:
+        return hashlib.sha256(open(path, "rb").read()).hexdigest()[:16]
+    except OSError:
+        return None
 
 
 def quant_bytes(n, k, sym=False):
@@ -165,13 +186,13 @@ def oracle_sample(step_index: int):
 def cpu_baseline(target_s=12.0):
     """The oracle as it stands, timed on this host on a bounded sample."""
     tot_b, tot_t, i = 0.0, 0.0, 0
-    while tot_t < target_s and i < 28:
+    while tot_t < target_s and i < 196:
         b, t = oracle_sample(i)
         tot_b += b
         tot_t += t
         i += 1
     return {"value": tot_b / tot_t / 1e9, "unit": "GB/s", "cores": cpu_threads(), "kind": "oracle",
-            "sample": f"{i} linears of the Qwen3-1.7B block (rotating shapes): numpy binary32 "
+            "sample": f"{i} linears of the Qwen3-1.7B-shaped blocks (rotating shapes): numpy binary32 "
                       f"quantize+pack, then binary64 decode at M=1,4,8; {tot_t:.1f} s"}
 
 
@@ -497,10 +518,18 @@ def main():
         dom = ("quantize_pack", qb / (q_ms * 1e-3) / 1e9, model.launches["quantize"])
     else:
         dom = ("gemv_w4a16", db / (gemv_ms * 1e-3) / 1e9, model.launches["gemv"])
+    bytes_per_launch = (qb if dom[0] == "quantize_pack" else db) / dom[2]
+    cap = TRAFFIC_CAPTURES.get(dom[0])
+    traffic = None
+    if cap and source_digest(cap["source"]) == cap["digest"]:
+        traffic = cap["ratio"] * bytes_per_launch
     roofline = {"kernel": dom[0], "bound": "hbm", "achieved": dom[1], "peak": hbm, "unit": "GB/s",
-                "frac": dom[1] / hbm, "peak_kind": peak_kind, "traffic": None,
+                "frac": dom[1] / hbm, "peak_kind": peak_kind, "traffic": traffic,
+                "algorithmic_bytes_per_launch": bytes_per_launch,
                 "note": "achieved = algorithmic bytes of the kernel's launches in the timed region "
-                        "/ their CUDA-event time (graph phase, launch gaps included)"}
+                        "/ their CUDA-event time (graph phase, launch gaps included); traffic = "
+                        "the ncu capture's DRAM bytes / algorithmic bytes, times this launch's "
+                        "algorithmic bytes (null once the kernel source differs from the capture's)"}
 
     out = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
