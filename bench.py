@@ -255,8 +255,12 @@ class Model:
         self.d_items = {m: w4.linear_items([(self.x[(m, k)], qw, sc, zr, self.y[m][j])
                                             for j, (k, n, w, qw, sc, zr) in enumerate(self.lin)])
                         for m in DECODE_M}
+        # w4a16_linear_batched launches one GEMV per 32 linears of equal K.
+        per_k = {}
+        for (k, *_r) in self.lin:
+            per_k[k] = per_k.get(k, 0) + 1
         self.launches = {"quantize": -(-len(self.lin) // 64),
-                         "gemv": len(DECODE_M) * -(-len(self.lin) // 32)}
+                         "gemv": len(DECODE_M) * sum(-(-c // 32) for c in per_k.values())}
 
     def quantize_all(self):
         """All 196 weights through w4_quantize_pack_batched (64 per launch)."""

@@ -2,6 +2,7 @@
 // argument validation, path selection and workspace layout.  Nothing is
 // launched unless every check passes; the library allocates nothing.
 #include <cmath>
+#include <cstdint>
 #include <cstdio>
 #include <cstring>
 
@@ -260,36 +261,41 @@ w4_status w4a16_linear_batched(const w4_linear_item* items, int count, int64_t M
     }
     return W4_OK;
   }
+  // Launches group the linears by K, largest K first: a launch's shared
+  // memory ring is sized by its longest K slice, so launches of one K size
+  // their CTAs exactly (short K fits more CTAs per SM), and no launch ends
+  // with a trail of long CTAs.  Results do not depend on the grouping.
   for (int64_t m0 = 0; m0 < M; m0 += 16) {
     const int mc = static_cast<int>(M - m0 < 16 ? M - m0 : 16);
-    for (int i0 = 0; i0 < count; i0 += kGemvBatch) {
+    int64_t k_prev = INT64_MAX;
+    for (;;) {
+      int64_t kv = 0;  // the largest K below k_prev
+      for (int i = 0; i < count; ++i)
+        if (items[i].K < k_prev && items[i].K > kv) kv = items[i].K;
+      if (kv == 0) break;
+      k_prev = kv;
       GemvBatch b;
       b.count = 0;
       b.cta_start[0] = 0;
       b.M = mc;
-      // Longest K first: the launch's longest CTAs start first instead of
-      // trailing at its end (results do not depend on the order).
-      int order[kGemvBatch];
-      const int nb = (count - i0) < kGemvBatch ? (count - i0) : kGemvBatch;
-      for (int j = 0; j < nb; ++j) {
-        int p = j;
-        while (p > 0 && items[i0 + order[p - 1]].K < items[i0 + j].K) {
-          order[p] = order[p - 1];
-          --p;
+      for (int i = 0; i <= count; ++i) {
+        if (i < count && items[i].K == kv) {
+          const w4_linear_item& it = items[i];
+          const void* xc = static_cast<const uint16_t*>(it.x_bf16) + m0 * it.K;
+          void* yc = static_cast<uint16_t*>(it.y_bf16) + m0 * it.N;
+          st = cuda_status(gemv_batch_add(b, xc, it.qweight, it.scales_f16, it.zeros_f16,
+                                          static_cast<int>(it.N), static_cast<int>(it.K), yc),
+                           "tensor map");
+          if (st != W4_OK) return st;
         }
-        order[p] = j;
+        if (b.count == kGemvBatch || (i == count && b.count > 0)) {
+          st = cuda_status(launch_gemv_batch(b, sym, pdl, stat, s, sms, err),
+                           "batched decode GEMV launch");
+          if (st != W4_OK) return st;
+          b.count = 0;
+          b.cta_start[0] = 0;
+        }
       }
-      for (int j = 0; j < nb; ++j) {
-        const w4_linear_item& it = items[i0 + order[j]];
-        const void* xc = static_cast<const uint16_t*>(it.x_bf16) + m0 * it.K;
-        void* yc = static_cast<uint16_t*>(it.y_bf16) + m0 * it.N;
-        st = cuda_status(gemv_batch_add(b, xc, it.qweight, it.scales_f16, it.zeros_f16,
-                                        static_cast<int>(it.N), static_cast<int>(it.K), yc),
-                         "tensor map");
-        if (st != W4_OK) return st;
-      }
-      st = cuda_status(launch_gemv_batch(b, sym, pdl, stat, s, sms, err), "batched decode GEMV launch");
-      if (st != W4_OK) return st;
     }
   }
   return W4_OK;
