@@ -29,32 +29,41 @@ namespace w4 {
 
 namespace {
 
-constexpr int BM = 128;
+constexpr int BM = 128;   // rows of one UMMA (and of a CTA tile with MT = 1)
 constexpr int BN = 256;
 constexpr int BK = 64;
-constexpr int kStages = 4;
 constexpr int kThreads = 320;
 constexpr int kProducerWarps = 8;
-constexpr uint32_t kTileABytes = BM * BK * 2;  // 16 KB
 constexpr uint32_t kTileBBytes = BN * BK * 2;  // 32 KB
-constexpr uint32_t kTmemCols = 256;
 constexpr int kLoadAhead = 4;  // stages of packed codes in flight per producer thread
+
+// A CTA tile is MT x 128 rows by 256 columns: MT UMMAs per k-step share one
+// B tile, so with MT = 2 each dequantized weight feeds twice the flops.
+// Accumulators: MT x 256 fp32 TMEM columns.  Stages: 4 (MT = 1) or 3.
+template <int MT>
+struct Tile {
+  static constexpr int kStages = MT == 1 ? 4 : 3;
+  static constexpr uint32_t kTileABytes = MT * BM * BK * 2;  // 16 or 32 KB
+  static constexpr uint32_t kTmemCols = MT * 256;
+};
 
 enum : int { kBDequant = 0, kBTma = 1 };
 enum : int { kEpiStoreBf16 = 0, kEpiSumSquares = 1 };
 
 constexpr unsigned kKernelIdGemm = 2;
 
+template <int MT>
 struct SmemLayout {
+  static constexpr int kStages = Tile<MT>::kStages;
   // offsets from a 1024-byte aligned base
   static constexpr uint32_t a = 0;
-  static constexpr uint32_t b = a + kStages * kTileABytes;
+  static constexpr uint32_t b = a + kStages * Tile<MT>::kTileABytes;
   static constexpr uint32_t bars = b + kStages * kTileBBytes;
   // full_a[S], full_b[S], empty[S], acc_full, done
   static constexpr uint32_t misc = bars + (3 * kStages + 2) * 8;
   static constexpr uint32_t total = misc + 64 + 16 * 16 * 8;  // + chunk sums
+  static constexpr size_t bytes = total + 1024;
 };
-constexpr size_t kGemmSmemBytes = SmemLayout::total + 1024;
 
 struct SumSqArgs {
   double* partials;     // [n_cand][n_seg][tiles]
@@ -130,7 +139,7 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v) {
                : "memory");
 }
 
-template <int BSRC, int EPI, bool SYM>
+template <int BSRC, int EPI, bool SYM, int MT>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_a,
                    const __grid_constant__ CUtensorMap tmap_b,  // kBTma only
@@ -144,22 +153,26 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t base = (raw_addr + 1023u) & ~1023u;
   uint8_t* base_ptr = smem_raw + (base - raw_addr);
 
-  const uint32_t sA = base + SmemLayout::a;
-  const uint32_t sB = base + SmemLayout::b;
-  const uint32_t bar0 = base + SmemLayout::bars;
+  using SL = SmemLayout<MT>;
+  constexpr int kStages = SL::kStages;
+  constexpr uint32_t kTileABytes = Tile<MT>::kTileABytes;
+  constexpr uint32_t kTmemCols = Tile<MT>::kTmemCols;
+  const uint32_t sA = base + SL::a;
+  const uint32_t sB = base + SL::b;
+  const uint32_t bar0 = base + SL::bars;
   auto full_a = [&](int s) { return bar0 + 8u * s; };
   auto full_b = [&](int s) { return bar0 + 8u * (kStages + s); };
   auto empty = [&](int s) { return bar0 + 8u * (2 * kStages + s); };
   const uint32_t acc_full = bar0 + 8u * (3 * kStages);
   const uint32_t done_bar = acc_full + 8u;
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(base_ptr + SmemLayout::misc);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base_ptr + SmemLayout::misc + 8);
-  double* chunk_sums = reinterpret_cast<double*>(base_ptr + SmemLayout::misc + 64);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(base_ptr + SL::misc);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base_ptr + SL::misc + 8);
+  double* chunk_sums = reinterpret_cast<double*>(base_ptr + SL::misc + 64);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int n0 = blockIdx.x * BN;
-  const int m0 = blockIdx.y * BM;
+  const int m0 = blockIdx.y * (MT * BM);
   const int cand = blockIdx.z;
   const int num_kb = K / BK;
 
@@ -232,8 +245,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint64_t db = sdesc_k_sw128(sB + s * kTileBBytes);
 #pragma unroll
         for (int kk = 0; kk < BK / 16; ++kk) {
-          // +32 bytes along K inside the swizzle atom = +2 in the address field
-          umma_f16(tmem_base, da + 2ull * kk, db + 2ull * kk, idesc, (kb | kk) != 0);
+          // +32 bytes along K inside the swizzle atom = +2 in the address
+          // field; row block mt of A starts 16 KB (+1024) further.
+#pragma unroll
+          for (int mt = 0; mt < MT; ++mt)
+            umma_f16(tmem_base + 256u * mt, da + 1024ull * mt + 2ull * kk, db + 2ull * kk, idesc,
+                     (kb | kk) != 0);
         }
         issued = true;
         umma_commit(empty(s));
@@ -332,12 +349,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool ok = mbar_wait(acc_full, 0, abort_flag, err, kKernelIdGemm);
     tc_fence_after();
     if (ok) {
-      const int m = m0 + 32 * q + lane;
       if (EPI == kEpiStoreBf16) {
+        for (int mt = 0; mt < MT; ++mt)
         for (int c = 0; c < 8; ++c) {
+          const int m = m0 + 128 * mt + 32 * q + lane;
           const int col = 128 * ch + 16 * c;
           uint32_t r[16];
-          tmem_ld_32x32b_x16(tmem_base + (static_cast<uint32_t>(32 * q) << 16) + col, r);
+          tmem_ld_32x32b_x16(tmem_base + (static_cast<uint32_t>(32 * q) << 16) + 256 * mt + col, r);
           tmem_ld_wait();
           const int n = n0 + col;
           if (m < M && n < N) {
@@ -363,6 +381,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         // Sum of squares per 16-column chunk: thread -> fixed-order shuffle
         // tree over the 32 rows of this warp -> shared -> fixed order over
         // the 4 warps of this column half -> per-segment sums.
+        static_assert(EPI != kEpiSumSquares || MT == 1, "sum of squares uses 128-row tiles");
+        const int m = m0 + 32 * q + lane;
         for (int c = 0; c < 8; ++c) {
           const int col = 128 * ch + 16 * c;
           uint32_t r[16];
@@ -433,7 +453,7 @@ CUresult encode_tmap(CUtensorMap* map, CUtensorMapDataType dt, int rank, const u
 
 // One instantiation per kernel (the cache below must be per kernel, and
 // every instantiation of gemm_tc_kernel has the same function type).
-template <auto kern>
+template <auto kern, size_t kSmemBytes>
 cudaError_t launch_gemm(dim3 grid, bool pdl, cudaStream_t stream,
                         const CUtensorMap& ta, const CUtensorMap& tb, const uint32_t* qw,
                         const uint16_t* sc, const uint16_t* z, __nv_bfloat16* y,
@@ -447,14 +467,14 @@ cudaError_t launch_gemm(dim3 grid, bool pdl, cudaStream_t stream,
   if (e != cudaSuccess) return e;
   if (dev >= 64 || !(__atomic_load_n(&attr_done, __ATOMIC_ACQUIRE) & (1ull << dev))) {
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(kGemmSmemBytes));
+                             static_cast<int>(kSmemBytes));
     if (e != cudaSuccess) return e;
     if (dev < 64) __atomic_fetch_or(&attr_done, 1ull << dev, __ATOMIC_RELEASE);
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = kGemmSmemBytes;
+  cfg.dynamicSmemBytes = kSmemBytes;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   if (pdl) {
@@ -471,23 +491,41 @@ cudaError_t launch_gemm(dim3 grid, bool pdl, cudaStream_t stream,
 cudaError_t launch_prefill_gemm(const void* x, int M, const int32_t* qw, const uint16_t* sc,
                                 const uint16_t* z, int N, int K, void* y, bool pdl,
                                 bool static_w, cudaStream_t stream, unsigned* err) {
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  // 256-row tiles halve the dequantization per flop; used while they still
+  // give every SM a tile.
+  const int n_tiles = (N + BN - 1) / BN;
+#ifndef W4_GEMM_TALL
+#define W4_GEMM_TALL 1
+#endif
+  const bool tall = W4_GEMM_TALL && M >= 2 * BM && n_tiles * ((M + 2 * BM - 1) / (2 * BM)) >= sms;
+  const int bm = tall ? 2 * BM : BM;
   CUtensorMap ta, tb;
   const uint64_t dims[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(M)};
   const uint64_t str[1] = {static_cast<uint64_t>(K) * 2};
-  const uint32_t box[2] = {BK, BM};
+  const uint32_t box[2] = {BK, static_cast<uint32_t>(bm)};
   if (encode_tmap(&ta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, dims, str, box, x) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
   tb = ta;  // unused by the dequant variant
   SumSqArgs ss = {};
-  dim3 grid((N + BN - 1) / BN, (M + BM - 1) / BM, 1);
+  dim3 grid(n_tiles, (M + bm - 1) / bm, 1);
   const uint32_t* q = reinterpret_cast<const uint32_t*>(qw);
   __nv_bfloat16* yp = static_cast<__nv_bfloat16*>(y);
   const int ps = (pdl && static_w) ? 1 : 0;
+  if (tall) {
+    if (z == nullptr)
+      return launch_gemm<gemm_tc_kernel<kBDequant, kEpiStoreBf16, true, 2>, SmemLayout<2>::bytes>(
+          grid, pdl, stream, ta, tb, q, sc, z, yp, ss, M, N, K, ps, err);
+    return launch_gemm<gemm_tc_kernel<kBDequant, kEpiStoreBf16, false, 2>, SmemLayout<2>::bytes>(
+        grid, pdl, stream, ta, tb, q, sc, z, yp, ss, M, N, K, ps, err);
+  }
   if (z == nullptr)
-    return launch_gemm<gemm_tc_kernel<kBDequant, kEpiStoreBf16, true>>(grid, pdl, stream, ta, tb,
-                       q, sc, z, yp, ss, M, N, K, ps, err);
-  return launch_gemm<gemm_tc_kernel<kBDequant, kEpiStoreBf16, false>>(grid, pdl, stream, ta, tb,
-                     q, sc, z, yp, ss, M, N, K, ps, err);
+    return launch_gemm<gemm_tc_kernel<kBDequant, kEpiStoreBf16, true, 1>, SmemLayout<1>::bytes>(
+        grid, pdl, stream, ta, tb, q, sc, z, yp, ss, M, N, K, ps, err);
+  return launch_gemm<gemm_tc_kernel<kBDequant, kEpiStoreBf16, false, 1>, SmemLayout<1>::bytes>(
+      grid, pdl, stream, ta, tb, q, sc, z, yp, ss, M, N, K, ps, err);
 }
 
 cudaError_t launch_sumsq_gemm(const void* a_f16, int M, const void* b_f16, int N, int K,
@@ -511,8 +549,8 @@ cudaError_t launch_sumsq_gemm(const void* a_f16, int M, const void* b_f16, int N
   for (int i = 0; i <= n_seg; ++i) ss.seg_off[i] = seg_off[i];
   dim3 grid((N + BN - 1) / BN, (M + BM - 1) / BM, n_cand);
   ss.tiles = grid.x * grid.y;
-  return launch_gemm<gemm_tc_kernel<kBTma, kEpiSumSquares, false>>(grid, false, stream, ta, tb,
-                     nullptr, nullptr, nullptr, nullptr, ss, M, N, K, 0, err);
+  return launch_gemm<gemm_tc_kernel<kBTma, kEpiSumSquares, false, 1>, SmemLayout<1>::bytes>(
+      grid, false, stream, ta, tb, nullptr, nullptr, nullptr, nullptr, ss, M, N, K, 0, err);
 }
 
 int sumsq_tiles(int M, int N) { return ((N + BN - 1) / BN) * ((M + BM - 1) / BM); }
