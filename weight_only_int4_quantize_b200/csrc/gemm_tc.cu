@@ -494,13 +494,15 @@ cudaError_t launch_prefill_gemm(const void* x, int M, const int32_t* qw, const u
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess)
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  // 256-row tiles halve the dequantization per flop; used while they still
-  // give every SM a tile.
+  // A 256-row tile costs the same dequantization as a 128-row one (its B
+  // tile is the same) for twice the flops, and the kernel is bound by that
+  // dequantization: 256-row tiles win whenever they need fewer waves of CTAs
+  // (one CTA per SM), and tie when both fit in one wave (then the 128-row
+  // tiles, using more SMs, are kept).
   const int n_tiles = (N + BN - 1) / BN;
-#ifndef W4_GEMM_TALL
-#define W4_GEMM_TALL 1
-#endif
-  const bool tall = W4_GEMM_TALL && M >= 2 * BM && n_tiles * ((M + 2 * BM - 1) / (2 * BM)) >= sms;
+  const long t1 = static_cast<long>(n_tiles) * ((M + BM - 1) / BM);
+  const long t2 = static_cast<long>(n_tiles) * ((M + 2 * BM - 1) / (2 * BM));
+  const bool tall = M >= 2 * BM && (t2 + sms - 1) / sms < (t1 + sms - 1) / sms;
   const int bm = tall ? 2 * BM : BM;
   CUtensorMap ta, tb;
   const uint64_t dims[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(M)};
