@@ -65,11 +65,13 @@ __host__ __device__ inline GemvLayout gemv_layout(int nt, int gs_max) {
   const int max_stages = (nt == 1 ? 6 : 2) * kConsumerWarps;
   L.stages = gs_max < max_stages ? (gs_max < 1 ? 1 : gs_max) : max_stages;
   L.ring = 0;
-  L.sz = L.ring + L.stages * L.stage;            // [64][gs_max] (scale | zero << 16)
+  // Scale table [64][gs_max | 1] (scale | zero << 16): an odd row pitch puts
+  // the eight rows that one epilogue read touches in distinct banks.
+  L.sz = L.ring + L.stages * L.stage;
   // The per-warp partial sums reuse the ring once every stage is consumed.
   L.red = L.ring;                                // [4][tokens][64] f32
   const uint32_t red_end = L.red + kConsumerWarps * tokens * kRows * 4;
-  L.part = L.sz + ((kRows * gs_max * 4 + 15) & ~15u);  // [tokens][64] f32
+  L.part = L.sz + ((kRows * (gs_max | 1) * 4 + 15) & ~15u);  // [tokens][64] f32
   if (L.part < red_end) L.part = red_end;
   L.bars = L.part + tokens * kRows * 4;          // full[S], empty[S]
   L.misc = L.bars + 2 * L.stages * 8;
@@ -276,7 +278,7 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
         for (int j = 0; j < 10; ++j) {
           const int q = q0 + 2 * j + (threadIdx.x & 1);
-          if (q < gs) s_sz[r * gs_max + q] = sv[j] | (zv[j] << 16);
+          if (q < gs) s_sz[r * (gs_max | 1) + q] = sv[j] | (zv[j] << 16);
         }
       }
     }
@@ -363,8 +365,8 @@ __global__ void __launch_bounds__(kThreads, 2)
         for (int n = 0; n < NT; ++n) tile_group(c[rt][n], wv[rt][0], wv[rt][1], xv[n]);
 #pragma unroll
       for (int rt = 0; rt < 4; ++rt) {
-        const uint32_t sza = s_sz[(16 * rt + g) * gs_max + i];
-        const uint32_t szb = s_sz[(16 * rt + g + 8) * gs_max + i];
+        const uint32_t sza = s_sz[(16 * rt + g) * (gs_max | 1) + i];
+        const uint32_t szb = s_sz[(16 * rt + g + 8) * (gs_max | 1) + i];
         const float sa = __half2float(__ushort_as_half(static_cast<uint16_t>(sza & 0xFFFFu)));
         const float sb = __half2float(__ushort_as_half(static_cast<uint16_t>(szb & 0xFFFFu)));
         const float za = 128.0f + __half2float(__ushort_as_half(static_cast<uint16_t>(sza >> 16)));
