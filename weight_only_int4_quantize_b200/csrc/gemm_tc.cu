@@ -30,21 +30,25 @@ namespace w4 {
 namespace {
 
 constexpr int BM = 128;   // rows of one UMMA (and of a CTA tile with MT = 1)
-constexpr int BN = 256;
+constexpr int BN = 256;   // widest B tile (the sum-of-squares GEMM always uses it)
 constexpr int BK = 64;
 constexpr int kThreads = 320;
 constexpr int kProducerWarps = 8;
-constexpr uint32_t kTileBBytes = BN * BK * 2;  // 32 KB
 constexpr int kLoadAhead = 4;  // stages of packed codes in flight per producer thread
 
-// A CTA tile is MT x 128 rows by 256 columns: MT UMMAs per k-step share one
-// B tile, so with MT = 2 each dequantized weight feeds twice the flops.
-// Accumulators: MT x 256 fp32 TMEM columns.  Stages: 4 (MT = 1) or 3.
-template <int MT>
+// A CTA tile is MT x 128 rows by NB (128 or 256) columns: MT UMMAs per k-step
+// share one B tile, so with MT = 2 each dequantized weight feeds twice the
+// flops, and NB = 128 halves a CTA's dequantization for grids that would
+// otherwise leave SMs idle.  Accumulators: MT x NB fp32 TMEM columns.
+template <int MT, int NB>
 struct Tile {
-  static constexpr int kStages = MT == 1 ? 4 : 3;
   static constexpr uint32_t kTileABytes = MT * BM * BK * 2;  // 16 or 32 KB
-  static constexpr uint32_t kTmemCols = MT * 256;
+  static constexpr uint32_t kTileBBytes = NB * BK * 2;       // 16 or 32 KB
+  static constexpr int kStages =
+      static_cast<int>((196u * 1024u) / (kTileABytes + kTileBBytes)) > 6
+          ? 6
+          : static_cast<int>((196u * 1024u) / (kTileABytes + kTileBBytes));
+  static constexpr uint32_t kTmemCols = MT * NB;
 };
 
 enum : int { kBDequant = 0, kBTma = 1 };
@@ -52,13 +56,13 @@ enum : int { kEpiStoreBf16 = 0, kEpiSumSquares = 1 };
 
 constexpr unsigned kKernelIdGemm = 2;
 
-template <int MT>
+template <int MT, int NB>
 struct SmemLayout {
-  static constexpr int kStages = Tile<MT>::kStages;
+  static constexpr int kStages = Tile<MT, NB>::kStages;
   // offsets from a 1024-byte aligned base
   static constexpr uint32_t a = 0;
-  static constexpr uint32_t b = a + kStages * Tile<MT>::kTileABytes;
-  static constexpr uint32_t bars = b + kStages * kTileBBytes;
+  static constexpr uint32_t b = a + kStages * Tile<MT, NB>::kTileABytes;
+  static constexpr uint32_t bars = b + kStages * Tile<MT, NB>::kTileBBytes;
   // full_a[S], full_b[S], empty[S], acc_full, done
   static constexpr uint32_t misc = bars + (3 * kStages + 2) * 8;
   static constexpr uint32_t total = misc + 64 + 16 * 16 * 8;  // + chunk sums
@@ -139,7 +143,7 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v) {
                : "memory");
 }
 
-template <int BSRC, int EPI, bool SYM, int MT>
+template <int BSRC, int EPI, bool SYM, int MT, int NB>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_a,
                    const __grid_constant__ CUtensorMap tmap_b,  // kBTma only
@@ -153,10 +157,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t base = (raw_addr + 1023u) & ~1023u;
   uint8_t* base_ptr = smem_raw + (base - raw_addr);
 
-  using SL = SmemLayout<MT>;
+  using SL = SmemLayout<MT, NB>;
   constexpr int kStages = SL::kStages;
-  constexpr uint32_t kTileABytes = Tile<MT>::kTileABytes;
-  constexpr uint32_t kTmemCols = Tile<MT>::kTmemCols;
+  constexpr uint32_t kTileABytes = Tile<MT, NB>::kTileABytes;
+  constexpr uint32_t kTileBBytes = Tile<MT, NB>::kTileBBytes;
+  constexpr uint32_t kTmemCols = Tile<MT, NB>::kTmemCols;
   const uint32_t sA = base + SL::a;
   const uint32_t sB = base + SL::b;
   const uint32_t bar0 = base + SL::bars;
@@ -171,7 +176,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int n0 = blockIdx.x * BN;
+  const int n0 = blockIdx.x * NB;
   const int m0 = blockIdx.y * (MT * BM);
   const int cand = blockIdx.z;
   const int num_kb = K / BK;
@@ -233,7 +238,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA --
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_f16(BM, BN, EPI == kEpiStoreBf16);
+      constexpr uint32_t idesc = idesc_f16(BM, NB, EPI == kEpiStoreBf16);
       bool issued = false;
       for (int kb = 0; kb < num_kb; ++kb) {
         const int s = kb % kStages;
@@ -249,8 +254,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           // field; row block mt of A starts 16 KB (+1024) further.
 #pragma unroll
           for (int mt = 0; mt < MT; ++mt)
-            umma_f16(tmem_base + 256u * mt, da + 1024ull * mt + 2ull * kk, db + 2ull * kk, idesc,
-                     (kb | kk) != 0);
+            umma_f16(tmem_base + static_cast<uint32_t>(NB) * mt, da + 1024ull * mt + 2ull * kk,
+                     db + 2ull * kk, idesc, (kb | kk) != 0);
         }
         issued = true;
         umma_commit(empty(s));
@@ -267,7 +272,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int pt = threadIdx.x - 64;  // 0..255
     // ------------------------------------------------- B producers ----
     if (BSRC == kBDequant) {
-      // Thread pt owns rows r = it*128 + pt/2 (it = 0, 1) and half (pt & 1)
+      // Thread pt owns rows r = it*128 + pt/2 (it < NB / 128) and half (pt & 1)
       // of each row's 64-channel stage slice: 4 packed words -> 4 chunks.
       // A register ring keeps kLoadAhead stages of codes (and their group's
       // scale/zero) in flight ahead of the stage being written.
@@ -280,7 +285,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint16_t* srow[2];
       const uint16_t* zrow[2];
 #pragma unroll
-      for (int it = 0; it < 2; ++it) {
+      for (int it = 0; it < NB / 128; ++it) {
         rows[it] = it * 128 + (pt >> 1);
         valid[it] = (n0 + rows[it]) < N;
         const size_t row = static_cast<size_t>(valid[it] ? n0 + rows[it] : 0);
@@ -292,7 +297,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t ring_sz[kLoadAhead][2];
       auto fetch = [&](int kb, uint4 (&q)[2], uint32_t (&sz)[2]) {
 #pragma unroll
-        for (int it = 0; it < 2; ++it) {
+        for (int it = 0; it < NB / 128; ++it) {
           q[it] = make_uint4(0, 0, 0, 0);
           sz[it] = 0x48000000u;  // scale 0, zero 8
           if (valid[it] && kb < num_kb) {
@@ -318,7 +323,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           fetch(kb + kLoadAhead, ring[d], ring_sz[d]);
           DqConst dc[2];
 #pragma unroll
-          for (int it = 0; it < 2; ++it)
+          for (int it = 0; it < NB / 128; ++it)
             dc[it] = dq_const(__half2float(__ushort_as_half(static_cast<uint16_t>(csz[it] & 0xFFFFu))),
                               __half2float(__ushort_as_half(static_cast<uint16_t>(csz[it] >> 16))));
           if (!mbar_wait(empty(s), ph ^ 1u, abort_flag, err, kKernelIdGemm)) {
@@ -327,7 +332,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           const uint32_t tile = sB + s * kTileBBytes;
 #pragma unroll
-          for (int it = 0; it < 2; ++it) {
+          for (int it = 0; it < NB / 128; ++it) {
             const uint32_t w4[4] = {cur[it].x, cur[it].y, cur[it].z, cur[it].w};
 #pragma unroll
             for (int j = 0; j < 4; ++j)
@@ -351,11 +356,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (ok) {
       if (EPI == kEpiStoreBf16) {
         for (int mt = 0; mt < MT; ++mt)
-        for (int c = 0; c < 8; ++c) {
+        for (int c = 0; c < NB / 32; ++c) {
           const int m = m0 + 128 * mt + 32 * q + lane;
-          const int col = 128 * ch + 16 * c;
+          const int col = (NB / 2) * ch + 16 * c;
           uint32_t r[16];
-          tmem_ld_32x32b_x16(tmem_base + (static_cast<uint32_t>(32 * q) << 16) + 256 * mt + col, r);
+          tmem_ld_32x32b_x16(tmem_base + (static_cast<uint32_t>(32 * q) << 16) + NB * mt + col, r);
           tmem_ld_wait();
           const int n = n0 + col;
           if (m < M && n < N) {
@@ -381,7 +386,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         // Sum of squares per 16-column chunk: thread -> fixed-order shuffle
         // tree over the 32 rows of this warp -> shared -> fixed order over
         // the 4 warps of this column half -> per-segment sums.
-        static_assert(EPI != kEpiSumSquares || MT == 1, "sum of squares uses 128-row tiles");
+        static_assert(EPI != kEpiSumSquares || (MT == 1 && NB == BN),
+                      "sum of squares uses 128 x 256 tiles");
         const int m = m0 + 32 * q + lane;
         for (int c = 0; c < 8; ++c) {
           const int col = 128 * ch + 16 * c;
@@ -494,16 +500,32 @@ cudaError_t launch_prefill_gemm(const void* x, int M, const int32_t* qw, const u
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess)
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  // A 256-row tile costs the same dequantization as a 128-row one (its B
-  // tile is the same) for twice the flops, and the kernel is bound by that
-  // dequantization: 256-row tiles win whenever they need fewer waves of CTAs
-  // (one CTA per SM), and tie when both fit in one wave (then the 128-row
-  // tiles, using more SMs, are kept).
-  const int n_tiles = (N + BN - 1) / BN;
-  const long t1 = static_cast<long>(n_tiles) * ((M + BM - 1) / BM);
-  const long t2 = static_cast<long>(n_tiles) * ((M + 2 * BM - 1) / (2 * BM));
-  const bool tall = M >= 2 * BM && (t2 + sms - 1) / sms < (t1 + sms - 1) / sms;
-  const int bm = tall ? 2 * BM : BM;
+  // Tile shape (MT x 128 rows, NB columns), one CTA per SM.  Measured time of
+  // one wave of CTAs relative to 128 x 256 tiles (same K): 256 x 256 1.32,
+  // 128 x 256 1.00, 256 x 128 0.80, 128 x 128 0.68 -- the B dequantization
+  // scales with NB and the MMAs with MT x NB.  The shape with the smallest
+  // waves x wave time wins; on equal cost the earlier (larger) one.
+  struct Shape { int mt, nb, cost; };
+  const Shape shapes[4] = {{2, 256, 132}, {1, 256, 100}, {2, 128, 80}, {1, 128, 68}};
+  int best = -1;
+  long best_cost = 0;
+  for (int i = 0; i < 4; ++i) {
+    const Shape sh = shapes[i];
+    if (sh.mt == 2 && M < 2 * BM) continue;  // 256-row tiles only when rows fill them
+    const long tiles = static_cast<long>((N + sh.nb - 1) / sh.nb) *
+                       ((M + sh.mt * BM - 1) / (sh.mt * BM));
+    const long cost = ((tiles + sms - 1) / sms) * sh.cost;
+#ifdef W4_GEMM_FORCE_SHAPE
+    if (i != W4_GEMM_FORCE_SHAPE) continue;
+#endif
+    if (best < 0 || cost < best_cost) {
+      best = i;
+      best_cost = cost;
+    }
+  }
+  if (best < 0) best = 1;
+  const int mt = shapes[best].mt, nb = shapes[best].nb;
+  const int bm = mt * BM;
   CUtensorMap ta, tb;
   const uint64_t dims[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(M)};
   const uint64_t str[1] = {static_cast<uint64_t>(K) * 2};
@@ -512,22 +534,23 @@ cudaError_t launch_prefill_gemm(const void* x, int M, const int32_t* qw, const u
     return cudaErrorInvalidValue;
   tb = ta;  // unused by the dequant variant
   SumSqArgs ss = {};
-  dim3 grid(n_tiles, (M + bm - 1) / bm, 1);
+  dim3 grid((N + nb - 1) / nb, (M + bm - 1) / bm, 1);
   const uint32_t* q = reinterpret_cast<const uint32_t*>(qw);
   __nv_bfloat16* yp = static_cast<__nv_bfloat16*>(y);
   const int ps = (pdl && static_w) ? 1 : 0;
-  if (tall) {
-    if (z == nullptr)
-      return launch_gemm<gemm_tc_kernel<kBDequant, kEpiStoreBf16, true, 2>, SmemLayout<2>::bytes>(
-          grid, pdl, stream, ta, tb, q, sc, z, yp, ss, M, N, K, ps, err);
-    return launch_gemm<gemm_tc_kernel<kBDequant, kEpiStoreBf16, false, 2>, SmemLayout<2>::bytes>(
-        grid, pdl, stream, ta, tb, q, sc, z, yp, ss, M, N, K, ps, err);
-  }
-  if (z == nullptr)
-    return launch_gemm<gemm_tc_kernel<kBDequant, kEpiStoreBf16, true, 1>, SmemLayout<1>::bytes>(
-        grid, pdl, stream, ta, tb, q, sc, z, yp, ss, M, N, K, ps, err);
-  return launch_gemm<gemm_tc_kernel<kBDequant, kEpiStoreBf16, false, 1>, SmemLayout<1>::bytes>(
-      grid, pdl, stream, ta, tb, q, sc, z, yp, ss, M, N, K, ps, err);
+#define W4_PREFILL_LAUNCH(MT_, NB_)                                                          \
+  (z == nullptr                                                                            \
+       ? launch_gemm<gemm_tc_kernel<kBDequant, kEpiStoreBf16, true, MT_, NB_>,              \
+                     SmemLayout<MT_, NB_>::bytes>(grid, pdl, stream, ta, tb, q, sc, z, yp, ss, \
+                                                  M, N, K, ps, err)                         \
+       : launch_gemm<gemm_tc_kernel<kBDequant, kEpiStoreBf16, false, MT_, NB_>,             \
+                     SmemLayout<MT_, NB_>::bytes>(grid, pdl, stream, ta, tb, q, sc, z, yp, ss, \
+                                                  M, N, K, ps, err))
+  if (mt == 2 && nb == 256) return W4_PREFILL_LAUNCH(2, 256);
+  if (mt == 2) return W4_PREFILL_LAUNCH(2, 128);
+  if (nb == 256) return W4_PREFILL_LAUNCH(1, 256);
+  return W4_PREFILL_LAUNCH(1, 128);
+#undef W4_PREFILL_LAUNCH
 }
 
 cudaError_t launch_sumsq_gemm(const void* a_f16, int M, const void* b_f16, int N, int K,
@@ -551,7 +574,7 @@ cudaError_t launch_sumsq_gemm(const void* a_f16, int M, const void* b_f16, int N
   for (int i = 0; i <= n_seg; ++i) ss.seg_off[i] = seg_off[i];
   dim3 grid((N + BN - 1) / BN, (M + BM - 1) / BM, n_cand);
   ss.tiles = grid.x * grid.y;
-  return launch_gemm<gemm_tc_kernel<kBTma, kEpiSumSquares, false, 1>, SmemLayout<1>::bytes>(
+  return launch_gemm<gemm_tc_kernel<kBTma, kEpiSumSquares, false, 1, BN>, SmemLayout<1, BN>::bytes>(
       grid, false, stream, ta, tb, nullptr, nullptr, nullptr, nullptr, ss, M, N, K, 0, err);
 }
 
