@@ -386,20 +386,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         // Sum of squares per 16-column chunk: thread -> fixed-order shuffle
         // tree over the 32 rows of this warp -> shared -> fixed order over
         // the 4 warps of this column half -> per-segment sums.
-        static_assert(EPI != kEpiSumSquares || (MT == 1 && NB == BN),
-                      "sum of squares uses 128 x 256 tiles");
-        const int m = m0 + 32 * q + lane;
+        // With MT = 2 a thread takes its row of each 128-row half in turn
+        // (fixed order).
+        static_assert(EPI != kEpiSumSquares || NB == BN, "sum of squares uses 256-column tiles");
         for (int c = 0; c < 8; ++c) {
           const int col = 128 * ch + 16 * c;
-          uint32_t r[16];
-          tmem_ld_32x32b_x16(tmem_base + (static_cast<uint32_t>(32 * q) << 16) + col, r);
-          tmem_ld_wait();
           double acc = 0.0;
-          if (m < M) {
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const double v = static_cast<double>(__uint_as_float(r[i]));
-              if (n0 + col + i < N) acc = fma(v, v, acc);
+          for (int mt = 0; mt < MT; ++mt) {
+            const int m = m0 + 128 * mt + 32 * q + lane;
+            uint32_t r[16];
+            tmem_ld_32x32b_x16(tmem_base + (static_cast<uint32_t>(32 * q) << 16) + NB * mt + col,
+                               r);
+            tmem_ld_wait();
+            if (m < M) {
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                const double v = static_cast<double>(__uint_as_float(r[i]));
+                if (n0 + col + i < N) acc = fma(v, v, acc);
+              }
             }
           }
 #pragma unroll
@@ -553,13 +558,18 @@ cudaError_t launch_prefill_gemm(const void* x, int M, const int32_t* qw, const u
 #undef W4_PREFILL_LAUNCH
 }
 
+// Row tiles of the sum-of-squares GEMM: 256 rows (two UMMAs per k-step
+// sharing each B tile) whenever M fills them.
+int sumsq_mt(int M) { return M >= 2 * BM ? 2 : 1; }
+
 cudaError_t launch_sumsq_gemm(const void* a_f16, int M, const void* b_f16, int N, int K,
                               int n_cand, double* partials, int n_seg, const int* seg_off,
                               cudaStream_t stream, unsigned* err) {
   CUtensorMap ta, tb;
   const uint64_t da[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(M)};
   const uint64_t sa[1] = {static_cast<uint64_t>(K) * 2};
-  const uint32_t ba[2] = {BK, BM};
+  const int mt = sumsq_mt(M);
+  const uint32_t ba[2] = {BK, static_cast<uint32_t>(mt * BM)};
   if (encode_tmap(&ta, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, da, sa, ba, a_f16) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
   const uint64_t db[3] = {static_cast<uint64_t>(K), static_cast<uint64_t>(N),
@@ -572,12 +582,18 @@ cudaError_t launch_sumsq_gemm(const void* a_f16, int M, const void* b_f16, int N
   ss.partials = partials;
   ss.n_seg = n_seg;
   for (int i = 0; i <= n_seg; ++i) ss.seg_off[i] = seg_off[i];
-  dim3 grid((N + BN - 1) / BN, (M + BM - 1) / BM, n_cand);
+  dim3 grid((N + BN - 1) / BN, (M + mt * BM - 1) / (mt * BM), n_cand);
   ss.tiles = grid.x * grid.y;
+  if (mt == 2)
+    return launch_gemm<gemm_tc_kernel<kBTma, kEpiSumSquares, false, 2, BN>,
+                       SmemLayout<2, BN>::bytes>(grid, false, stream, ta, tb, nullptr, nullptr,
+                                                 nullptr, nullptr, ss, M, N, K, 0, err);
   return launch_gemm<gemm_tc_kernel<kBTma, kEpiSumSquares, false, 1, BN>, SmemLayout<1, BN>::bytes>(
       grid, false, stream, ta, tb, nullptr, nullptr, nullptr, nullptr, ss, M, N, K, 0, err);
 }
 
-int sumsq_tiles(int M, int N) { return ((N + BN - 1) / BN) * ((M + BM - 1) / BM); }
+int sumsq_tiles(int M, int N) {
+  return ((N + BN - 1) / BN) * ((M + sumsq_mt(M) * BM - 1) / (sumsq_mt(M) * BM));
+}
 
 }  // namespace w4
