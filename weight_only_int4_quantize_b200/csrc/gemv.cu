@@ -488,10 +488,46 @@ cudaError_t launch_gemv_batch_t(GemvBatch& b, bool pdl, bool static_w, cudaStrea
     g_min = b.K[i] / 128 < g_min ? b.K[i] / 128 : g_min;
     g_max = b.K[i] / 128 > g_max ? b.K[i] / 128 : g_max;
   }
+  // Resident CTAs per SM for a given layout (its shared memory depends on the
+  // slice), cached per device and layout size.
+  static uint32_t occ_total[64][4] = {};
+  static int occ_blocks[64][4] = {};
+  auto resident = [&](uint32_t total, int& out) -> cudaError_t {
+    if (dev < 64)
+      for (int j = 0; j < 4; ++j)
+        if (occ_total[dev][j] == total) {
+          out = occ_blocks[dev][j] * num_sms;
+          return cudaSuccess;
+        }
+    int nb = 0;
+    const cudaError_t r = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, kern, kThreads, total);
+    if (r != cudaSuccess) return r;
+    if (dev < 64) {
+      int j = 0;
+      while (j < 3 && occ_total[dev][j] != 0) ++j;
+      occ_total[dev][j] = total;
+      occ_blocks[dev][j] = nb;
+    }
+    out = nb * num_sms;
+    return cudaSuccess;
+  };
+  // The largest split (1..8) whose grid still fits in one wave, with every
+  // rank keeping at least two groups and a slice within the scale table.
   int ks = 1;
-  while (ks < 8 && row_blocks * ks * 2 <= capacity && g_min / (ks * 2) >= 2) ks *= 2;
-  while ((g_max + ks - 1) / ks > kMaxSliceGroups && ks < 8) ks *= 2;
+  for (int cand = 8; cand > 1; --cand) {
+    const int gs = (g_max + cand - 1) / cand;
+    if (g_min / cand < 2 || gs > kMaxSliceGroups) continue;
+    int cap = 0;
+    e = resident(gemv_layout(NT, gs).total, cap);
+    if (e != cudaSuccess) return e;
+    if (row_blocks * cand <= cap) {
+      ks = cand;
+      break;
+    }
+  }
+  while ((g_max + ks - 1) / ks > kMaxSliceGroups && ks < 8) ++ks;
   if ((g_max + ks - 1) / ks > kMaxSliceGroups) return cudaErrorInvalidValue;
+  (void)capacity;
   b.ksplit = ks;
   b.gs_max = (g_max + ks - 1) / ks;
   const GemvLayout L = gemv_layout(NT, b.gs_max);
