@@ -10,8 +10,8 @@ weights N(0, 0.02), int4 asymmetric g128.  A step runs
       zeros) through the batched entry point (64 tensors per launch), then
   (2) the decode W4A16 GEMV through all 196 linears at M = 1, 4 and 8 tokens
       (bf16 x ~ N(0, 1)).  Every linear has its own input, so the 196 are
-      independent problems: the batched entry point runs 32 per launch, with
-      programmatic dependent launch.
+      independent problems: the batched entry point decodes up to 256 of them
+      in one persistent launch, with programmatic dependent launch.
 value = algorithmic bytes of the step / step time (GB/s): 2.53125 B/weight
 for quantize, 0.53125 B/weight + 2MK + 2MN bytes per decode linear.  The step
 is one CUDA graph; its working set (2.8 GB bf16 weights, 0.75 GB packed) is
@@ -50,8 +50,8 @@ FALLBACK_BF16_TFLOPS = 1590.0
 # summaries under profiles/ give the commands), with the digest of the kernel
 # source the capture was taken on.  A changed source reports traffic null.
 TRAFFIC_CAPTURES = {
-    # decode_batch --m 1 --blocks 4: 111.07 MB over 106.92 MB algorithmic
-    "gemv_w4a16": {"source": "gemv.cu", "digest": "fb9e87eb5d8c1cfd", "ratio": 111.07 / 106.92},
+    # (no capture of the streaming decode kernel yet: traffic is reported null)
+    "gemv_w4a16": {"source": "gemv_stream.cu", "digest": None, "ratio": None},
     # quantize 17408 x 5120: 202.90 MB over 225.67 MB (part of the written codes
     # is still in the write-back L2 when the kernel ends)
     "quantize_pack": {"source": "quantize.cu", "digest": "fe920be4faac0b8e", "ratio": 202.90 / 225.67},
@@ -255,12 +255,10 @@ class Model:
         self.d_items = {m: w4.linear_items([(self.x[(m, k)], qw, sc, zr, self.y[m][j])
                                             for j, (k, n, w, qw, sc, zr) in enumerate(self.lin)])
                         for m in DECODE_M}
-        # w4a16_linear_batched launches one GEMV per 32 linears of equal K.
-        per_k = {}
-        for (k, *_r) in self.lin:
-            per_k[k] = per_k.get(k, 0) + 1
+        # w4a16_linear_batched (M <= 8) runs up to STREAM_BATCH linears per
+        # persistent launch.
         self.launches = {"quantize": -(-len(self.lin) // 64),
-                         "gemv": len(DECODE_M) * sum(-(-c // 32) for c in per_k.values())}
+                         "gemv": len(DECODE_M) * -(-len(self.lin) // w4.STREAM_BATCH)}
 
     def quantize_all(self):
         """All 196 weights through w4_quantize_pack_batched (64 per launch)."""
@@ -270,7 +268,7 @@ class Model:
 
     def decode_all(self, m, flags):
         """All 196 linears (independent inputs) through w4a16_linear_batched
-        (32 per launch)."""
+        (one persistent launch)."""
         import weight_only_int4_quantize_b200 as w4
         w4.w4a16_linear_batched(self.d_items[m], m, flags,
                                 stream=self.torch.cuda.current_stream(self.dev).cuda_stream)
@@ -525,7 +523,7 @@ def main():
     bytes_per_launch = (qb if dom[0] == "quantize_pack" else db) / dom[2]
     cap = TRAFFIC_CAPTURES.get(dom[0])
     traffic = None
-    if cap and source_digest(cap["source"]) == cap["digest"]:
+    if cap and cap["digest"] and source_digest(cap["source"]) == cap["digest"]:
         traffic = cap["ratio"] * bytes_per_launch
     roofline = {"kernel": dom[0], "bound": "hbm", "achieved": dom[1], "peak": hbm, "unit": "GB/s",
                 "frac": dom[1] / hbm, "peak_kind": peak_kind, "traffic": traffic,
@@ -544,7 +542,7 @@ def main():
                    "decode_M": list(DECODE_M), "parallelism": f"replicas x{world}",
                    "l2": "working set 3.6 GB >> 126 MB L2 (no flush needed)",
                    "graph": "one CUDA graph per phase; the 196 linears are independent "
-                            "problems, batched: 4 quantize launches + 7 decode launches per M",
+                            "problems, batched: 4 quantize launches + 1 decode launch per M",
                    "l2_note": "inputs (3.6 GB) exceed L2; no flush"},
         "phases": {"quantize_ms": q_ms, "quantize_gbs": qb / (q_ms * 1e-3) / 1e9,
                    **{f"decode_M{m}_ms": d_ms[m] for m in DECODE_M},

@@ -147,10 +147,15 @@ w4_status w4_quantize_pack_batched(const w4_quant_item* items, int count, int gr
  *           rounded once to bf16).
  * flags     bitwise OR of W4_LINEAR_* below (0 for defaults).
  *
- * M <= 16 (and K <= 81920) runs the decode GEMV (tensor-core mma over
+ * M <= 16 (and K <= 81920) runs a decode GEMV (tensor-core mma over
  * register-dequantized weight fragments, HBM-bound); larger M runs the
  * prefill GEMM (tcgen05 with TMEM accumulators, weight tiles dequantized into
- * shared memory).
+ * shared memory).  There are two decode kernels: a persistent streaming
+ * kernel (M <= 8; every warp streams 64-row units through its own ring) for
+ * launches with at least two of its 4-warp bundles per SM, and a per-CTA
+ * tensor-map kernel (K split over a thread-block cluster) for smaller
+ * launches and 9 <= M <= 64.  W4_LINEAR_DECODE_STREAM / _TILED override the
+ * choice; both meet the same error bound.
  */
 #define W4_LINEAR_FORCE_GEMV 0x1u  /* decode kernel at any M <= 64 (K <= 81920) */
 #define W4_LINEAR_FORCE_GEMM 0x2u  /* prefill kernel at any M */
@@ -163,6 +168,10 @@ w4_status w4_quantize_pack_batched(const w4_quant_item* items, int count, int gr
                                       written by preceding work still in
                                       flight, so the kernel may start streaming
                                       them before the dependency wait */
+#define W4_LINEAR_DECODE_STREAM 0x10u /* decode through the persistent
+                                      streaming kernel (M <= 8 only) */
+#define W4_LINEAR_DECODE_TILED 0x20u  /* decode through the per-CTA
+                                      tensor-map kernel (M <= 64) */
 w4_status w4a16_linear(const void* x_bf16, int64_t M, const int32_t* qweight,
                        const uint16_t* scales_f16, const uint16_t* zeros_f16,
                        int64_t N, int64_t K, int group, void* y_bf16,
@@ -171,10 +180,12 @@ w4_status w4a16_linear(const void* x_bf16, int64_t M, const int32_t* qweight,
 /*
  * w4a16_linear_batched -- w4a16_linear over `count` independent linears that
  * share the token count M and the symmetry (all zeros NULL or none), for
- * example every projection of a decode step whose inputs are ready.  M <= 64
- * (K <= 81920) runs the decode kernel with up to 32 linears per launch;
- * larger M runs one prefill GEMM per linear.  flags: W4_LINEAR_PDL and
- * W4_LINEAR_STATIC_WEIGHTS only.  items: host array.  Each result meets the
+ * example every projection of a decode step whose inputs are ready.  M <= 8
+ * runs up to 256 linears per persistent streaming launch (or, for a launch
+ * too small to fill the GPU, the tensor-map kernel); 9 <= M <= 64 (K <=
+ * 81920) runs the tensor-map kernel with up to 32 linears per launch; larger
+ * M runs one prefill GEMM per linear.  flags: W4_LINEAR_PDL,
+ * W4_LINEAR_STATIC_WEIGHTS and the W4_LINEAR_DECODE_* choice only.  items: host array.  Each result meets the
  * same error bound as a per-linear call (the K split of a batch, and so the
  * binary32 summation order, may differ from a single call's).
  */

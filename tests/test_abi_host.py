@@ -69,6 +69,21 @@ def test_linear_validation(L):
     assert f(A, 1, A, A, None, 8, 128, 32, B, 0, None) == 4
     assert f(A, 100, A, A, None, 8, 128, 128, B, 0x1, None) == 4        # GEMV beyond 64 rows
     assert f(A, 1, A, A, None, 8, 128, 128, B + 8, 0, None) == 3
+    assert f(A, 1, A, A, None, 8, 128, 128, B, 0x30, None) == 1        # both decode kernels
+    assert f(A, 1, A, A, None, 8, 128, 128, B, 0x12, None) == 1        # stream + prefill
+    assert f(A, 9, A, A, None, 8, 128, 128, B, 0x10, None) == 4        # stream beyond 8 rows
+    assert f(A, 65, A, A, None, 8, 128, 128, B, 0x20, None) == 4       # tiled beyond 64 rows
+
+
+def test_linear_batched_validation(L):
+    import weight_only_int4_quantize_b200 as w4
+    f = L.w4a16_linear_batched
+    it = (w4.LinearItem * 1)(w4.LinearItem(A, A, A, None, 8, 128, B))
+    assert f(None, 1, 1, 128, 0, None) == 1
+    assert f(it, 1, 1, 128, 0x1, None) == 1                            # not a batched flag
+    assert f(it, 1, 1, 128, 0x30, None) == 1                           # both decode kernels
+    assert f(it, 1, 9, 128, 0x10, None) == 4                           # stream beyond 8 rows
+    assert f(it, 1, 1, 64, 0, None) == 4                               # group != 128
 
 
 def test_awq_validation(L):

@@ -157,15 +157,45 @@ def linear_case(m, n, k, sym, seed, flags=0, std=0.02, n_out=0, out_scale=1.0, r
     return max_rel_err(y[torch.as_tensor(rows, device=DEV)], y_ref)
 
 
+DECODE_KERNELS = {"auto": 0, "stream": w4.LINEAR_DECODE_STREAM, "tiled": w4.LINEAR_DECODE_TILED}
+
+
+@pytest.mark.parametrize("kernel", ["auto", "stream", "tiled"])
 @pytest.mark.parametrize("m", [1, 2, 3, 5, 8, 9, 15, 16])
 @pytest.mark.parametrize("sym", [False, True])
-def test_gemv_parity_ragged(m, sym):
-    assert linear_case(m, 1000, 1024, sym, seed=100 + m) <= Y_RTOL
+def test_gemv_parity_ragged(m, sym, kernel):
+    if kernel == "stream" and m > 8:
+        pytest.skip("the streaming decode kernel takes at most 8 tokens")
+    assert linear_case(m, 1000, 1024, sym, seed=100 + m, flags=DECODE_KERNELS[kernel]) <= Y_RTOL
 
 
 @pytest.mark.parametrize("m", [1, 16])
 def test_gemv_single_linear_2048_outliers(m):
     assert linear_case(m, 2048, 2048, False, seed=0, n_out=8, out_scale=20.0) <= Y_RTOL
+
+
+@pytest.mark.parametrize("m,n,k", [(1, 7, 128), (8, 33, 128), (3, 100, 256), (4, 100, 1024),
+                                   (2, 16, 2048), (6, 1, 384), (7, 4100, 640)])
+@pytest.mark.parametrize("sym", [False, True])
+def test_gemv_stream_small_and_split(m, n, k, sym):
+    """Decode shapes that exercise the streaming kernel's edges: one group
+    (K = 128), ragged 64-row units and 16-row tiles, N = 1, and K split over
+    2 or 4 warps of a row block (few row blocks), plus one shape with more
+    bundles than the grid has CTAs."""
+    err = linear_case(m, n, k, sym, seed=1000 + m * 7 + n + k, flags=w4.LINEAR_DECODE_STREAM)
+    assert err <= Y_RTOL
+
+
+def test_gemv_stream_deterministic():
+    """Split-K partial sums are reduced in a fixed order: repeated calls give
+    identical bits."""
+    w = synth.normal_weight(96, 2048, 0.02, seed=61)
+    x = synth.normal_activations(5, 2048, seed=62).to(DEV)
+    qw, sc, zr = w4.quantize_pack(w.to(DEV), False)
+    y0 = w4.w4a16_linear(x, qw, sc, zr, flags=w4.LINEAR_DECODE_STREAM)
+    y1 = w4.w4a16_linear(x, qw, sc, zr, flags=w4.LINEAR_DECODE_STREAM)
+    torch.cuda.synchronize()
+    assert torch.equal(y0.view(torch.int16), y1.view(torch.int16))
 
 
 @pytest.mark.parametrize("m", [17, 40, 64])
@@ -193,6 +223,14 @@ def test_linear_27b_shapes(k, n, m):
     rows = None if m <= 512 else np.sort(np.random.default_rng(m + n).choice(m, 128, replace=False))
     err = linear_case(m, n, k, True, seed=500 + n, std=0.015, n_out=k // 100, out_scale=10.0,
                       rows=rows)
+    assert err <= Y_RTOL
+
+
+@pytest.mark.parametrize("k,n", [(5120, 17408), (17408, 5120)])
+@pytest.mark.parametrize("m", [1, 8])
+def test_linear_27b_shapes_streaming_kernel(k, n, m):
+    err = linear_case(m, n, k, True, seed=500 + n, std=0.015, n_out=k // 100, out_scale=10.0,
+                      flags=w4.LINEAR_DECODE_STREAM)
     assert err <= Y_RTOL
 
 
@@ -297,9 +335,37 @@ def test_quantize_batched_mixed_tensors(sym):
         assert_quant_equal((qw, sc, zr), ref, sym)
 
 
-@pytest.mark.parametrize("m", [1, 5, 16, 40])
+def test_linear_batched_more_than_one_launch():
+    """More linears than one streaming launch takes (STREAM_BATCH), mixed K
+    and ragged N, at 3 tokens: every result meets the bound."""
+    rng = np.random.default_rng(5)
+    count = w4.STREAM_BATCH + 44
+    items, refs = [], []
+    for i in range(count):
+        k = int(rng.choice([128, 256, 384, 1024]))
+        n = int(rng.integers(1, 70))
+        w = synth.normal_weight(n, k, 0.02, seed=3000 + i)
+        x = synth.normal_activations(3, k, seed=6000 + i)
+        qw, sc, zr = w4.quantize_pack(w.to(DEV), False)
+        y = torch.empty(3, n, dtype=torch.bfloat16, device=DEV)
+        items.append((x.to(DEV), qw, sc, zr, y))
+        oc, os_, oz = O.quantize_rtn(synth.bits(w), False)
+        refs.append(O.linear(synth.bits(x), O.dequantize(oc, os_, oz)))
+    for kernel in ("auto", "stream"):
+        for it in items:
+            it[4].zero_()
+        w4.w4a16_linear_batched(items, 3, DECODE_KERNELS[kernel])
+        torch.cuda.synchronize()
+        worst = max(max_rel_err(it[4], ref) for it, ref in zip(items, refs))
+        assert worst <= Y_RTOL, kernel
+
+
+@pytest.mark.parametrize("kernel", ["auto", "stream", "tiled"])
+@pytest.mark.parametrize("m", [1, 5, 8, 16, 40])
 @pytest.mark.parametrize("sym", [False, True])
-def test_linear_batched_qwen_block(m, sym):
+def test_linear_batched_qwen_block(m, sym, kernel):
+    if kernel == "stream" and m > 8:
+        pytest.skip("the streaming decode kernel takes at most 8 tokens")
     shapes = [(n, k) for _, k, n in synth.QWEN3_1P7B_BLOCK] + [(72, 640)]
     items, refs = [], []
     for i, (n, k) in enumerate(shapes):
@@ -310,7 +376,7 @@ def test_linear_batched_qwen_block(m, sym):
         items.append((x.to(DEV), qw, sc, zr, y))
         oc, os_, oz = O.quantize_rtn(synth.bits(w), sym)
         refs.append(O.linear(synth.bits(x), O.dequantize(oc, os_, oz)))
-    w4.w4a16_linear_batched(items, m)
+    w4.w4a16_linear_batched(items, m, DECODE_KERNELS[kernel])
     torch.cuda.synchronize()
     for (x, qw, sc, zr, y), ref in zip(items, refs):
         assert max_rel_err(y, ref) <= Y_RTOL

@@ -19,6 +19,7 @@ __all__ = [
     "w4a16_linear_batched", "awq_scales", "awq_score_grid", "awq_score_grid_static_scratch",
     "awq_workspace_bytes", "device_error", "selftest_bounded_wait",
     "LINEAR_FORCE_GEMV", "LINEAR_FORCE_GEMM", "LINEAR_PDL", "LINEAR_STATIC_WEIGHTS",
+    "LINEAR_DECODE_STREAM", "LINEAR_DECODE_TILED", "STREAM_BATCH",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libw4.so")
@@ -27,6 +28,11 @@ LINEAR_FORCE_GEMV = 0x1
 LINEAR_FORCE_GEMM = 0x2
 LINEAR_PDL = 0x4
 LINEAR_STATIC_WEIGHTS = 0x8
+LINEAR_DECODE_STREAM = 0x10   # decode through the persistent streaming kernel (M <= 8)
+LINEAR_DECODE_TILED = 0x20    # decode through the per-CTA tensor-map kernel (M <= 64)
+# Linears per launch of w4a16_linear_batched at M <= 8 (one persistent
+# streaming launch per this many).
+STREAM_BATCH = 256
 
 _STATUS = {
     0: "W4_OK", 1: "W4_ERR_INVALID_ARG", 2: "W4_ERR_SHAPE", 3: "W4_ERR_ALIGNMENT",

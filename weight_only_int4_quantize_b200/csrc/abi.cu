@@ -5,6 +5,8 @@
 #include <cstdint>
 #include <cstdio>
 #include <cstring>
+#include <algorithm>
+#include <vector>
 
 #include "w4.h"
 #include "w4_common.cuh"
@@ -192,23 +194,34 @@ static w4_status check_linear_item(const void* x_bf16, int64_t M, const int32_t*
 
 static constexpr int64_t kGemvMaxK = 8 * 80 * 128;  // decode kernel: K slice <= 80 groups x 8
 
+// The persistent streaming decode kernel is chosen for launches that deal
+// at least this many 4-warp bundles per SM; smaller launches (a single
+// linear, a few short ones) run the per-CTA tensor-map kernel, whose K split
+// over a thread-block cluster fills the GPU with few rows.
+static constexpr int kStreamMinBundlesPerSm = 2;
+
+static constexpr unsigned kDecodeChoice = W4_LINEAR_DECODE_STREAM | W4_LINEAR_DECODE_TILED;
+
 w4_status w4a16_linear(const void* x_bf16, int64_t M, const int32_t* qweight,
                        const uint16_t* scales_f16, const uint16_t* zeros_f16, int64_t N,
                        int64_t K, int group, void* y_bf16, unsigned flags, void* stream) {
   if (!x_bf16 || !qweight || !scales_f16 || !y_bf16) return W4_ERR_INVALID_ARG;
   const unsigned known = W4_LINEAR_FORCE_GEMV | W4_LINEAR_FORCE_GEMM | W4_LINEAR_PDL |
-                         W4_LINEAR_STATIC_WEIGHTS;
+                         W4_LINEAR_STATIC_WEIGHTS | kDecodeChoice;
   if (flags & ~known) return W4_ERR_INVALID_ARG;
   if ((flags & W4_LINEAR_FORCE_GEMV) && (flags & W4_LINEAR_FORCE_GEMM)) return W4_ERR_INVALID_ARG;
+  if ((flags & kDecodeChoice) == kDecodeChoice) return W4_ERR_INVALID_ARG;
+  if ((flags & kDecodeChoice) && (flags & W4_LINEAR_FORCE_GEMM)) return W4_ERR_INVALID_ARG;
   if (group != 128) return W4_ERR_UNSUPPORTED;
   w4_status st = check_linear_item(x_bf16, M, qweight, scales_f16, zeros_f16, N, K, y_bf16);
   if (st != W4_OK) return st;
-  // The decode kernel keeps a CTA's K slice (at most 8 x 80 groups) in a
+  // The decode kernels keep a CTA's K slice (at most 8 x 80 groups) in a
   // shared scale table; longer K goes to the prefill kernel.
   const bool gemv_ok = K <= kGemvMaxK;
-  const bool gemv = (flags & W4_LINEAR_FORCE_GEMV) ||
+  const bool gemv = (flags & (W4_LINEAR_FORCE_GEMV | kDecodeChoice)) ||
                     (M <= 16 && gemv_ok && !(flags & W4_LINEAR_FORCE_GEMM));
   if (gemv && (M > 64 || !gemv_ok)) return W4_ERR_UNSUPPORTED;
+  if ((flags & W4_LINEAR_DECODE_STREAM) && M > 8) return W4_ERR_UNSUPPORTED;
   if (!gemv && (M + 127) / 128 > 65535) return W4_ERR_UNSUPPORTED;
   int sms = 0;
   unsigned* err = nullptr;
@@ -217,6 +230,21 @@ w4_status w4a16_linear(const void* x_bf16, int64_t M, const int32_t* qweight,
   const bool pdl = (flags & W4_LINEAR_PDL) != 0;
   const bool stat = (flags & W4_LINEAR_STATIC_WEIGHTS) != 0;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (gemv && M <= 8 && !(flags & W4_LINEAR_DECODE_TILED)) {
+    StreamBatch b;
+    b.count = 0;
+    b.unit_start[0] = 0;
+    b.M = static_cast<int>(M);
+    stream_batch_add(b, x_bf16, qweight, scales_f16, zeros_f16, static_cast<int>(N),
+                     static_cast<int>(K), y_bf16);
+    int bundles = 0;
+    st = cuda_status(plan_gemv_stream(b, zeros_f16 == nullptr, sms, &bundles),
+                     "decode GEMV plan");
+    if (st != W4_OK) return st;
+    if ((flags & W4_LINEAR_DECODE_STREAM) || bundles >= kStreamMinBundlesPerSm * sms)
+      return cuda_status(launch_gemv_stream(b, zeros_f16 == nullptr, pdl, stat, s, sms),
+                         "decode GEMV launch");
+  }
   if (gemv)
     return cuda_status(launch_gemv(x_bf16, static_cast<int>(M), qweight, scales_f16, zeros_f16,
                                    static_cast<int>(N), static_cast<int>(K), y_bf16, pdl, stat, s,
@@ -228,12 +256,60 @@ w4_status w4a16_linear(const void* x_bf16, int64_t M, const int32_t* qweight,
                      "prefill tcgen05 GEMM launch");
 }
 
+// Decodes items idx[0..n) through the per-CTA tensor-map kernel.  Launches
+// group the linears by K, largest K first: a launch's shared memory ring is
+// sized by its longest K slice, so launches of one K size their CTAs exactly
+// (short K fits more CTAs per SM), and no launch ends with a trail of long
+// CTAs.  Results do not depend on the grouping.
+static w4_status decode_tiled(const w4_linear_item* items, const int* idx, int n, int64_t M,
+                              bool sym, bool pdl, bool stat, cudaStream_t s, int sms,
+                              unsigned* err) {
+  for (int64_t m0 = 0; m0 < M; m0 += 16) {
+    const int mc = static_cast<int>(M - m0 < 16 ? M - m0 : 16);
+    int64_t k_prev = INT64_MAX;
+    for (;;) {
+      int64_t kv = 0;  // the largest K below k_prev
+      for (int j = 0; j < n; ++j)
+        if (items[idx[j]].K < k_prev && items[idx[j]].K > kv) kv = items[idx[j]].K;
+      if (kv == 0) break;
+      k_prev = kv;
+      GemvBatch b;
+      b.count = 0;
+      b.cta_start[0] = 0;
+      b.M = mc;
+      for (int j = 0; j <= n; ++j) {
+        if (j < n && items[idx[j]].K == kv) {
+          const w4_linear_item& it = items[idx[j]];
+          const void* xc = static_cast<const uint16_t*>(it.x_bf16) + m0 * it.K;
+          void* yc = static_cast<uint16_t*>(it.y_bf16) + m0 * it.N;
+          w4_status st = cuda_status(gemv_batch_add(b, xc, it.qweight, it.scales_f16,
+                                                    it.zeros_f16, static_cast<int>(it.N),
+                                                    static_cast<int>(it.K), yc),
+                                     "tensor map");
+          if (st != W4_OK) return st;
+        }
+        if (b.count == kGemvBatch || (j == n && b.count > 0)) {
+          w4_status st = cuda_status(launch_gemv_batch(b, sym, pdl, stat, s, sms, err),
+                                     "batched decode GEMV launch");
+          if (st != W4_OK) return st;
+          b.count = 0;
+          b.cta_start[0] = 0;
+        }
+      }
+    }
+  }
+  return W4_OK;
+}
+
 w4_status w4a16_linear_batched(const w4_linear_item* items, int count, int64_t M, int group,
                                unsigned flags, void* stream) {
   if (!items || count < 1) return W4_ERR_INVALID_ARG;
-  const unsigned known = W4_LINEAR_PDL | W4_LINEAR_STATIC_WEIGHTS;
+  const unsigned known = W4_LINEAR_PDL | W4_LINEAR_STATIC_WEIGHTS | kDecodeChoice;
   if (flags & ~known) return W4_ERR_INVALID_ARG;
+  if ((flags & kDecodeChoice) == kDecodeChoice) return W4_ERR_INVALID_ARG;
   if (group != 128) return W4_ERR_UNSUPPORTED;
+  if ((flags & W4_LINEAR_DECODE_STREAM) && M > 8) return W4_ERR_UNSUPPORTED;
+  if ((flags & W4_LINEAR_DECODE_TILED) && M > 64) return W4_ERR_UNSUPPORTED;
   const bool sym = items[0].zeros_f16 == nullptr;
   for (int i = 0; i < count; ++i) {
     const w4_linear_item& it = items[i];
@@ -261,42 +337,39 @@ w4_status w4a16_linear_batched(const w4_linear_item* items, int count, int64_t M
     }
     return W4_OK;
   }
-  // Launches group the linears by K, largest K first: a launch's shared
-  // memory ring is sized by its longest K slice, so launches of one K size
-  // their CTAs exactly (short K fits more CTAs per SM), and no launch ends
-  // with a trail of long CTAs.  Results do not depend on the grouping.
-  for (int64_t m0 = 0; m0 < M; m0 += 16) {
-    const int mc = static_cast<int>(M - m0 < 16 ? M - m0 : 16);
-    int64_t k_prev = INT64_MAX;
-    for (;;) {
-      int64_t kv = 0;  // the largest K below k_prev
-      for (int i = 0; i < count; ++i)
-        if (items[i].K < k_prev && items[i].K > kv) kv = items[i].K;
-      if (kv == 0) break;
-      k_prev = kv;
-      GemvBatch b;
-      b.count = 0;
-      b.cta_start[0] = 0;
-      b.M = mc;
-      for (int i = 0; i <= count; ++i) {
-        if (i < count && items[i].K == kv) {
-          const w4_linear_item& it = items[i];
-          const void* xc = static_cast<const uint16_t*>(it.x_bf16) + m0 * it.K;
-          void* yc = static_cast<uint16_t*>(it.y_bf16) + m0 * it.N;
-          st = cuda_status(gemv_batch_add(b, xc, it.qweight, it.scales_f16, it.zeros_f16,
-                                          static_cast<int>(it.N), static_cast<int>(it.K), yc),
-                           "tensor map");
-          if (st != W4_OK) return st;
-        }
-        if (b.count == kGemvBatch || (i == count && b.count > 0)) {
-          st = cuda_status(launch_gemv_batch(b, sym, pdl, stat, s, sms, err),
-                           "batched decode GEMV launch");
-          if (st != W4_OK) return st;
-          b.count = 0;
-          b.cta_start[0] = 0;
-        }
-      }
+  std::vector<int> order(count);
+  for (int i = 0; i < count; ++i) order[i] = i;
+  if (M > 8 || (flags & W4_LINEAR_DECODE_TILED))
+    return decode_tiled(items, order.data(), count, M, sym, pdl, stat, s, sms, err);
+  // M <= 8: persistent streaming launches of up to kStreamBatch linears,
+  // longest K first (the launch deals its units in that order, so the long
+  // ones are spread first and the short ones even out the warps' totals);
+  // a launch too small to fill the GPU goes to the tensor-map kernel.
+  std::stable_sort(order.begin(), order.end(),
+                   [&](int a, int c) { return items[a].K > items[c].K; });
+  for (int i0 = 0; i0 < count;) {
+    StreamBatch b;
+    b.count = 0;
+    b.unit_start[0] = 0;
+    b.M = static_cast<int>(M);
+    int j = i0;
+    // (a launch's bundles are counted in int: at most 2^30 of them)
+    for (; j < count && j < i0 + kStreamBatch; ++j) {
+      const w4_linear_item& it = items[order[j]];
+      if (b.count > 0 && b.unit_start[b.count] + (it.N + 63) / 64 > (int64_t{1} << 30)) break;
+      stream_batch_add(b, it.x_bf16, it.qweight, it.scales_f16, it.zeros_f16,
+                       static_cast<int>(it.N), static_cast<int>(it.K), it.y_bf16);
     }
+    int bundles = 0;
+    st = cuda_status(plan_gemv_stream(b, sym, sms, &bundles), "decode GEMV plan");
+    if (st != W4_OK) return st;
+    if ((flags & W4_LINEAR_DECODE_STREAM) || bundles >= kStreamMinBundlesPerSm * sms)
+      st = cuda_status(launch_gemv_stream(b, sym, pdl, stat, s, sms),
+                       "batched decode GEMV launch");
+    else
+      st = decode_tiled(items, order.data() + i0, j - i0, M, sym, pdl, stat, s, sms, err);
+    if (st != W4_OK) return st;
+    i0 = j;
   }
   return W4_OK;
 }

@@ -62,6 +62,30 @@ cudaError_t launch_gemv(const void* x, int M, const int32_t* qw, const uint16_t*
                         const uint16_t* z, int N, int K, void* y, bool pdl, bool static_w,
                         cudaStream_t stream, int num_sms, unsigned* err);
 
+// Up to kStreamBatch independent linears with the same token count (<= 8)
+// decoded by one persistent streaming launch (kernel parameter).
+constexpr int kStreamBatch = 256;
+struct StreamBatch {
+  const __nv_bfloat16* x[kStreamBatch];  // bf16 [M, K]
+  const uint8_t* qw[kStreamBatch];       // packed codes, [N, K/2] bytes
+  const uint16_t* scales[kStreamBatch];  // fp16 [N, K/128]
+  const uint16_t* zeros[kStreamBatch];   // fp16 [N, K/128]; NULL: symmetric
+  __nv_bfloat16* y[kStreamBatch];        // bf16 [M, N]
+  int N[kStreamBatch];
+  int K[kStreamBatch];
+  int ks[kStreamBatch];                  // K parts of each linear (1, 2 or 4)
+  int unit_start[kStreamBatch + 1];      // prefix sums of bundles (4 warp units each)
+  int count, M;
+};
+void stream_batch_add(StreamBatch& b, const void* x, const int32_t* qw, const uint16_t* sc,
+                      const uint16_t* z, int N, int K, void* y);
+// Chooses the K split of every linear for the launch's grid; *bundles is the
+// number of 4-warp bundles the launch would deal (launch_gemv_stream plans
+// the same way, so planning first does not change the launch).
+cudaError_t plan_gemv_stream(StreamBatch& b, bool symmetric, int num_sms, int* bundles);
+cudaError_t launch_gemv_stream(StreamBatch& b, bool symmetric, bool pdl, bool static_w,
+                               cudaStream_t stream, int num_sms);
+
 cudaError_t launch_prefill_gemm(const void* x, int M, const int32_t* qw, const uint16_t* sc,
                                 const uint16_t* z, int N, int K, void* y, bool pdl,
                                 bool static_w, cudaStream_t stream, unsigned* err);
