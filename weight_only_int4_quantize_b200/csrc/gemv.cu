@@ -1,6 +1,9 @@
-// Decode W4A16 GEMV: y[M, N] = x[M, K] . dequant(Wq)^T for M <= 16 (up to 64
-// with W4_LINEAR_FORCE_GEMV, in chunks of 16 tokens).  HBM-bound on the
-// packed weight stream (0.53125 B/weight asymmetric, 0.515625 symmetric).
+// Decode W4A16 GEMV, tensor-map kernel: y[M, N] = x[M, K] . dequant(Wq)^T for
+// M <= 16 (up to 64 with W4_LINEAR_FORCE_GEMV, in chunks of 16 tokens).
+// HBM-bound on the packed weight stream (0.53125 B/weight asymmetric,
+// 0.515625 symmetric).  It serves 9 <= M <= 64 and decode launches too small
+// for the persistent streaming kernel (gemv_stream.cu), which it beats there
+// because its cluster K split fills the GPU with few rows.
 //
 // A CTA owns 64 weight rows and one K slice (the K dimension is split over
 // the CTAs of a thread-block cluster).  One producer thread streams the
