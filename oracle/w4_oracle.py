@@ -25,6 +25,9 @@ Sources (model-card pages; cited by page title and section):
       (int4, group size 128, symmetric, weight-only, activations 16-bit).
   [awq-ppl] "AWQ INT4-g128 WikiText-2 perplexity delta vs fp16, Llama-2 7B",
       'Methodology' (group size 128; grid size 20 for the alpha search).
+  [rebuttal-cmp] the same "ghostchoir/rebuttal_w4g128_awq_w2" card, the
+      'Comparability caveat' under the perplexity table (the d=0 arm uses
+      stock AWQ's per-output-channel clipping search).
 
 Readings where the pages are silent (each is pinned by a test in
 tests/test_oracle_pins.py; the exact list with reasons is in the repository's
@@ -40,7 +43,11 @@ design notes):
     even;
   * the AWQ scale multiplies before quantization (v = w * s in binary32) and
     the shrink ratio r scales the group's range in that s-domain;
-  * s_j = float32(pow(max(mean_m |x_mj|, 1e-8), alpha)), mean in binary64.
+  * s_j = float32(pow(max(mean_m |x_mj|, 1e-8), alpha)), mean in binary64;
+  * stock per-output-channel clipping: every output row takes its own ratio
+    from the same shrink grid, the one with the least output error of that
+    row, ||x E_n^T||^2 (the linear's output error is a sum over rows, so the
+    per-row choices minimise it jointly); ties go to the lowest grid index.
 """
 from __future__ import annotations
 
@@ -151,7 +158,9 @@ def quantize_rtn(w_bits: np.ndarray, symmetric: bool, awq_s: np.ndarray | None =
     assert k % group == 0
     v = w if awq_s is None else w * np.asarray(awq_s, dtype=np.float32)[None, :]
     vg = v.reshape(n, k // group, group)
-    r = np.float32(shrink)
+    # One ratio per linear, or one per output row (a length-N array).
+    r = (np.asarray(shrink, dtype=np.float32).reshape(n, 1) if np.ndim(shrink) == 1
+         else np.float32(shrink))
     floor = np.float32(1e-5)
     if symmetric:
         a = r * np.max(np.abs(vg), axis=2)
@@ -336,6 +345,34 @@ def relative_gap(values: np.ndarray) -> float:
     if v.size < 2 or v[0] <= 0:
         return float("inf")
     return float((v[1] - v[0]) / v[0])
+
+
+def clip_search_rows(x_bits, w_bits, awq_s, shrinks, symmetric, group=GROUP):
+    """Stock per-output-channel clipping search ([rebuttal-cmp]; contrasted in
+    [rebuttal] 'Clipping granularity' with the one global shrink ratio that a
+    look-ahead loss forces).
+
+    For every shrink r_j of the grid: E_j = W - Q_{r_j}(W diag(s)) diag(1/s)
+    (s = awq_s, or 1 when None) and the error of each output channel n,
+    sse_rows[j, n] = sum_m (x E_j^T)[m, n]^2, in binary64.  Row n takes
+    choice[n] = argmin_j sse_rows[j, n], the lowest j on equal values.
+    Returns (sse_rows [n_shrink, N] float64, choice int64 [N])."""
+    n, k = np.asarray(w_bits).shape
+    s = np.ones(k, dtype=np.float32) if awq_s is None else np.asarray(awq_s, dtype=np.float32)
+    x = bf16_bits_to_f32(x_bits).astype(np.float64)
+    sse = np.empty((len(shrinks), n), dtype=np.float64)
+    for j, r in enumerate(shrinks):
+        y = x @ candidate_error(w_bits, s, r, symmetric, group).T
+        sse[j] = np.sum(y * y, axis=0)
+    return sse, np.argmin(sse, axis=0)
+
+
+def quantize_pack_rows(w_bits, symmetric, awq_s, shrink_rows, group=GROUP):
+    """quantize_pack with one shrink ratio per output row (the per-channel
+    clipping's deployed weight)."""
+    codes, s16, z16 = quantize_rtn(w_bits, symmetric, awq_s,
+                                   np.asarray(shrink_rows, dtype=np.float32), group)
+    return pack_codes(codes), s16, z16
 
 
 # ----------------------------------------------------------------------------

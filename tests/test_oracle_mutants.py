@@ -34,6 +34,13 @@ MUTANTS = [
     ("linear against the untransposed weight", "return x @ np.asarray(w_hat, dtype=np.float64).T",
      "return x @ np.asarray(w_hat, dtype=np.float64).T[::-1, ::-1]"),
     ("range floor dropped", "np.maximum(mx - mn, floor)", "(mx - mn)"),
+    ("per-row error summed over tokens' complement", "sse[j] = np.sum(y * y, axis=0)",
+     "sse[j] = np.sum(y * y, axis=0)[::-1]"),
+    ("per-row choice takes the last minimum", "return sse, np.argmin(sse, axis=0)",
+     "return sse, len(shrinks) - 1 - np.argmin(sse[::-1], axis=0)"),
+    ("per-row ratios applied to the wrong rows",
+     "np.asarray(shrink, dtype=np.float32).reshape(n, 1)",
+     "np.asarray(shrink, dtype=np.float32)[::-1].reshape(n, 1)"),
 ]
 
 
@@ -58,6 +65,10 @@ def _all_pins():
     yield P.test_linear_exact_rational_small, ()
     yield P.test_linear_closed_form_constant_weight, ()
     yield P.test_awq_scale_stat_and_pow_brute_force, ()
+    for sym in (False, True):
+        yield P.test_clip_rows_sse_brute_force_tiny, (sym,)
+        yield P.test_quantize_rows_reduces_to_per_linear_quantize, (sym,)
+    yield P.test_clip_rows_ties_take_the_lowest_index, ()
 
 
 @pytest.mark.parametrize("name,old,new", MUTANTS, ids=[m[0] for m in MUTANTS])

@@ -365,3 +365,88 @@ def test_segments_add_up():
     a, _ = O.awq_score_grid(x, w[:5], al, sh, False)
     b, _ = O.awq_score_grid(x, w[5:], al, sh, False)
     assert np.allclose(sse[0], a[0], rtol=1e-13) and np.allclose(sse[1], b[0], rtol=1e-13)
+
+
+# ------------------------------------------- per-output-channel clipping ----
+
+def _row_sse_exact(x_bits, w_bits, s, shrink, sym):
+    """Exact rational output error of every row at one shrink ratio."""
+    codes, s16, z16 = O.quantize_rtn(w_bits, sym, s, shrink)
+    what = O.dequantize(codes, s16, z16)
+    xf = O.bf16_bits_to_f32(x_bits)
+    wf = O.bf16_bits_to_f32(w_bits)
+    m_, k_ = xf.shape
+    out = []
+    for n in range(wf.shape[0]):
+        e = [Fraction(float(wf[n, k])) - Fraction(float(what[n, k])) / Fraction(float(s[k]))
+             for k in range(k_)]
+        tot = Fraction(0)
+        for m in range(m_):
+            y = sum(Fraction(float(xf[m, k])) * e[k] for k in range(k_))
+            tot += y * y
+        out.append(tot)
+    return out
+
+
+@pytest.mark.parametrize("sym", [False, True])
+def test_clip_rows_sse_brute_force_tiny(sym):
+    """Per-row output error of every shrink candidate, and each row's choice,
+    against exact rational arithmetic on a tiny linear."""
+    x = synth.bits(synth.student_t_calibration(3, 128, seed=71))
+    w = synth.bits(synth.normal_weight(4, 128, 0.02, seed=72, n_outliers=3, outlier_scale=20.0))
+    s = O.awq_scales(O.awq_channel_stat(x), [0.5])[0]
+    shrinks = np.array([1.0, 0.8, 0.6], np.float32)
+    sse, choice = O.clip_search_rows(x, w, s, shrinks, sym)
+    assert sse.shape == (3, 4) and choice.shape == (4,)
+    exact = [_row_sse_exact(x, w, s, float(r), sym) for r in shrinks]
+    for j in range(3):
+        for n in range(4):
+            assert abs(sse[j, n] - float(exact[j][n])) <= 1e-12 * float(exact[j][n])
+    for n in range(4):
+        col = [exact[j][n] for j in range(3)]
+        assert choice[n] == col.index(min(col))
+
+
+def test_clip_rows_ties_take_the_lowest_index():
+    """A grid that lists one ratio twice gives equal errors: the first wins."""
+    x = synth.bits(synth.student_t_calibration(8, 256, seed=73))
+    w = synth.bits(synth.normal_weight(6, 256, 0.02, seed=74, n_outliers=2, outlier_scale=20.0))
+    sse, choice = O.clip_search_rows(x, w, None, np.array([0.7, 1.0, 0.7, 1.0], np.float32), False)
+    assert np.array_equal(sse[0], sse[2]) and np.array_equal(sse[1], sse[3])
+    assert set(choice.tolist()) <= {0, 1}
+
+
+def test_clip_rows_invariants():
+    """The per-row errors of one ratio add up to that ratio's whole-linear
+    error (a sum over output channels), and the per-row choice is never worse
+    than the best single ratio."""
+    x = synth.bits(synth.student_t_calibration(16, 256, seed=75))
+    w = synth.bits(synth.normal_weight(10, 256, 0.02, seed=76, n_outliers=2, outlier_scale=20.0))
+    shrinks = synth.shrink_grid(4)
+    s = O.awq_scales(O.awq_channel_stat(x), [0.3])[0]
+    sse, choice = O.clip_search_rows(x, w, s, shrinks, False)
+    xf = O.bf16_bits_to_f32(x).astype(np.float64)
+    for j, r in enumerate(shrinks):
+        y = xf @ O.candidate_error(w, s, r, False).T
+        assert sse[j].sum() == pytest.approx(float(np.sum(y * y)), rel=1e-12)
+    assert sse[choice, np.arange(10)].sum() <= sse.sum(axis=1).min()
+
+
+@pytest.mark.parametrize("sym", [False, True])
+def test_quantize_rows_reduces_to_per_linear_quantize(sym):
+    """One ratio for every row is the per-linear quantizer; distinct ratios
+    quantize each row as that row alone with its ratio."""
+    w = synth.bits(synth.normal_weight(5, 384, 0.02, seed=77, n_outliers=2, outlier_scale=20.0))
+    x = synth.bits(synth.student_t_calibration(4, 384, seed=78))
+    s = O.awq_scales(O.awq_channel_stat(x), [0.4])[0]
+    same = O.quantize_pack_rows(w, sym, s, np.full(5, 0.85, np.float32))
+    ref = O.quantize_pack(w, sym, s, 0.85)
+    for a, b in zip(same, ref):
+        assert (a is None and b is None) or np.array_equal(a, b)
+    rows = np.array([1.0, 0.55, 0.9, 0.75, 0.6], np.float32)
+    mixed = O.quantize_pack_rows(w, sym, s, rows)
+    for n in range(5):
+        one = O.quantize_pack(w[n:n + 1], sym, s, float(rows[n]))
+        assert np.array_equal(mixed[0][n:n + 1], one[0]) and np.array_equal(mixed[1][n:n + 1], one[1])
+        if not sym:
+            assert np.array_equal(mixed[2][n:n + 1], one[2])
