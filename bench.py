@@ -384,7 +384,28 @@ def breakdown(torch, dev, hbm, bf16_peak, bf16_sus):
                                    "frac_bf16_peak": flops / t / 1e9 / bf16_peak,
                                    "candidates": 200, "linears": len(rows),
                                    "argmins_group": arg[-1].tolist()}
-    del ws, w, x
+    del ws, w
+
+    # Per-output-channel clipping search on one Qwen gate_proj (2048 -> 6144)
+    # at alpha 0.5 over the 10-point grid, then the deploy quantize.
+    wg = weights(6144, k, 0.02, 700)
+    s05 = w4.awq_scales(x, [0.5])[0].contiguous()
+    cws = torch.empty(w4.clip_rows_workspace_bytes(2048, 6144, k, 10), dtype=torch.uint8,
+                      device=dev)
+    w4.awq_clip_search_rows(x, wg, sh, False, awq_s=s05, workspace=cws)
+    torch.cuda.synchronize()
+    a_ev.record()
+    for _ in range(reps):
+        sse_r, choice, rows_r = w4.awq_clip_search_rows(x, wg, sh, False, awq_s=s05, workspace=cws)
+    b_ev.record()
+    torch.cuda.synchronize()
+    t = a_ev.elapsed_time(b_ev) / reps
+    flops = 2.0 * 2048 * k * 6144 * 10
+    out["clip_rows_qwen_gate_2048tok_10r"] = {
+        "ms": t, "tflops": flops / t / 1e9, "frac_bf16_peak": flops / t / 1e9 / bf16_peak,
+        "candidates": 10, "rows": 6144,
+        "rows_per_ratio": torch.bincount(choice.long(), minlength=10).tolist()}
+    del cws, wg, x
     torch.cuda.empty_cache()
     return out
 

@@ -302,6 +302,60 @@ w4_status awq_score_grid_static_scratch(const void* x_bf16, int64_t M, const voi
                                         double* sse_out, int32_t* argmin_out, void* stream);
 
 /*
+ * awq_clip_search_rows -- stock per-output-channel clipping search
+ * ([rebuttal] 'Comparability caveat': the d=0 arm clips with stock AWQ's
+ * per-output-channel search; 'Clipping granularity' contrasts it with the one
+ * global ratio a look-ahead loss forces).  For one AWQ scale s (or none) and
+ * a grid of shrink ratios r_j, every output row n takes the ratio whose
+ * quantization error has the least output error in that row:
+ *
+ *   E_j = W - dequant(Q_{r_j}(W diag(s))) diag(1/s)
+ *   sse_rows[j, n] = sum_m (x E_j^T)[m, n]^2        (binary64, fixed order)
+ *   choice[n] = argmin_j sse_rows[j, n]              (lowest j on equal values)
+ *
+ * The linear's output error is the sum of its rows' errors, so the choices
+ * minimise it jointly over all per-row ratio assignments.  Scored in the
+ * s-domain on fp16 tensor-core operands with binary64 sums, like
+ * awq_score_grid (same codes as w4_quantize_pack).
+ *
+ * x_bf16, M      device bf16 [M, K] calibration activations, 1 <= M <= 2^24.
+ * w_bf16, N, K   device bf16 [N, K] weight, 1 <= N <= 2^24, K % 128 == 0.
+ * group          must be 128.
+ * symmetric      0: asymmetric with zero point; 1: symmetric.
+ * awq_s          device float32 [K] AWQ scale (for instance one row of
+ *                w4_awq_scales), or NULL for none (s = 1).
+ * shrinks        host float32 [n_shrink], each in (0, 1]; 1 <= n_shrink <= 64.
+ * sse_rows_out   device float64 [n_shrink, N] out.
+ * choice_out     device int32 [N] out: index into shrinks.
+ * shrink_rows_out  device float32 [N] out (the chosen ratios, ready for
+ *                w4_quantize_pack_rows), or NULL.
+ * workspace      device scratch of at least w4_clip_rows_workspace_bytes(...)
+ *                bytes, 256-byte aligned.
+ * Errors: as awq_score_grid.  Nothing is launched unless every check passes.
+ */
+size_t w4_clip_rows_workspace_bytes(int64_t M, int64_t N, int64_t K, int n_shrink);
+w4_status awq_clip_search_rows(const void* x_bf16, int64_t M, const void* w_bf16, int64_t N,
+                               int64_t K, int group, int symmetric, const float* awq_s,
+                               const float* shrinks, int n_shrink, double* sse_rows_out,
+                               int32_t* choice_out, float* shrink_rows_out, void* workspace,
+                               size_t workspace_bytes, void* stream);
+
+/*
+ * w4_quantize_pack_rows -- w4_quantize_pack with one shrink ratio per output
+ * row (the weight that per-output-channel clipping deploys, [rebuttal]
+ * 'Comparability caveat').  shrink_rows: device float32 [N], 4-byte aligned,
+ * each expected in (0, 1] (device data, not checked: a ratio outside that
+ * range quantizes its row with that wider or degenerate range, and never
+ * reads or writes out of bounds).  Every other argument, the layouts and the
+ * arithmetic are those of w4_quantize_pack; a row's codes, scales and zeros
+ * equal w4_quantize_pack of that row alone with its ratio.
+ */
+w4_status w4_quantize_pack_rows(const void* w_bf16, int64_t N, int64_t K, int group,
+                                int symmetric, const float* awq_s, const float* shrink_rows,
+                                int32_t* qweight, uint16_t* scales_f16, uint16_t* zeros_f16,
+                                void* stream);
+
+/*
  * w4_device_error -- reads (and with clear != 0 resets) the library's device
  * error word.  Every wait inside the tcgen05 kernels is bounded (about one
  * second); a kernel that gives up records it here and returns early, leaving

@@ -111,3 +111,29 @@ def test_binding_fails_loudly_without_library(monkeypatch):
     monkeypatch.setattr(w4, "LIB_PATH", "/nonexistent/libw4.so")
     with pytest.raises(RuntimeError, match="no CPU fallback"):
         w4.lib()
+
+
+def test_clip_rows_validation(L):
+    import ctypes
+    import numpy as np
+    f = L.awq_clip_search_rows
+    r = np.array([1.0, 0.9], np.float32)
+    rp = r.ctypes.data
+    big = 1 << 40
+    assert f(None, 4, A, 8, 128, 128, 0, None, rp, 2, A, A, None, A, big, None) == 1
+    assert f(A, 4, A, 8, 128, 64, 0, None, rp, 2, A, A, None, A, big, None) == 4     # group
+    assert f(A, 4, A, 8, 128, 128, 0, None, rp, 0, A, A, None, A, big, None) == 4    # no grid
+    assert f(A, 4, A, 8, 100, 128, 0, None, rp, 2, A, A, None, A, big, None) == 2    # K % 128
+    bad = np.array([1.0, 1.5], np.float32)
+    assert f(A, 4, A, 8, 128, 128, 0, None, bad.ctypes.data, 2, A, A, None, A, big, None) == 1
+    assert f(A + 2, 4, A, 8, 128, 128, 0, None, rp, 2, A, A, None, A, big, None) == 3
+    assert f(A, 4, A, 8, 128, 128, 0, None, rp, 2, A, A, None, None, 0, None) == 5   # workspace
+    need = L.w4_clip_rows_workspace_bytes(4, 8, 128, 2)
+    assert need > 0
+    assert f(A, 4, A, 8, 128, 128, 0, None, rp, 2, A, A, None, A, need - 1, None) == 5
+    assert f(A, 4, A, 8, 128, 128, 0, None, rp, 2, A, A, None, A + 16, need, None) == 3
+    q = L.w4_quantize_pack_rows
+    assert q(A, 4, 128, 128, 0, None, None, A, A, A, None) == 1                       # no ratios
+    assert q(A, 4, 128, 128, 0, None, A + 2, A, A, A, None) == 3                      # misaligned
+    assert q(A, 4, 128, 128, 1, None, A, A, A, A, None) == 1                          # sym + zeros
+    assert q(A, 4, 128, 64, 0, None, A, A, A, A, None) == 4                           # group

@@ -298,6 +298,71 @@ def test_awq_grid_qwen_k_proj_full_size():
     check_awq(x, w, synth.alpha_grid(20), synth.shrink_grid(10), False)
 
 
+# ------------------------------------ per-output-channel clipping ----
+
+# Per-row errors: each row's sum has only M * K products (no averaging over
+# rows), so the fp16 operand rounding (2^-11 relative on each of x/s and the
+# error operand) can move one row's value by up to ~4 * 2^-11 ~ 2e-3.
+ROW_SSE_RTOL = 2e-3
+
+
+def check_clip_rows(x, w, shrinks, sym, alpha):
+    s = None
+    s_ref = None
+    if alpha is not None:
+        s = w4.awq_scales(x.to(DEV), [alpha])[0].contiguous()
+        s_ref = O.awq_scales(O.awq_channel_stat(synth.bits(x)), [alpha])[0]
+        torch.cuda.synchronize()
+        assert np.array_equal(s.cpu().numpy().view(np.uint32), s_ref.view(np.uint32))
+    sse, choice, rows = w4.awq_clip_search_rows(x.to(DEV), w.to(DEV), shrinks, sym, awq_s=s)
+    torch.cuda.synchronize()
+    sse = sse.cpu().numpy()
+    choice = choice.cpu().numpy()
+    ref, ref_choice = O.clip_search_rows(synth.bits(x), synth.bits(w), s_ref, shrinks, sym)
+    rel = np.max(np.abs(sse - ref) / ref)
+    assert rel <= ROW_SSE_RTOL, f"per-row SSE relative error {rel:.3e}"
+    n = ref.shape[1]
+    # Each row's pick must be least within the comparison's own error.
+    picked = ref[choice, np.arange(n)]
+    assert np.all(picked <= ref.min(axis=0) * (1 + 2 * ROW_SSE_RTOL))
+    exact_ties = int(np.sum(choice != ref_choice))
+    print(f"rows {n}: {exact_ties} picks differ from the oracle's inside the error band")
+    assert np.allclose(rows.cpu().numpy(), np.asarray(shrinks, np.float32)[choice])
+    # Deploy: quantize with the chosen ratios, bit-exact against the oracle.
+    qw, sc, zr = w4.quantize_pack_rows(w.to(DEV), sym, rows, awq_s=s)
+    torch.cuda.synchronize()
+    oq, os_, oz = O.quantize_pack_rows(synth.bits(w), sym, s_ref, np.asarray(shrinks, np.float32)[choice])
+    assert_quant_equal((qw, sc, zr), (oq, os_, oz), sym)
+    return rel
+
+
+@pytest.mark.parametrize("sym", [False, True])
+@pytest.mark.parametrize("alpha", [None, 0.5])
+def test_clip_rows_small(sym, alpha):
+    x = synth.student_t_calibration(200, 640, seed=81)   # ragged token tile
+    w = synth.normal_weight(300, 640, 0.02, seed=82, n_outliers=6, outlier_scale=20.0)
+    check_clip_rows(x, w, synth.shrink_grid(10), sym, alpha)
+
+
+def test_clip_rows_qwen_k_proj_full_size():
+    """One Qwen3-1.7B k_proj (2048 -> 1024) on 2048 heavy-tailed calibration
+    tokens, the 10-point shrink grid at alpha 0.5."""
+    x = synth.student_t_calibration(2048, 2048, seed=83)
+    w = synth.normal_weight(1024, 2048, 0.02, seed=84)
+    check_clip_rows(x, w, synth.shrink_grid(10), False, 0.5)
+
+
+@pytest.mark.parametrize("sym", [False, True])
+def test_quantize_rows_uniform_equals_per_linear(sym):
+    w = synth.normal_weight(257, 1024, 0.02, seed=85, n_outliers=4, outlier_scale=20.0).to(DEV)
+    rows = torch.full((257,), 0.8, dtype=torch.float32, device=DEV)
+    a = w4.quantize_pack_rows(w, sym, rows)
+    b = w4.quantize_pack(w, sym, None, 0.8)
+    torch.cuda.synchronize()
+    for u, v in zip(a, b):
+        assert (u is None and v is None) or torch.equal(u, v)
+
+
 # ------------------------------------------------------ failure path ----
 
 def test_bounded_wait_reports_and_context_survives():

@@ -15,7 +15,8 @@ import os
 from typing import Optional, Sequence
 
 __all__ = [
-    "W4Error", "lib", "quantize_pack", "quantize_pack_batched", "w4a16_linear",
+    "W4Error", "lib", "quantize_pack", "quantize_pack_batched", "quantize_pack_rows",
+    "awq_clip_search_rows", "clip_rows_workspace_bytes", "w4a16_linear",
     "w4a16_linear_batched", "awq_scales", "awq_score_grid", "awq_score_grid_static_scratch",
     "awq_workspace_bytes", "device_error", "selftest_bounded_wait",
     "LINEAR_FORCE_GEMV", "LINEAR_FORCE_GEMM", "LINEAR_PDL", "LINEAR_STATIC_WEIGHTS",
@@ -87,6 +88,14 @@ def _declare(L: ctypes.CDLL) -> None:
     L.awq_score_grid_static_scratch.argtypes = [_p, _i64, _p, _i64, _i64, ctypes.c_int,
                                                 ctypes.c_int, _p, ctypes.c_int, _p, ctypes.c_int,
                                                 _p, ctypes.c_int, _p, _p, _p]
+    L.w4_clip_rows_workspace_bytes.restype = ctypes.c_size_t
+    L.w4_clip_rows_workspace_bytes.argtypes = [_i64, _i64, _i64, ctypes.c_int]
+    L.awq_clip_search_rows.restype = ctypes.c_int
+    L.awq_clip_search_rows.argtypes = [_p, _i64, _p, _i64, _i64, ctypes.c_int, ctypes.c_int, _p,
+                                       _p, ctypes.c_int, _p, _p, _p, _p, ctypes.c_size_t, _p]
+    L.w4_quantize_pack_rows.restype = ctypes.c_int
+    L.w4_quantize_pack_rows.argtypes = [_p, _i64, _i64, ctypes.c_int, ctypes.c_int, _p, _p, _p,
+                                        _p, _p, _p]
     L.w4_device_error.restype = ctypes.c_int
     L.w4_device_error.argtypes = [ctypes.c_int, _p]
     L.w4_selftest_bounded_wait.restype = ctypes.c_int
@@ -152,6 +161,29 @@ def quantize_pack(w, symmetric: bool, awq_s=None, shrink: float = 1.0, group: in
                                     float(shrink), qw.data_ptr(), sc.data_ptr(),
                                     None if zr is None else zr.data_ptr(), _stream(w.device))
     _check(st, "w4_quantize_pack")
+    return qw, sc, zr
+
+
+def quantize_pack_rows(w, symmetric: bool, shrink_rows, awq_s=None, group: int = 128):
+    """quantize_pack with one shrink ratio per output row (float32 [N] on the
+    weight's device), as chosen by awq_clip_search_rows."""
+    torch = _torch()
+    _cuda(w, torch.bfloat16, "w")
+    _cuda(shrink_rows, torch.float32, "shrink_rows")
+    n, k = w.shape
+    if shrink_rows.numel() != n:
+        raise ValueError("shrink_rows needs one ratio per output row")
+    if awq_s is not None:
+        _cuda(awq_s, torch.float32, "awq_s")
+    qw = torch.empty((n, k // 8), dtype=torch.int32, device=w.device)
+    sc = torch.empty((n, k // group), dtype=torch.int16, device=w.device)
+    zr = None if symmetric else torch.empty((n, k // group), dtype=torch.int16, device=w.device)
+    with torch.cuda.device(w.device):
+        st = lib().w4_quantize_pack_rows(w.data_ptr(), n, k, group, int(bool(symmetric)),
+                                         None if awq_s is None else awq_s.data_ptr(),
+                                         shrink_rows.data_ptr(), qw.data_ptr(), sc.data_ptr(),
+                                         None if zr is None else zr.data_ptr(), _stream(w.device))
+    _check(st, "w4_quantize_pack_rows")
     return qw, sc, zr
 
 
@@ -286,6 +318,41 @@ def awq_score_grid(x, w, alphas, shrinks, symmetric: bool, seg_offsets=None, wor
                                   _stream(x.device))
     _check(st, "awq_score_grid")
     return sse, arg
+
+
+def clip_rows_workspace_bytes(m: int, n: int, k: int, n_shrink: int) -> int:
+    return int(lib().w4_clip_rows_workspace_bytes(m, n, k, n_shrink))
+
+
+def awq_clip_search_rows(x, w, shrinks, symmetric: bool, awq_s=None, workspace=None,
+                         group: int = 128):
+    """Per-output-channel clipping search: (sse_rows float64 [n_shrink, N],
+    choice int32 [N], shrink_rows float32 [N]) on the tensors' device."""
+    torch = _torch()
+    import numpy as np
+    _cuda(x, torch.bfloat16, "x")
+    _cuda(w, torch.bfloat16, "w")
+    if awq_s is not None:
+        _cuda(awq_s, torch.float32, "awq_s")
+    m, k = x.shape
+    n = w.shape[0]
+    r = np.ascontiguousarray(np.asarray(shrinks, dtype=np.float32))
+    if workspace is None:
+        workspace = torch.empty(clip_rows_workspace_bytes(m, n, k, len(r)), dtype=torch.uint8,
+                                device=x.device)
+    sse = torch.empty((len(r), n), dtype=torch.float64, device=x.device)
+    choice = torch.empty(n, dtype=torch.int32, device=x.device)
+    rows = torch.empty(n, dtype=torch.float32, device=x.device)
+    with torch.cuda.device(x.device):
+        st = lib().awq_clip_search_rows(x.data_ptr(), m, w.data_ptr(), n, k, group,
+                                        int(bool(symmetric)),
+                                        None if awq_s is None else awq_s.data_ptr(),
+                                        r.ctypes.data, len(r), sse.data_ptr(), choice.data_ptr(),
+                                        rows.data_ptr(), workspace.data_ptr(),
+                                        workspace.numel() * workspace.element_size(),
+                                        _stream(x.device))
+    _check(st, "awq_clip_search_rows")
+    return sse, choice, rows
 
 
 def awq_score_grid_static_scratch(x, w, alphas, shrinks, symmetric: bool, seg_offsets=None,

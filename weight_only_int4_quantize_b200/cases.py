@@ -5,6 +5,7 @@ timing.  Inputs are seeded and generated on the device.
     python -m weight_only_int4_quantize_b200.cases linear --m 8 --n 17408 --k 5120 [--sym] [--gemm]
     python -m weight_only_int4_quantize_b200.cases awq --m 2048 --n 1024 --k 2048 --na 20 --nr 10
     python -m weight_only_int4_quantize_b200.cases decode_batch --m 1 --blocks 4
+    python -m weight_only_int4_quantize_b200.cases clip_rows --m 2048 --n 6144 --k 2048 --nr 10
 
 Each case captures --iters launches in one CUDA graph (so host launch
 overhead does not count), replays it once to warm up, times one replay with
@@ -60,7 +61,7 @@ def _time(fn, iters, graph=True):
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("case", choices=["quantize", "linear", "awq", "decode_batch"])
+    ap.add_argument("case", choices=["quantize", "linear", "awq", "decode_batch", "clip_rows"])
     ap.add_argument("--blocks", type=int, default=4,
                     help="decode_batch: Qwen3-1.7B-shaped blocks (7 linears each) in one batch")
     ap.add_argument("--m", type=int, default=8)
@@ -114,6 +115,15 @@ def main():
         flags = w4.LINEAR_PDL | w4.LINEAR_STATIC_WEIGHTS if a.pdl else 0
         ms = _time(lambda: w4.w4a16_linear_batched(arr, a.m, flags), a.iters, not a.eager)
         out.update(ms=ms, gbs=byts / ms / 1e6, linears=len(items))
+    elif a.case == "clip_rows":
+        g = torch.Generator(device="cuda")
+        g.manual_seed(3)
+        x = (torch.randn(a.m, a.k, generator=g, device="cuda")).to(torch.bfloat16)
+        sh = synth.shrink_grid(a.nr)
+        ws = torch.empty(w4.clip_rows_workspace_bytes(a.m, a.n, a.k, a.nr), dtype=torch.uint8,
+                         device="cuda")
+        ms = _time(lambda: w4.awq_clip_search_rows(x, w, sh, a.sym, workspace=ws), a.iters, False)
+        out.update(ms=ms, tflops=2.0 * a.m * a.n * a.k * a.nr / ms / 1e9)
     else:
         g = torch.Generator(device="cuda")
         g.manual_seed(3)

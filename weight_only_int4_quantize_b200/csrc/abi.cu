@@ -91,6 +91,22 @@ AwqWs awq_layout(int64_t M, int64_t N, int64_t K, int n_alpha, int n_shrink, int
   return w;
 }
 
+// Workspace of awq_clip_search_rows: every region 256-byte aligned.
+struct ClipWs {
+  size_t ones, a, e, partials, total;
+};
+
+ClipWs clip_layout(int64_t M, int64_t N, int64_t K, int n_shrink) {
+  ClipWs w;
+  w.ones = 0;
+  w.a = w.ones + round256(sizeof(float) * K);
+  w.e = w.a + round256(sizeof(uint16_t) * M * K);
+  w.partials = w.e + round256(sizeof(uint16_t) * static_cast<size_t>(n_shrink) * N * K);
+  w.total = w.partials + round256(sizeof(double) * n_shrink *
+                                  static_cast<size_t>(colsumsq_row_tiles(static_cast<int>(M))) * N);
+  return w;
+}
+
 }  // namespace
 }  // namespace w4
 
@@ -477,6 +493,89 @@ w4_status awq_score_grid(const void* x_bf16, int64_t M, const void* w_bf16, int6
   if (e != cudaSuccess) return cuda_status(e, "awq reduce");
   return cuda_status(launch_awq_argmin(sse_out, n_seg, n_alpha, n_shrink, c1, argmin_out, s),
                      "awq argmin");
+}
+
+size_t w4_clip_rows_workspace_bytes(int64_t M, int64_t N, int64_t K, int n_shrink) {
+  if (M < 1 || N < 1 || K < 1 || n_shrink < 1) return 0;
+  return clip_layout(M, N, K, n_shrink).total;
+}
+
+w4_status awq_clip_search_rows(const void* x_bf16, int64_t M, const void* w_bf16, int64_t N,
+                               int64_t K, int group, int symmetric, const float* awq_s,
+                               const float* shrinks, int n_shrink, double* sse_rows_out,
+                               int32_t* choice_out, float* shrink_rows_out, void* workspace,
+                               size_t workspace_bytes, void* stream) {
+  if (!x_bf16 || !w_bf16 || !shrinks || !sse_rows_out || !choice_out) return W4_ERR_INVALID_ARG;
+  if (group != 128) return W4_ERR_UNSUPPORTED;
+  if (n_shrink < 1 || n_shrink > kMaxGrid) return W4_ERR_UNSUPPORTED;
+  if (M < 1 || N < 1 || !valid_k(K) || M > (int64_t{1} << 24) || N > (int64_t{1} << 24))
+    return W4_ERR_SHAPE;
+  ShrinkList sl;
+  sl.n = n_shrink;
+  for (int j = 0; j < n_shrink; ++j) {
+    if (!(shrinks[j] > 0.0f && shrinks[j] <= 1.0f)) return W4_ERR_INVALID_ARG;
+    sl.v[j] = shrinks[j];
+  }
+  if (!aligned16(x_bf16) || !aligned16(w_bf16) || !aligned16(sse_rows_out) ||
+      !aligned16(choice_out) || (awq_s && !aligned16(awq_s)) ||
+      (shrink_rows_out && (reinterpret_cast<uintptr_t>(shrink_rows_out) & 3u) != 0))
+    return W4_ERR_ALIGNMENT;
+  const ClipWs L = clip_layout(M, N, K, n_shrink);
+  if (!workspace || workspace_bytes < L.total) return W4_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return W4_ERR_ALIGNMENT;
+
+  int sms = 0;
+  unsigned* err = nullptr;
+  w4_status st = device_info(&sms, &err);
+  if (st != W4_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const float* sv = awq_s;
+  cudaError_t e = cudaSuccess;
+  if (!sv) {
+    float* ones = reinterpret_cast<float*>(ws + L.ones);
+    e = launch_fill_ones(ones, K, s);
+    if (e != cudaSuccess) return cuda_status(e, "clip search unit scale");
+    sv = ones;
+  }
+  void* a_buf = ws + L.a;
+  void* e_buf = ws + L.e;
+  double* partials = reinterpret_cast<double*>(ws + L.partials);
+  e = launch_awq_xs(x_bf16, sv, M, K, a_buf, s, sms);
+  if (e != cudaSuccess) return cuda_status(e, "clip search x/s operand");
+  e = launch_awq_err(w_bf16, sv, N, K, symmetric != 0, sl, e_buf, s, sms);
+  if (e != cudaSuccess) return cuda_status(e, "clip search error operand");
+  e = launch_colsumsq_gemm(a_buf, static_cast<int>(M), e_buf, static_cast<int>(N),
+                           static_cast<int>(K), n_shrink, partials, s, err);
+  if (e != cudaSuccess) return cuda_status(e, "clip search tcgen05 column sum-of-squares GEMM");
+  return cuda_status(launch_clip_rows_select(partials, n_shrink,
+                                             colsumsq_row_tiles(static_cast<int>(M)), N, sl,
+                                             sse_rows_out, choice_out, shrink_rows_out, s),
+                     "clip search row selection");
+}
+
+w4_status w4_quantize_pack_rows(const void* w_bf16, int64_t N, int64_t K, int group,
+                                int symmetric, const float* awq_s, const float* shrink_rows,
+                                int32_t* qweight, uint16_t* scales_f16, uint16_t* zeros_f16,
+                                void* stream) {
+  if (!shrink_rows) return W4_ERR_INVALID_ARG;
+  if (group != 128 && w_bf16 && qweight && scales_f16) return W4_ERR_UNSUPPORTED;
+  w4_status st = check_quant_item(w_bf16, N, K, symmetric, awq_s, 1.0f, qweight, scales_f16,
+                                  zeros_f16);
+  if (st != W4_OK) return st;
+  if (group != 128) return W4_ERR_UNSUPPORTED;
+  if ((reinterpret_cast<uintptr_t>(shrink_rows) & 3u) != 0) return W4_ERR_ALIGNMENT;
+  int sms = 0;
+  unsigned* err = nullptr;
+  st = device_info(&sms, &err);
+  if (st != W4_OK) return st;
+  QuantBatch b;
+  b.count = 0;
+  b.unit_start[0] = 0;
+  quant_batch_add(b, w_bf16, N, K, awq_s, 1.0f, qweight, scales_f16, zeros_f16, shrink_rows);
+  return cuda_status(launch_quantize_pack_batch(b, symmetric != 0,
+                                                static_cast<cudaStream_t>(stream), sms, err),
+                     "quantize+pack (per-row shrink) launch");
 }
 
 // Variant of awq_score_grid for callers that cannot allocate a workspace:

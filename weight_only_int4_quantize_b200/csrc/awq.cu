@@ -13,6 +13,11 @@
 // binary64; awq_reduce_kernel adds the tile sums in fixed order and
 // awq_argmin_kernel takes the selections.  The codes of every candidate are
 // the quantize+pack kernel's codes (same quant_group.cuh arithmetic).
+//
+// The per-output-channel clipping search ("Comparability caveat" of the same
+// card: stock AWQ's per-output-channel clipping) uses the same operands for
+// one s and the shrink grid, a per-column epilogue of the same GEMM, and
+// clip_rows_select_kernel for each row's least-error ratio.
 #include "quant_group.cuh"
 #include "w4_kernels.h"
 
@@ -180,7 +185,52 @@ __global__ void awq_argmin_kernel(const double* __restrict__ sse, int n_seg, int
   out[4 * n_seg + 3] = -1;
 }
 
+// Per-output-channel clipping: sse_rows[c, n] = sum over row tiles (fixed
+// order) of the column sums, choice[n] = the lowest c of least error, and
+// the chosen ratio itself.  One thread per output channel.
+__global__ void clip_rows_select_kernel(const double* __restrict__ partials, int n_cand,
+                                        int row_tiles, int64_t N, ShrinkList shrinks,
+                                        double* __restrict__ sse_rows, int32_t* __restrict__ choice,
+                                        float* __restrict__ shrink_rows) {
+  const int64_t n = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (n >= N) return;
+  int best = 0;
+  double best_v = 0.0;
+  for (int c = 0; c < n_cand; ++c) {
+    double v = 0.0;
+    for (int t = 0; t < row_tiles; ++t) v += partials[(static_cast<size_t>(c) * row_tiles + t) * N + n];
+    sse_rows[static_cast<size_t>(c) * N + n] = v;
+    if (c == 0 || v < best_v) {
+      best = c;
+      best_v = v;
+    }
+  }
+  choice[n] = best;
+  if (shrink_rows) shrink_rows[n] = shrinks.v[best];
+}
+
+__global__ void fill_ones_kernel(float* __restrict__ p, int64_t n) {
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x)
+    p[i] = 1.0f;
+}
+
 }  // namespace
+
+cudaError_t launch_clip_rows_select(const double* partials, int n_cand, int row_tiles, int64_t N,
+                                    const ShrinkList& shrinks, double* sse_rows, int32_t* choice,
+                                    float* shrink_rows, cudaStream_t stream) {
+  const int64_t blocks = (N + 127) / 128;
+  clip_rows_select_kernel<<<static_cast<unsigned>(blocks), 128, 0, stream>>>(
+      partials, n_cand, row_tiles, N, shrinks, sse_rows, choice, shrink_rows);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_fill_ones(float* p, int64_t n, cudaStream_t stream) {
+  fill_ones_kernel<<<static_cast<unsigned>((n + 255) / 256 < 1024 ? (n + 255) / 256 : 1024), 256,
+                     0, stream>>>(p, n);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_awq_scales(const void* x, int64_t M, int64_t K, const AlphaList& alphas,
                               float* s_out, cudaStream_t stream) {

@@ -15,7 +15,10 @@
 //     epilogue stores y in bf16;
 //   - AWQ candidate scoring: A = x / s (fp16, TMA), B = W s - w_hat (fp16,
 //     TMA, one candidate per grid z), epilogue writes per-tile sums of y^2
-//     in binary64 (deterministic order).
+//     in binary64 (deterministic order);
+//   - the per-output-channel clipping search: the same operands, epilogue
+//     writes per-column (output channel) sums of y^2 over the tile's rows in
+//     binary64 (deterministic order).
 //
 // Every mbarrier wait is bounded (w4_common.cuh); a CTA that gives up sets
 // the device error word, drains its own TMA loads and MMAs, frees its TMEM
@@ -52,7 +55,7 @@ struct Tile {
 };
 
 enum : int { kBDequant = 0, kBTma = 1 };
-enum : int { kEpiStoreBf16 = 0, kEpiSumSquares = 1 };
+enum : int { kEpiStoreBf16 = 0, kEpiSumSquares = 1, kEpiColSumSquares = 2 };
 
 constexpr unsigned kKernelIdGemm = 2;
 
@@ -65,12 +68,14 @@ struct SmemLayout {
   static constexpr uint32_t bars = b + kStages * Tile<MT, NB>::kTileBBytes;
   // full_a[S], full_b[S], empty[S], acc_full, done
   static constexpr uint32_t misc = bars + (3 * kStages + 2) * 8;
-  static constexpr uint32_t total = misc + 64 + 16 * 16 * 8;  // + chunk sums
+  // + chunk sums (sum of squares) or per-column sums of the four TMEM lane
+  // quarters (column sums of squares): 4 x 256 doubles.
+  static constexpr uint32_t total = misc + 64 + 4 * 256 * 8;
   static constexpr size_t bytes = total + 1024;
 };
 
 struct SumSqArgs {
-  double* partials;     // [n_cand][n_seg][tiles]
+  double* partials;     // [n_cand][n_seg][tiles]; column sums: [n_cand][m_tiles][N]
   int n_seg;
   int seg_off[17];      // column (N) boundaries, multiples of 16 inside
   int tiles;            // m_tiles * n_tiles
@@ -382,6 +387,51 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         }
+      } else if (EPI == kEpiColSumSquares) {
+        // Column sums of y^2 over the tile's rows: per 16-column chunk each
+        // thread squares its row's 16 values (its row of each 128-row half
+        // in turn), a fixed butterfly over the warp's 32 lanes leaves lane
+        // pair (2c, 2c+1) with the sum of the chunk's column c, and the four
+        // lane quarters are added in order below.
+        static_assert(EPI != kEpiColSumSquares || NB == BN, "column sums use 256-column tiles");
+        double* colq = chunk_sums;  // [4][256]
+        for (int c = 0; c < 8; ++c) {
+          const int col = 128 * ch + 16 * c;
+          double d[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) d[i] = 0.0;
+#pragma unroll
+          for (int mt = 0; mt < MT; ++mt) {
+            const int m = m0 + 128 * mt + 32 * q + lane;
+            uint32_t r[16];
+            tmem_ld_32x32b_x16(tmem_base + (static_cast<uint32_t>(32 * q) << 16) + NB * mt + col,
+                               r);
+            tmem_ld_wait();
+            if (m < M) {
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                const double v = static_cast<double>(__uint_as_float(r[i]));
+                d[i] = fma(v, v, d[i]);
+              }
+            }
+          }
+          // Reduce-scatter: at width w the lanes with bit w set keep the upper
+          // half of their columns and receive it from the partner lane.
+#pragma unroll
+          for (int w = 16, nv = 8; w >= 2; w >>= 1, nv >>= 1) {
+            const bool up = (lane & w) != 0;
+#pragma unroll
+            for (int i = 0; i < nv; ++i) {
+              const double keep = up ? d[nv + i] : d[i];
+              const double send = up ? d[i] : d[nv + i];
+              d[i] = keep + __shfl_xor_sync(0xffffffffu, send, w);
+            }
+          }
+          d[0] += __shfl_xor_sync(0xffffffffu, d[0], 1);
+          const int cl = ((lane >> 4) & 1) * 8 + ((lane >> 3) & 1) * 4 + ((lane >> 2) & 1) * 2 +
+                         ((lane >> 1) & 1);
+          if ((lane & 1) == 0) colq[q * 256 + col + cl] = d[0];
+        }
       } else {
         // Sum of squares per 16-column chunk: thread -> fixed-order shuffle
         // tree over the 32 rows of this warp -> shared -> fixed order over
@@ -411,6 +461,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int o = 16; o; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
           if (lane == 0) chunk_sums[(8 * ch + c) * 4 + q] = acc;
         }
+      }
+    }
+    if (EPI == kEpiColSumSquares) {
+      asm volatile("bar.sync 1, 256;" ::: "memory");  // the eight epilogue warps
+      const int n = n0 + pt;
+      if (n < N && !*abort_flag) {
+        const double* colq = chunk_sums;
+        const double v = ((colq[pt] + colq[256 + pt]) + colq[512 + pt]) + colq[768 + pt];
+        ss.partials[(static_cast<size_t>(cand) * gridDim.y + blockIdx.y) * N + n] = v;
       }
     }
     if (EPI == kEpiSumSquares) {
@@ -591,6 +650,37 @@ cudaError_t launch_sumsq_gemm(const void* a_f16, int M, const void* b_f16, int N
   return launch_gemm<gemm_tc_kernel<kBTma, kEpiSumSquares, false, 1, BN>, SmemLayout<1, BN>::bytes>(
       grid, false, stream, ta, tb, nullptr, nullptr, nullptr, nullptr, ss, M, N, K, 0, err);
 }
+
+cudaError_t launch_colsumsq_gemm(const void* a_f16, int M, const void* b_f16, int N, int K,
+                                 int n_cand, double* partials, cudaStream_t stream,
+                                 unsigned* err) {
+  CUtensorMap ta, tb;
+  const uint64_t da[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(M)};
+  const uint64_t sa[1] = {static_cast<uint64_t>(K) * 2};
+  const int mt = sumsq_mt(M);
+  const uint32_t ba[2] = {BK, static_cast<uint32_t>(mt * BM)};
+  if (encode_tmap(&ta, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, da, sa, ba, a_f16) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+  const uint64_t db[3] = {static_cast<uint64_t>(K), static_cast<uint64_t>(N),
+                          static_cast<uint64_t>(n_cand)};
+  const uint64_t sb[2] = {static_cast<uint64_t>(K) * 2, static_cast<uint64_t>(K) * 2 * N};
+  const uint32_t bb[3] = {BK, BN, 1};
+  if (encode_tmap(&tb, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, db, sb, bb, b_f16) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+  SumSqArgs ss = {};
+  ss.partials = partials;
+  dim3 grid((N + BN - 1) / BN, (M + mt * BM - 1) / (mt * BM), n_cand);
+  ss.tiles = grid.x * grid.y;
+  if (mt == 2)
+    return launch_gemm<gemm_tc_kernel<kBTma, kEpiColSumSquares, false, 2, BN>,
+                       SmemLayout<2, BN>::bytes>(grid, false, stream, ta, tb, nullptr, nullptr,
+                                                 nullptr, nullptr, ss, M, N, K, 0, err);
+  return launch_gemm<gemm_tc_kernel<kBTma, kEpiColSumSquares, false, 1, BN>,
+                     SmemLayout<1, BN>::bytes>(grid, false, stream, ta, tb, nullptr, nullptr,
+                                               nullptr, nullptr, ss, M, N, K, 0, err);
+}
+
+int colsumsq_row_tiles(int M) { return (M + sumsq_mt(M) * BM - 1) / (sumsq_mt(M) * BM); }
 
 int sumsq_tiles(int M, int N) {
   return ((N + BN - 1) / BN) * ((M + sumsq_mt(M) * BM - 1) / (sumsq_mt(M) * BM));

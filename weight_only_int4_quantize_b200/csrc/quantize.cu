@@ -423,7 +423,11 @@ __global__ void __launch_bounds__(kQThreads, kQCtasPerSm)
       gmax = SYM ? ax : mx;
       gmin = mn;
     }
-    const GroupQ g = group_params<SYM>(gmax, gmin, b.shrink[it]);
+    const float* srow = b.shrink_rows[it];
+    // (lanes past the last group read no row ratio)
+    const float shrink =
+        (srow && valid) ? __ldg(srow + gi / b.groups_per_row[it]) : b.shrink[it];
+    const GroupQ g = group_params<SYM>(gmax, gmin, shrink);
     const float amax = SYM ? gmax : fmaxf(fabsf(gmax), fabsf(gmin));
     const bool big = !(__fmul_rn(amax, g.rcp) < 16384.0f);
     const float rh = __fmul_rn(g.rcp, 1.000003814697265625f);  // 1 + 2^-18
@@ -493,11 +497,13 @@ cudaError_t launch_quantize_pack_batch(const QuantBatch& b, bool symmetric, cuda
 }
 
 void quant_batch_add(QuantBatch& b, const void* w, int64_t N, int64_t K, const float* s,
-                     float shrink, int32_t* qweight, uint16_t* scales, uint16_t* zeros) {
+                     float shrink, int32_t* qweight, uint16_t* scales, uint16_t* zeros,
+                     const float* shrink_rows) {
   const int i = b.count;
   b.w[i] = w;
   b.s[i] = s;
   b.shrink[i] = shrink;
+  b.shrink_rows[i] = shrink_rows;
   b.qw[i] = qweight;
   b.scales[i] = scales;
   b.zeros[i] = zeros;

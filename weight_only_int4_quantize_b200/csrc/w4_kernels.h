@@ -27,6 +27,7 @@ struct QuantBatch {
   const void* w[kQuantBatch];
   const float* s[kQuantBatch];
   float shrink[kQuantBatch];
+  const float* shrink_rows[kQuantBatch];  // per-row ratios [N] (device) or NULL
   void* qw[kQuantBatch];
   uint16_t* scales[kQuantBatch];
   uint16_t* zeros[kQuantBatch];
@@ -35,7 +36,8 @@ struct QuantBatch {
   int64_t unit_start[kQuantBatch + 1];  // prefix sums of ceil(groups / 32) (chunks)
 };
 void quant_batch_add(QuantBatch& b, const void* w, int64_t N, int64_t K, const float* s,
-                     float shrink, int32_t* qweight, uint16_t* scales, uint16_t* zeros);
+                     float shrink, int32_t* qweight, uint16_t* scales, uint16_t* zeros,
+                     const float* shrink_rows = nullptr);
 cudaError_t launch_quantize_pack_batch(const QuantBatch& b, bool symmetric, cudaStream_t stream,
                                        int num_sms, unsigned* err);
 
@@ -94,6 +96,12 @@ cudaError_t launch_sumsq_gemm(const void* a_f16, int M, const void* b_f16, int N
                               int n_cand, double* partials, int n_seg, const int* seg_off,
                               cudaStream_t stream, unsigned* err);
 int sumsq_tiles(int M, int N);
+// Per-column sums of (A . B_c^T)^2 over the rows of each row tile:
+// partials[c][row_tile][n] in binary64 (fixed order).
+cudaError_t launch_colsumsq_gemm(const void* a_f16, int M, const void* b_f16, int N, int K,
+                                 int n_cand, double* partials, cudaStream_t stream,
+                                 unsigned* err);
+int colsumsq_row_tiles(int M);
 
 cudaError_t launch_awq_scales(const void* x, int64_t M, int64_t K, const AlphaList& alphas,
                               float* s_out, cudaStream_t stream);
@@ -105,6 +113,11 @@ cudaError_t launch_awq_reduce(const double* partials, int n_cand, int n_seg, int
                               double* sse, cudaStream_t stream);
 cudaError_t launch_awq_argmin(const double* sse, int n_seg, int n_a, int n_r, int c1,
                               int32_t* out, cudaStream_t stream);
+
+cudaError_t launch_clip_rows_select(const double* partials, int n_cand, int row_tiles, int64_t N,
+                                    const ShrinkList& shrinks, double* sse_rows, int32_t* choice,
+                                    float* shrink_rows, cudaStream_t stream);
+cudaError_t launch_fill_ones(float* p, int64_t n, cudaStream_t stream);
 
 // Device address of the fixed scratch behind awq_score_grid_static_scratch
 // on the current device (looked up once per device, then cached).
