@@ -53,10 +53,9 @@ TRAFFIC_CAPTURES = {
     # decode_batch --m 1 --blocks 4 (streaming kernel): 111.51 MB over 107.27 MB algorithmic
     "gemv_w4a16": {"source": "gemv_stream.cu", "digest": "000ccc3d7684a4dc",
                    "ratio": 111.51 / 107.27},
-    # quantize 17408 x 5120: 202.90 MB over 225.67 MB (part of the written codes
+    # quantize 17408 x 5120: 202.47 MB over 225.67 MB (part of the written codes
     # is still in the write-back L2 when the kernel ends)
-    "quantize_pack": {"source": "quantize.cu", "digest": "fe920be4faac0b8e", "ratio": 202.90 / 225.67},
-}
+    "quantize_pack": {"source": "quantize.cu", "digest": "f3061dcc5ac9fd85", "ratio": 202.47 / 225.67},
 
 # --------------------------------------------------------------------------
 
@@ -350,6 +349,18 @@ def breakdown(torch, dev, hbm, bf16_peak, bf16_sus):
             rec["frac_bf16_peak"] = rec["tflops"] / bf16_peak
             rec["frac_hbm"] = rec["gbs"] / hbm
             out[f"{tag}_M{m}"] = rec
+            if m >= 512:
+                # The same linears as one batched call (independent problems):
+                # grouped prefill launches share the GPU between linears.
+                ys_g = [torch.empty(m, n, dtype=torch.bfloat16, device=dev)
+                        for (k, n, cnt, qw, sc) in packed for _ in range(cnt)]
+                arr = w4.linear_items([(xs[k], qw, sc, None, yg) for (k, n, cnt, qw, sc), yg in
+                                       zip([p for p in packed for _ in range(p[2])], ys_g)])
+                gr2 = capture(torch, lambda arr=arr, m=m: w4.w4a16_linear_batched(arr, m))
+                t2 = time_graph(torch, gr2, 20)
+                out[f"{tag}_M{m}_grouped"] = {"ms": t2, "tflops": flops / t2 / 1e9,
+                                              "frac_bf16_peak": flops / t2 / 1e9 / bf16_peak}
+                del gr2, arr, ys_g
             del gr, xs, ys
         del packed
     torch.cuda.empty_cache()

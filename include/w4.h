@@ -184,7 +184,8 @@ w4_status w4a16_linear(const void* x_bf16, int64_t M, const int32_t* qweight,
  * runs up to 256 linears per persistent streaming launch (or, for a launch
  * too small to fill the GPU, the tensor-map kernel); 9 <= M <= 64 (K <=
  * 81920) runs the tensor-map kernel with up to 32 linears per launch; larger
- * M runs one prefill GEMM per linear.  flags: W4_LINEAR_PDL,
+ * M runs grouped prefill GEMM launches, up to 16 linears each (every CTA
+ * finds its linear and tile; the tile shape is chosen for the group).  flags: W4_LINEAR_PDL,
  * W4_LINEAR_STATIC_WEIGHTS and the W4_LINEAR_DECODE_* choice only.  items: host array.  Each result meets the
  * same error bound as a per-linear call (the K split of a batch, and so the
  * binary32 summation order, may differ from a single call's).

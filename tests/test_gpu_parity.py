@@ -400,6 +400,28 @@ def test_quantize_batched_mixed_tensors(sym):
         assert_quant_equal((qw, sc, zr), ref, sym)
 
 
+@pytest.mark.parametrize("sym", [False, True])
+def test_prefill_grouped_many_linears(sym):
+    """More linears than one grouped prefill launch takes (16), mixed K and
+    ragged N, at a ragged token count: every result meets the bound."""
+    rng = np.random.default_rng(9)
+    items, refs = [], []
+    for i in range(21):
+        k = int(rng.choice([128, 384, 1024]))
+        n = int(rng.integers(1, 600))
+        w = synth.normal_weight(n, k, 0.02, seed=4000 + i)
+        x = synth.normal_activations(130, k, seed=7000 + i)
+        qw, sc, zr = w4.quantize_pack(w.to(DEV), sym)
+        y = torch.empty(130, n, dtype=torch.bfloat16, device=DEV)
+        items.append((x.to(DEV), qw, sc, zr, y))
+        oc, os_, oz = O.quantize_rtn(synth.bits(w), sym)
+        refs.append(O.linear(synth.bits(x), O.dequantize(oc, os_, oz)))
+    w4.w4a16_linear_batched(items, 130)
+    torch.cuda.synchronize()
+    worst = max(max_rel_err(it[4], ref) for it, ref in zip(items, refs))
+    assert worst <= Y_RTOL
+
+
 def test_linear_batched_more_than_one_launch():
     """More linears than one streaming launch takes (STREAM_BATCH), mixed K
     and ragged N, at 3 tokens: every result meets the bound."""
@@ -426,11 +448,13 @@ def test_linear_batched_more_than_one_launch():
 
 
 @pytest.mark.parametrize("kernel", ["auto", "stream", "tiled"])
-@pytest.mark.parametrize("m", [1, 5, 8, 16, 40])
+@pytest.mark.parametrize("m", [1, 5, 8, 16, 40, 200])
 @pytest.mark.parametrize("sym", [False, True])
 def test_linear_batched_qwen_block(m, sym, kernel):
     if kernel == "stream" and m > 8:
         pytest.skip("the streaming decode kernel takes at most 8 tokens")
+    if kernel == "tiled" and m > 64:
+        pytest.skip("the tensor-map decode kernel takes at most 64 tokens")
     shapes = [(n, k) for _, k, n in synth.QWEN3_1P7B_BLOCK] + [(72, 640)]
     items, refs = [], []
     for i, (n, k) in enumerate(shapes):

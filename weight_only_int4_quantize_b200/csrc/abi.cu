@@ -342,16 +342,17 @@ w4_status w4a16_linear_batched(const w4_linear_item* items, int count, int64_t M
   const bool pdl = (flags & W4_LINEAR_PDL) != 0;
   const bool stat = (flags & W4_LINEAR_STATIC_WEIGHTS) != 0;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (M > 64) {  // prefill: one tcgen05 GEMM per linear
+  if (M > 64) {  // prefill: grouped tcgen05 launches (up to 16 linears each)
+    if ((M + 127) / 128 > 65535) return W4_ERR_UNSUPPORTED;
+    std::vector<PrefillItem> pi(count);
     for (int i = 0; i < count; ++i) {
       const w4_linear_item& it = items[i];
-      st = cuda_status(launch_prefill_gemm(it.x_bf16, static_cast<int>(M), it.qweight,
-                                           it.scales_f16, it.zeros_f16, static_cast<int>(it.N),
-                                           static_cast<int>(it.K), it.y_bf16, pdl, stat, s, err),
-                       "prefill tcgen05 GEMM launch");
-      if (st != W4_OK) return st;
+      pi[i] = PrefillItem{it.x_bf16, it.qweight, it.scales_f16, it.zeros_f16, it.y_bf16,
+                          static_cast<int>(it.N), static_cast<int>(it.K)};
     }
-    return W4_OK;
+    return cuda_status(launch_prefill_gemm_group(pi.data(), count, static_cast<int>(M), pdl,
+                                                 stat, s, err),
+                       "grouped prefill tcgen05 GEMM launch");
   }
   std::vector<int> order(count);
   for (int i = 0; i < count; ++i) order[i] = i;

@@ -25,6 +25,8 @@
 // and returns.  No TMA multicast.
 #include <cudaTypedefs.h>
 
+#include <cmath>
+
 #include "w4_common.cuh"
 #include "w4_kernels.h"
 
@@ -79,6 +81,22 @@ struct SumSqArgs {
   int n_seg;
   int seg_off[17];      // column (N) boundaries, multiples of 16 inside
   int tiles;            // m_tiles * n_tiles
+};
+
+// A prefill launch decodes a group of linears that share the token count:
+// CTA tiles of linear i are [tile_start[i], tile_start[i + 1]) of the 1-D
+// grid, n-tile fastest (consecutive CTAs share their x tile).
+constexpr int kGemmGroup = 16;
+struct GemmGroup {
+  CUtensorMap ta[kGemmGroup];  // x of each linear, bf16 [M, K], box 64 x (MT x 128)
+  const uint32_t* qw[kGemmGroup];
+  const uint16_t* scales[kGemmGroup];
+  const uint16_t* zeros[kGemmGroup];
+  __nv_bfloat16* y[kGemmGroup];
+  int N[kGemmGroup];
+  int K[kGemmGroup];
+  int tile_start[kGemmGroup + 1];
+  int count;
 };
 
 __device__ __forceinline__ void tma_load_3d(uint32_t smem_dst, const CUtensorMap* map, int c0,
@@ -150,13 +168,11 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v) {
 
 template <int BSRC, int EPI, bool SYM, int MT, int NB>
 __global__ void __launch_bounds__(kThreads, 1)
-    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_a,
-                   const __grid_constant__ CUtensorMap tmap_b,  // kBTma only
-                   const uint32_t* __restrict__ qw, const uint16_t* __restrict__ scales,
-                   const uint16_t* __restrict__ zeros,          // kBDequant only
-                   __nv_bfloat16* __restrict__ y,               // kEpiStoreBf16 only
-                   const __grid_constant__ SumSqArgs ss,        // kEpiSumSquares only
-                   int M, int N, int K, int pdl_static, unsigned* err) {
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_a,    // kBTma only
+                   const __grid_constant__ CUtensorMap tmap_b,    // kBTma only
+                   const __grid_constant__ GemmGroup grp,         // kBDequant only
+                   const __grid_constant__ SumSqArgs ss,          // sum-of-squares epilogues
+                   int M, int N_arg, int K_arg, int pdl_static, unsigned* err) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   const uint32_t base = (raw_addr + 1023u) & ~1023u;
@@ -181,8 +197,35 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int n0 = blockIdx.x * NB;
-  const int m0 = blockIdx.y * (MT * BM);
+  // This CTA's operands: the scoring GEMMs take one A and a candidate-indexed
+  // B; a prefill CTA finds its linear in the group and its tile in it.
+  const CUtensorMap* ta = &tmap_a;
+  const uint32_t* __restrict__ qw = nullptr;
+  const uint16_t* __restrict__ scales = nullptr;
+  const uint16_t* __restrict__ zeros = nullptr;
+  __nv_bfloat16* __restrict__ y = nullptr;
+  int N = N_arg, K = K_arg;
+  int tile_n = blockIdx.x, tile_m = blockIdx.y;
+  if constexpr (BSRC == kBDequant) {
+    int lo = 0, hi = grp.count - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (grp.tile_start[mid] <= static_cast<int>(blockIdx.x)) lo = mid; else hi = mid - 1;
+    }
+    ta = &grp.ta[lo];
+    qw = grp.qw[lo];
+    scales = grp.scales[lo];
+    zeros = grp.zeros[lo];
+    y = grp.y[lo];
+    N = grp.N[lo];
+    K = grp.K[lo];
+    const int local = static_cast<int>(blockIdx.x) - grp.tile_start[lo];
+    const int n_tiles = (N + NB - 1) / NB;
+    tile_n = local % n_tiles;
+    tile_m = local / n_tiles;
+  }
+  const int n0 = tile_n * NB;
+  const int m0 = tile_m * (MT * BM);
   const int cand = blockIdx.z;
   const int num_kb = K / BK;
 
@@ -198,7 +241,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
-    tma_prefetch_desc(&tmap_a);
+    tma_prefetch_desc(ta);
     if (BSRC == kBTma) tma_prefetch_desc(&tmap_b);
   }
   if (warp == 1) {
@@ -221,11 +264,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!mbar_wait(empty(s), ph ^ 1u, abort_flag, err, kKernelIdGemm)) break;
         if (BSRC == kBTma) {
           mbar_arrive_expect_tx(full_a(s), kTileABytes + kTileBBytes);
-          tma_load_2d(sA + s * kTileABytes, &tmap_a, kb * BK, m0, full_a(s));
+          tma_load_2d(sA + s * kTileABytes, ta, kb * BK, m0, full_a(s));
           tma_load_3d(sB + s * kTileBBytes, &tmap_b, kb * BK, n0, cand, full_a(s));
         } else {
           mbar_arrive_expect_tx(full_a(s), kTileABytes);
-          tma_load_2d(sA + s * kTileABytes, &tmap_a, kb * BK, m0, full_a(s));
+          tma_load_2d(sA + s * kTileABytes, ta, kb * BK, m0, full_a(s));
         }
         kb_stop = kb + 1;
       }
@@ -523,12 +566,13 @@ CUresult encode_tmap(CUtensorMap* map, CUtensorMapDataType dt, int rank, const u
 
 // One instantiation per kernel (the cache below must be per kernel, and
 // every instantiation of gemm_tc_kernel has the same function type).
+// The scoring GEMMs carry no group.
+const GemmGroup kNoGroup = {};
+
 template <auto kern, size_t kSmemBytes>
-cudaError_t launch_gemm(dim3 grid, bool pdl, cudaStream_t stream,
-                        const CUtensorMap& ta, const CUtensorMap& tb, const uint32_t* qw,
-                        const uint16_t* sc, const uint16_t* z, __nv_bfloat16* y,
-                        const SumSqArgs& ss, int M, int N, int K, int pdl_static,
-                        unsigned* err) {
+cudaError_t launch_gemm(dim3 grid, bool pdl, cudaStream_t stream, const CUtensorMap& ta,
+                        const CUtensorMap& tb, const GemmGroup& grp, const SumSqArgs& ss, int M,
+                        int N, int K, int pdl_static, unsigned* err) {
   // The opt-in shared-memory size is a per-device function attribute; set it
   // once per device and kernel instantiation.
   static unsigned long long attr_done = 0;  // bit d: device d
@@ -553,68 +597,105 @@ cudaError_t launch_gemm(dim3 grid, bool pdl, cudaStream_t stream,
     cfg.attrs = attr;
     cfg.numAttrs = 1;
   }
-  return cudaLaunchKernelEx(&cfg, kern, ta, tb, qw, sc, z, y, ss, M, N, K, pdl_static, err);
+  return cudaLaunchKernelEx(&cfg, kern, ta, tb, grp, ss, M, N, K, pdl_static, err);
 }
 
 }  // namespace
 
-cudaError_t launch_prefill_gemm(const void* x, int M, const int32_t* qw, const uint16_t* sc,
-                                const uint16_t* z, int N, int K, void* y, bool pdl,
-                                bool static_w, cudaStream_t stream, unsigned* err) {
+cudaError_t launch_prefill_gemm_group(const PrefillItem* items_in, int count, int M,
+                                      bool pdl, bool static_w, cudaStream_t stream,
+                                      unsigned* err) {
+  if (count < 1) return cudaSuccess;
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess)
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  // Tile shape (MT x 128 rows, NB columns), one CTA per SM.  Measured time of
-  // one wave of CTAs relative to 128 x 256 tiles (same K): 256 x 256 1.32,
-  // 128 x 256 1.00, 256 x 128 0.80, 128 x 128 0.68 -- the B dequantization
-  // scales with NB and the MMAs with MT x NB.  The shape with the smallest
-  // waves x wave time wins; on equal cost the earlier (larger) one.
-  struct Shape { int mt, nb, cost; };
-  const Shape shapes[4] = {{2, 256, 132}, {1, 256, 100}, {2, 128, 80}, {1, 128, 68}};
-  int best = -1;
-  long best_cost = 0;
-  for (int i = 0; i < 4; ++i) {
-    const Shape sh = shapes[i];
-    if (sh.mt == 2 && M < 2 * BM) continue;  // 256-row tiles only when rows fill them
-    const long tiles = static_cast<long>((N + sh.nb - 1) / sh.nb) *
-                       ((M + sh.mt * BM - 1) / (sh.mt * BM));
-    const long cost = ((tiles + sms - 1) / sms) * sh.cost;
-#ifdef W4_GEMM_FORCE_SHAPE
-    if (i != W4_GEMM_FORCE_SHAPE) continue;
-#endif
-    if (best < 0 || cost < best_cost) {
-      best = i;
-      best_cost = cost;
+  // Longest K first: the long CTAs start first and the short ones fill in.
+  PrefillItem items[kGemmGroup];
+  for (int i0 = 0; i0 < count; i0 += kGemmGroup) {
+    const int n = count - i0 < kGemmGroup ? count - i0 : kGemmGroup;
+    for (int i = 0; i < n; ++i) items[i] = items_in[i0 + i];
+    for (int i = 1; i < n; ++i)
+      for (int j = i; j > 0 && items[j].K > items[j - 1].K; --j) {
+        const PrefillItem t = items[j];
+        items[j] = items[j - 1];
+        items[j - 1] = t;
+      }
+    const bool sym = items[0].z == nullptr;
+    // Tile shape (MT x 128 rows, NB columns), one CTA per SM.  Measured time
+    // of one wave of CTAs relative to 128 x 256 tiles (same K): 256 x 256
+    // 1.32, 128 x 256 1.00, 256 x 128 0.80, 128 x 128 0.68 -- the B
+    // dequantization scales with NB and the MMAs with MT x NB.  The group's
+    // tiles count in units of its longest K; the shape with the smallest
+    // waves x wave time wins, on equal cost the earlier (larger) one.
+    struct Shape { int mt, nb, cost; };
+    const Shape shapes[4] = {{2, 256, 132}, {1, 256, 100}, {2, 128, 80}, {1, 128, 68}};
+    const int k_max = items[0].K;
+    int best = -1;
+    long best_cost = 0;
+    for (int si = 0; si < 4; ++si) {
+      const Shape sh = shapes[si];
+      if (sh.mt == 2 && M < 2 * BM) continue;  // 256-row tiles only when rows fill them
+      double eq = 0.0;  // tiles of the longest K
+      for (int i = 0; i < n; ++i)
+        eq += static_cast<double>((items[i].N + sh.nb - 1) / sh.nb) *
+              ((M + sh.mt * BM - 1) / (sh.mt * BM)) * items[i].K / k_max;
+      const long cost = static_cast<long>(std::ceil(eq / sms - 1e-9)) * sh.cost;
+      if (best < 0 || cost < best_cost) {
+        best = si;
+        best_cost = cost;
+      }
     }
-  }
-  if (best < 0) best = 1;
-  const int mt = shapes[best].mt, nb = shapes[best].nb;
-  const int bm = mt * BM;
-  CUtensorMap ta, tb;
-  const uint64_t dims[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(M)};
-  const uint64_t str[1] = {static_cast<uint64_t>(K) * 2};
-  const uint32_t box[2] = {BK, static_cast<uint32_t>(bm)};
-  if (encode_tmap(&ta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, dims, str, box, x) != CUDA_SUCCESS)
-    return cudaErrorInvalidValue;
-  tb = ta;  // unused by the dequant variant
-  SumSqArgs ss = {};
-  dim3 grid((N + nb - 1) / nb, (M + bm - 1) / bm, 1);
-  const uint32_t* q = reinterpret_cast<const uint32_t*>(qw);
-  __nv_bfloat16* yp = static_cast<__nv_bfloat16*>(y);
-  const int ps = (pdl && static_w) ? 1 : 0;
-#define W4_PREFILL_LAUNCH(MT_, NB_)                                                          \
-  (z == nullptr                                                                            \
-       ? launch_gemm<gemm_tc_kernel<kBDequant, kEpiStoreBf16, true, MT_, NB_>,              \
-                     SmemLayout<MT_, NB_>::bytes>(grid, pdl, stream, ta, tb, q, sc, z, yp, ss, \
-                                                  M, N, K, ps, err)                         \
-       : launch_gemm<gemm_tc_kernel<kBDequant, kEpiStoreBf16, false, MT_, NB_>,             \
-                     SmemLayout<MT_, NB_>::bytes>(grid, pdl, stream, ta, tb, q, sc, z, yp, ss, \
-                                                  M, N, K, ps, err))
-  if (mt == 2 && nb == 256) return W4_PREFILL_LAUNCH(2, 256);
-  if (mt == 2) return W4_PREFILL_LAUNCH(2, 128);
-  if (nb == 256) return W4_PREFILL_LAUNCH(1, 256);
-  return W4_PREFILL_LAUNCH(1, 128);
+    if (best < 0) best = 1;
+    const int mt = shapes[best].mt, nb = shapes[best].nb;
+    const int bm = mt * BM;
+    GemmGroup grp;
+    grp.count = n;
+    grp.tile_start[0] = 0;
+    for (int i = 0; i < n; ++i) {
+      const PrefillItem& it = items[i];
+      const uint64_t dims[2] = {static_cast<uint64_t>(it.K), static_cast<uint64_t>(M)};
+      const uint64_t str[1] = {static_cast<uint64_t>(it.K) * 2};
+      const uint32_t box[2] = {BK, static_cast<uint32_t>(bm)};
+      if (encode_tmap(&grp.ta[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, dims, str, box, it.x) !=
+          CUDA_SUCCESS)
+        return cudaErrorInvalidValue;
+      grp.qw[i] = reinterpret_cast<const uint32_t*>(it.qw);
+      grp.scales[i] = it.sc;
+      grp.zeros[i] = it.z;
+      grp.y[i] = static_cast<__nv_bfloat16*>(it.y);
+      grp.N[i] = it.N;
+      grp.K[i] = it.K;
+      const long tiles = static_cast<long>((it.N + nb - 1) / nb) * ((M + bm - 1) / bm);
+      if (grp.tile_start[i] + tiles > 0x7FFFFFFFL) return cudaErrorInvalidValue;
+      grp.tile_start[i + 1] = grp.tile_start[i] + static_cast<int>(tiles);
+    }
+    CUtensorMap none = grp.ta[0];  // unused by the dequantizing variant
+    SumSqArgs ss = {};
+    dim3 grid(grp.tile_start[n], 1, 1);
+    const int ps = (pdl && static_w) ? 1 : 0;
+    cudaError_t e;
+#define W4_PREFILL_LAUNCH(MT_, NB_)                                                           \
+  (sym ? launch_gemm<gemm_tc_kernel<kBDequant, kEpiStoreBf16, true, MT_, NB_>,                \
+                     SmemLayout<MT_, NB_>::bytes>(grid, pdl, stream, none, none, grp, ss, M, 0, \
+                                                  0, ps, err)                                 \
+       : launch_gemm<gemm_tc_kernel<kBDequant, kEpiStoreBf16, false, MT_, NB_>,               \
+                     SmemLayout<MT_, NB_>::bytes>(grid, pdl, stream, none, none, grp, ss, M, 0, \
+                                                  0, ps, err))
+    if (mt == 2 && nb == 256) e = W4_PREFILL_LAUNCH(2, 256);
+    else if (mt == 2) e = W4_PREFILL_LAUNCH(2, 128);
+    else if (nb == 256) e = W4_PREFILL_LAUNCH(1, 256);
+    else e = W4_PREFILL_LAUNCH(1, 128);
 #undef W4_PREFILL_LAUNCH
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+cudaError_t launch_prefill_gemm(const void* x, int M, const int32_t* qw, const uint16_t* sc,
+                                const uint16_t* z, int N, int K, void* y, bool pdl,
+                                bool static_w, cudaStream_t stream, unsigned* err) {
+  const PrefillItem it{x, qw, sc, z, y, N, K};
+  return launch_prefill_gemm_group(&it, 1, M, pdl, static_w, stream, err);
 }
 
 // Row tiles of the sum-of-squares GEMM: 256 rows (two UMMAs per k-step
@@ -645,10 +726,10 @@ cudaError_t launch_sumsq_gemm(const void* a_f16, int M, const void* b_f16, int N
   ss.tiles = grid.x * grid.y;
   if (mt == 2)
     return launch_gemm<gemm_tc_kernel<kBTma, kEpiSumSquares, false, 2, BN>,
-                       SmemLayout<2, BN>::bytes>(grid, false, stream, ta, tb, nullptr, nullptr,
-                                                 nullptr, nullptr, ss, M, N, K, 0, err);
+                       SmemLayout<2, BN>::bytes>(grid, false, stream, ta, tb, kNoGroup, ss, M, N,
+                                                 K, 0, err);
   return launch_gemm<gemm_tc_kernel<kBTma, kEpiSumSquares, false, 1, BN>, SmemLayout<1, BN>::bytes>(
-      grid, false, stream, ta, tb, nullptr, nullptr, nullptr, nullptr, ss, M, N, K, 0, err);
+      grid, false, stream, ta, tb, kNoGroup, ss, M, N, K, 0, err);
 }
 
 cudaError_t launch_colsumsq_gemm(const void* a_f16, int M, const void* b_f16, int N, int K,
@@ -673,11 +754,11 @@ cudaError_t launch_colsumsq_gemm(const void* a_f16, int M, const void* b_f16, in
   ss.tiles = grid.x * grid.y;
   if (mt == 2)
     return launch_gemm<gemm_tc_kernel<kBTma, kEpiColSumSquares, false, 2, BN>,
-                       SmemLayout<2, BN>::bytes>(grid, false, stream, ta, tb, nullptr, nullptr,
-                                                 nullptr, nullptr, ss, M, N, K, 0, err);
+                       SmemLayout<2, BN>::bytes>(grid, false, stream, ta, tb, kNoGroup, ss, M, N,
+                                                 K, 0, err);
   return launch_gemm<gemm_tc_kernel<kBTma, kEpiColSumSquares, false, 1, BN>,
-                     SmemLayout<1, BN>::bytes>(grid, false, stream, ta, tb, nullptr, nullptr,
-                                               nullptr, nullptr, ss, M, N, K, 0, err);
+                     SmemLayout<1, BN>::bytes>(grid, false, stream, ta, tb, kNoGroup, ss, M, N,
+                                               K, 0, err);
 }
 
 int colsumsq_row_tiles(int M) { return (M + sumsq_mt(M) * BM - 1) / (sumsq_mt(M) * BM); }

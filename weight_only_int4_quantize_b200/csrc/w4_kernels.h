@@ -88,6 +88,18 @@ cudaError_t plan_gemv_stream(StreamBatch& b, bool symmetric, int num_sms, int* b
 cudaError_t launch_gemv_stream(StreamBatch& b, bool symmetric, bool pdl, bool static_w,
                                cudaStream_t stream, int num_sms);
 
+// One linear of a grouped prefill launch (all share M).
+struct PrefillItem {
+  const void* x;       // bf16 [M, K]
+  const int32_t* qw;   // packed [N, K/8]
+  const uint16_t* sc;  // fp16 [N, K/128]
+  const uint16_t* z;   // fp16 [N, K/128]; NULL: symmetric (the same for all items)
+  void* y;             // bf16 [M, N]
+  int N, K;
+};
+// Up to 16 linears per tcgen05 launch (more in further launches).
+cudaError_t launch_prefill_gemm_group(const PrefillItem* items, int count, int M, bool pdl,
+                                      bool static_w, cudaStream_t stream, unsigned* err);
 cudaError_t launch_prefill_gemm(const void* x, int M, const int32_t* qw, const uint16_t* sc,
                                 const uint16_t* z, int N, int K, void* y, bool pdl,
                                 bool static_w, cudaStream_t stream, unsigned* err);
