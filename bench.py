@@ -56,6 +56,7 @@ TRAFFIC_CAPTURES = {
     # quantize 17408 x 5120: 202.47 MB over 225.67 MB (part of the written codes
     # is still in the write-back L2 when the kernel ends)
     "quantize_pack": {"source": "quantize.cu", "digest": "f3061dcc5ac9fd85", "ratio": 202.47 / 225.67},
+}
 
 # --------------------------------------------------------------------------
 
