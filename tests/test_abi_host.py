@@ -137,3 +137,11 @@ def test_clip_rows_validation(L):
     assert q(A, 4, 128, 128, 0, None, A + 2, A, A, A, None) == 3                      # misaligned
     assert q(A, 4, 128, 128, 1, None, A, A, A, A, None) == 1                          # sym + zeros
     assert q(A, 4, 128, 64, 0, None, A, A, A, A, None) == 4                           # group
+
+
+def test_bench_and_entry_scripts_compile():
+    """The driver runs these files directly: they must at least compile."""
+    import py_compile
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    for name in ("bench.py", "__graft_entry__.py"):
+        py_compile.compile(os.path.join(root, name), doraise=True)
