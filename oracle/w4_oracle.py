@@ -25,6 +25,10 @@ Sources (model-card pages; cited by page title and section):
       (int4, group size 128, symmetric, weight-only, activations 16-bit).
   [awq-ppl] "AWQ INT4-g128 WikiText-2 perplexity delta vs fp16, Llama-2 7B",
       'Methodology' (group size 128; grid size 20 for the alpha search).
+  [qsrt] "malaiwah/GLM-5.2-QSRT-Fruit-Instruct" card: 'What is included'
+      (W4A8 decode execution), the storage paragraph (W4A8 and W4A16 use
+      the same stored weights) and the runtime paragraph (W4A8 for
+      decode-sized batches of at most 16 rows).
   [rebuttal-cmp] the same "ghostchoir/rebuttal_w4g128_awq_w2" card, the
       'Comparability caveat' under the perplexity table (the d=0 arm uses
       stock AWQ's per-output-channel clipping search).
@@ -47,7 +51,11 @@ design notes):
   * stock per-output-channel clipping: every output row takes its own ratio
     from the same shrink grid, the one with the least output error of that
     row, ||x E_n^T||^2 (the linear's output error is a sum over rows, so the
-    per-row choices minimise it jointly); ties go to the lowest grid index.
+    per-row choices minimise it jointly); ties go to the lowest grid index;
+  * W4A8 activations ([qsrt] fixes no format): per token row, symmetric
+    int8, scale = max_k |x_mk| / 127 in binary32, code = clamp(rint(x /
+    scale), -127, 127) with IEEE division and ties to even; a row of zeros
+    has scale 0 and codes 0.
 """
 from __future__ import annotations
 
@@ -373,6 +381,40 @@ def quantize_pack_rows(w_bits, symmetric, awq_s, shrink_rows, group=GROUP):
     codes, s16, z16 = quantize_rtn(w_bits, symmetric, awq_s,
                                    np.asarray(shrink_rows, dtype=np.float32), group)
     return pack_codes(codes), s16, z16
+
+
+# ----------------------------------------------------------------------------
+# W4A8 decode: the same stored int4 weights against int8 activations ([qsrt]).
+# ----------------------------------------------------------------------------
+
+
+def quantize_act_int8(x_bits: np.ndarray):
+    """Per-token symmetric int8 activations.  Returns (codes int8 [M, K],
+    scale float32 [M]); x ~ codes * scale per row."""
+    x = bf16_bits_to_f32(x_bits)
+    amax = np.max(np.abs(x), axis=1)
+    scale = (amax / np.float32(127.0)).astype(np.float32)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        t = np.rint(x / scale[:, None])
+    t = np.where(scale[:, None] > 0, t, 0.0)
+    return np.clip(t, -127, 127).astype(np.int8), scale
+
+
+def w4a8_linear(xq: np.ndarray, xscale: np.ndarray, codes: np.ndarray, scale16: np.ndarray,
+                zero16: np.ndarray | None, group: int = GROUP) -> np.ndarray:
+    """y[m, n] = xscale_m * sum_g scale_ng * D[m, n, g], where the group dot
+    D = sum_{k in g} (q_nk - z_ng) * xq_mk is an exact integer; the scaling
+    and the sum over groups in binary64."""
+    n, k = codes.shape
+    g = k // group
+    z = (np.full((n, g), 8, dtype=np.int64) if zero16 is None
+         else f16_bits_to_f32(zero16).astype(np.int64))
+    w = codes.astype(np.int64).reshape(n, g, group) - z[:, :, None]
+    xg = np.asarray(xq, dtype=np.int64).reshape(xq.shape[0], g, group)
+    d = np.einsum("mgk,ngk->mng", xg, w)  # exact integers
+    sc = f16_bits_to_f32(scale16).astype(np.float64)
+    return np.asarray(xscale, dtype=np.float64)[:, None] * np.einsum("mng,ng->mn",
+                                                                     d.astype(np.float64), sc)
 
 
 # ----------------------------------------------------------------------------

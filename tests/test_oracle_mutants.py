@@ -38,6 +38,13 @@ MUTANTS = [
      "sse[j] = np.sum(y * y, axis=0)[::-1]"),
     ("per-row choice takes the last minimum", "return sse, np.argmin(sse, axis=0)",
      "return sse, len(shrinks) - 1 - np.argmin(sse[::-1], axis=0)"),
+    ("activation scale over 128", "scale = (amax / np.float32(127.0))", "scale = (amax / np.float32(128.0))"),
+    ("activation codes rounded away from zero", "t = np.rint(x / scale[:, None])",
+     "t = np.trunc(x / scale[:, None] + np.copysign(0.5, x))"),
+    ("W4A8 zero point dropped", "w = codes.astype(np.int64).reshape(n, g, group) - z[:, :, None]",
+     "w = codes.astype(np.int64).reshape(n, g, group)"),
+    ("W4A8 activation scale dropped", "return np.asarray(xscale, dtype=np.float64)[:, None] * np.einsum",
+     "return np.ones_like(np.asarray(xscale, dtype=np.float64))[:, None] * np.einsum"),
     ("per-row ratios applied to the wrong rows",
      "np.asarray(shrink, dtype=np.float32).reshape(n, 1)",
      "np.asarray(shrink, dtype=np.float32)[::-1].reshape(n, 1)"),
@@ -69,6 +76,10 @@ def _all_pins():
         yield P.test_clip_rows_sse_brute_force_tiny, (sym,)
         yield P.test_quantize_rows_reduces_to_per_linear_quantize, (sym,)
     yield P.test_clip_rows_ties_take_the_lowest_index, ()
+    yield P.test_act_int8_brute_force, ()
+    yield P.test_act_int8_ties_to_even_hand_case, ()
+    for sym in (False, True):
+        yield P.test_w4a8_linear_exact_rational_small, (sym,)
 
 
 @pytest.mark.parametrize("name,old,new", MUTANTS, ids=[m[0] for m in MUTANTS])

@@ -450,3 +450,76 @@ def test_quantize_rows_reduces_to_per_linear_quantize(sym):
         assert np.array_equal(mixed[0][n:n + 1], one[0]) and np.array_equal(mixed[1][n:n + 1], one[1])
         if not sym:
             assert np.array_equal(mixed[2][n:n + 1], one[2])
+
+
+# ------------------------------------------------------------- W4A8 -----
+
+def test_act_int8_brute_force():
+    """Every code is the integer nearest x / scale (exact rationals; the
+    binary32 quotient may sit a hair across a half), the row's largest
+    magnitude maps to +-127, and a zero row stays zero."""
+    x = synth.bits(synth.student_t_calibration(4, 256, seed=91))
+    x[2] = 0
+    q, sc = O.quantize_act_int8(x)
+    xf = O.bf16_bits_to_f32(x)
+    for m in range(4):
+        amax = max(abs(Fraction(float(v))) for v in xf[m])
+        if amax == 0:
+            assert sc[m] == 0 and np.all(q[m] == 0)
+            continue
+        assert sc[m] == np.float32(float(amax)) / np.float32(127.0)
+        s = Fraction(float(sc[m]))
+        for k in range(256):
+            r = Fraction(float(xf[m, k])) / s
+            assert abs(r - int(q[m, k])) <= Fraction(1, 2) + Fraction(1, 1 << 20)
+            assert -127 <= int(q[m, k]) <= 127
+        j = int(np.argmax(np.abs(xf[m])))
+        assert abs(int(q[m, j])) == 127
+
+
+@pytest.mark.parametrize("sym", [False, True])
+def test_w4a8_linear_exact_rational_small(sym):
+    x = synth.bits(synth.normal_activations(3, 256, seed=92))
+    w = synth.bits(synth.normal_weight(5, 256, 0.02, seed=93, n_outliers=2, outlier_scale=20.0))
+    q, xs = O.quantize_act_int8(x)
+    codes, s16, z16 = O.quantize_rtn(w, sym)
+    y = O.w4a8_linear(q, xs, codes, s16, z16)
+    sc = O.f16_bits_to_f32(s16)
+    z = np.full(sc.shape, 8.0) if z16 is None else O.f16_bits_to_f32(z16)
+    for m in range(3):
+        for n in range(5):
+            tot = Fraction(0)
+            for k in range(256):
+                g = k // 128
+                tot += (Fraction(int(codes[n, k])) - Fraction(float(z[n, g]))) * \
+                    Fraction(float(sc[n, g])) * int(q[m, k])
+            ex = tot * Fraction(float(xs[m]))
+            assert abs(y[m, n] - float(ex)) <= 1e-12 * abs(float(ex)) + 1e-300
+
+
+def test_w4a8_is_w4a16_on_the_quantized_activation():
+    """y_a16 - y_a8 = w_hat . (x - q * scale): the W4A8 result is the W4A16
+    linear of the dequantized activation (exact identity)."""
+    x = synth.bits(synth.normal_activations(4, 384, seed=94))
+    w = synth.bits(synth.normal_weight(7, 384, 0.02, seed=95))
+    q, xs = O.quantize_act_int8(x)
+    codes, s16, z16 = O.quantize_rtn(w, False)
+    what = O.dequantize(codes, s16, z16).astype(np.float64)
+    y8 = O.w4a8_linear(q, xs, codes, s16, z16)
+    xd = q.astype(np.float64) * xs.astype(np.float64)[:, None]
+    assert np.allclose(y8, xd @ what.T, rtol=1e-12, atol=1e-300)
+    y16 = O.linear(x, what)
+    err = O.bf16_bits_to_f32(x).astype(np.float64) - xd
+    bound = np.abs(err) @ np.abs(what).T
+    assert np.all(np.abs(y16 - y8) <= bound * (1 + 1e-9) + 1e-300)
+
+
+def test_act_int8_ties_to_even_hand_case():
+    """max |x| = 127 gives scale 1.0 exactly, so halves are exact ties; the
+    codes follow round-half-to-even: 0.5 -> 0, 1.5 -> 2, 2.5 -> 2, -2.5 -> -2,
+    3.5 -> 4 (hand-derived)."""
+    vals = np.array([[127.0, 0.5, 1.5, 2.5, -0.5, -2.5, 3.5, -127.0] + [0.0] * 120],
+                    np.float32)
+    q, sc = O.quantize_act_int8(f32_bits_to_bf16_exact(vals))
+    assert sc[0] == np.float32(1.0)
+    assert q[0, :8].tolist() == [127, 0, 2, 2, 0, -2, 4, -127]
