@@ -202,6 +202,55 @@ w4_status w4a16_linear_batched(const w4_linear_item* items, int count, int64_t M
                                unsigned flags, void* stream);
 
 /*
+ * W4A8 decode -- the same stored int4 weights against int8 activations
+ * ([qsrt] 'What is included': W4A8 decode execution; the storage paragraph:
+ * W4A8 and W4A16 use the same stored weights; the runtime paragraph: W4A8
+ * for decode-sized batches of at most 16 rows).  The pages fix no
+ * activation format; this library quantizes per token, symmetric:
+ *
+ *   xscale[m] = max_k |x_mk| / 127               (binary32)
+ *   xq[m, k]  = clamp(rint(x_mk / xscale[m]), -127, 127)
+ *               (IEEE division, ties to even; a zero row has scale 0, codes 0)
+ *   xsum[m, g] = sum_{k in group g} xq[m, k]      (int32)
+ *   y[m, n] = xscale[m] * sum_g scale[n, g] * sum_{k in g} (q[n, k] - z[n, g]) * xq[m, k]
+ *
+ * The group sums are exact integers (int8 x int4 tensor-core products with
+ * int32 accumulation); the scaling and the sum over groups run in binary32
+ * and y is rounded once to bf16.
+ *
+ * w4_quantize_act_int8 -- x_bf16 device bf16 [M, K] (K % 128 == 0) ->
+ *   xq_out int8 [M, K] (in every 8-channel chunk the channels are stored in
+ *   the order 0, 4, 1, 5, 2, 6, 3, 7, the order in which the nibble masks of
+ *   a packed weight word deliver its codes), xsum_out int32 [M, K/128],
+ *   xscale_out float32 [M].  All device, 16-byte aligned.  One quantization
+ *   serves every linear that reads the same x (q, k, v; gate, up).
+ * w4a8_linear -- y_bf16 [M, N] from those three arrays and a packed weight
+ *   (as for w4a16_linear), 1 <= M <= 16, K <= 81920; flags W4_LINEAR_PDL and
+ *   W4_LINEAR_STATIC_WEIGHTS only.  Runs the persistent streaming decode
+ *   kernel (8 tokens per launch).
+ * w4a8_linear_batched -- many such linears (host array of w4a8_item) sharing
+ *   M and the symmetry, up to 256 per launch.
+ */
+w4_status w4_quantize_act_int8(const void* x_bf16, int64_t M, int64_t K, int8_t* xq_out,
+                               int32_t* xsum_out, float* xscale_out, void* stream);
+w4_status w4a8_linear(const int8_t* xq, const int32_t* xsum, const float* xscale, int64_t M,
+                      const int32_t* qweight, const uint16_t* scales_f16,
+                      const uint16_t* zeros_f16, int64_t N, int64_t K, int group, void* y_bf16,
+                      unsigned flags, void* stream);
+typedef struct {
+  const int8_t* xq;            /* device, int8 [M, K] (w4_quantize_act_int8 layout) */
+  const int32_t* xsum;         /* device, int32 [M, K/128] */
+  const float* xscale;         /* device, float32 [M] */
+  const int32_t* qweight;      /* device, packed weight */
+  const uint16_t* scales_f16;
+  const uint16_t* zeros_f16;   /* NULL: symmetric */
+  int64_t N, K;
+  void* y_bf16;                /* device, bf16 [M, N] out */
+} w4a8_item;
+w4_status w4a8_linear_batched(const w4a8_item* items, int count, int64_t M, int group,
+                              unsigned flags, void* stream);
+
+/*
  * w4_awq_scales -- AWQ per-input-channel scales ([rebuttal] 'Search': AWQ
  * scale exponent grid; [awq-ppl] 'Methodology': grid of 20 alphas).
  *

@@ -145,3 +145,22 @@ def test_bench_and_entry_scripts_compile():
     root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
     for name in ("bench.py", "__graft_entry__.py"):
         py_compile.compile(os.path.join(root, name), doraise=True)
+
+
+def test_w4a8_validation(L):
+    import weight_only_int4_quantize_b200 as w4
+    q = L.w4_quantize_act_int8
+    assert q(None, 1, 128, A, A, A, None) == 1
+    assert q(A, 0, 128, A, A, A, None) == 2
+    assert q(A, 1, 100, A, A, A, None) == 2
+    assert q(A + 2, 1, 128, A, A, A, None) == 3
+    f = L.w4a8_linear
+    assert f(None, A, A, 1, A, A, None, 8, 128, 128, B, 0, None) == 1
+    assert f(A, A, A, 17, A, A, None, 8, 128, 128, B, 0, None) == 4      # > 16 rows
+    assert f(A, A, A, 1, A, A, None, 8, 128, 64, B, 0, None) == 4        # group
+    assert f(A, A, A, 1, A, A, None, 8, 128, 128, B, 0x1, None) == 1     # not a W4A8 flag
+    assert f(A, A, A, 1, A, A, None, 8, 130, 128, B, 0, None) == 2       # K % 128
+    assert f(A, A + 4, A, 1, A, A, None, 8, 128, 128, B, 0, None) == 3   # misaligned xsum
+    it = (w4.A8Item * 2)(w4.A8Item(A, A, A, A, A, None, 8, 128, B),
+                         w4.A8Item(A, A, A, A, A, A, 8, 128, B))
+    assert L.w4a8_linear_batched(it, 2, 1, 128, 0, None) == 1             # mixed symmetry

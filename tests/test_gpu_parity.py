@@ -363,6 +363,101 @@ def test_quantize_rows_uniform_equals_per_linear(sym):
         assert (u is None and v is None) or torch.equal(u, v)
 
 
+# ------------------------------------------------------------- W4A8 ----
+
+A8_PERM = (0, 4, 1, 5, 2, 6, 3, 7)  # stored order of the channels of a chunk
+
+
+def unpermute_act(xq):
+    """Channel order of w4_quantize_act_int8's codes back to natural order."""
+    m, k = xq.shape
+    out = np.empty_like(xq)
+    c = xq.reshape(m, k // 8, 8)
+    o = out.reshape(m, k // 8, 8)
+    for p, ch in enumerate(A8_PERM):
+        o[:, :, ch] = c[:, :, p]
+    return out
+
+
+def check_act_int8(x):
+    xq, xs, sc = w4.quantize_act_int8(x.to(DEV))
+    torch.cuda.synchronize()
+    q_ref, sc_ref = O.quantize_act_int8(synth.bits(x))
+    assert np.array_equal(sc.cpu().numpy().view(np.uint32), sc_ref.view(np.uint32))
+    q = unpermute_act(xq.cpu().numpy())
+    assert np.array_equal(q, q_ref)
+    m, k = q_ref.shape
+    assert np.array_equal(xs.cpu().numpy(), q_ref.astype(np.int64).reshape(m, k // 128, 128).sum(2))
+    return (xq, xs, sc), (q_ref, sc_ref)
+
+
+@pytest.mark.parametrize("m,k", [(1, 128), (5, 2048), (16, 6144), (3, 81920)])
+def test_act_int8_bit_exact(m, k):
+    x = synth.normal_activations(m, k, seed=90 + m)
+    if m > 2:
+        xb = x.clone()
+        xb[1] = 0  # a zero row: scale 0, codes 0
+        x = xb
+    check_act_int8(x)
+
+
+def w4a8_case(m, n, k, sym, seed, std=0.02, n_out=0, out_scale=1.0):
+    w = synth.normal_weight(n, k, std, seed=seed, n_outliers=n_out, outlier_scale=out_scale)
+    x = synth.normal_activations(m, k, seed=seed + 1)
+    (xq, xs, sc), (q_ref, sc_ref) = check_act_int8(x)
+    qw, s16, z16 = w4.quantize_pack(w.to(DEV), sym)
+    y = w4.w4a8_linear(xq, xs, sc, qw, s16, z16)
+    torch.cuda.synchronize()
+    oc, os_, oz = O.quantize_rtn(synth.bits(w), sym)
+    y_ref = O.w4a8_linear(q_ref, sc_ref, oc, os_, oz)
+    return y.float().cpu().numpy().astype(np.float64), y_ref
+
+
+# W4A8 bar: the group dots are exact on both sides; the GPU's binary32
+# scaling and group sum add a few ulps, and y is rounded once to bf16
+# (half an ulp, 2^-9 relative), so each element must lie within
+# 2^-8 |y_ref| + 1e-4 max|y_ref| of the binary64 oracle.
+def assert_w4a8_close(y, y_ref):
+    bound = 2.0 ** -8 * np.abs(y_ref) + 1e-4 * np.max(np.abs(y_ref))
+    assert np.all(np.abs(y - y_ref) <= bound), float(np.max(np.abs(y - y_ref) / bound))
+
+
+@pytest.mark.parametrize("m", [1, 3, 8, 9, 16])
+@pytest.mark.parametrize("sym", [False, True])
+def test_w4a8_linear_ragged(m, sym):
+    assert_w4a8_close(*w4a8_case(m, 1000, 1024, sym, seed=1100 + m))
+
+
+@pytest.mark.parametrize("k,n", [(5120, 17408), (17408, 5120)])
+@pytest.mark.parametrize("m", [1, 8])
+def test_w4a8_27b_shapes(k, n, m):
+    assert_w4a8_close(*w4a8_case(m, n, k, True, seed=1200 + n, std=0.015, n_out=k // 100,
+                                 out_scale=10.0))
+
+
+@pytest.mark.parametrize("m", [1, 4, 16])
+def test_w4a8_batched_qwen_block_shared_x(m):
+    """The seven Qwen linears, each input quantized once and shared where the
+    block shares it (q, k, v; gate, up), in one batched call."""
+    xs_by_k = {}
+    items, refs = [], []
+    for i, (_name, k, n) in enumerate(synth.QWEN3_1P7B_BLOCK):
+        if k not in xs_by_k:
+            x = synth.normal_activations(m, k, seed=1300 + k)
+            xs_by_k[k] = check_act_int8(x)
+        (xq, xsm, sc), (q_ref, sc_ref) = xs_by_k[k]
+        w = synth.normal_weight(n, k, 0.02, seed=1400 + i)
+        qw, s16, z16 = w4.quantize_pack(w.to(DEV), False)
+        y = torch.empty(m, n, dtype=torch.bfloat16, device=DEV)
+        items.append((xq, xsm, sc, qw, s16, z16, y))
+        oc, os_, oz = O.quantize_rtn(synth.bits(w), False)
+        refs.append(O.w4a8_linear(q_ref, sc_ref, oc, os_, oz))
+    w4.w4a8_linear_batched(items, m)
+    torch.cuda.synchronize()
+    for it, ref in zip(items, refs):
+        assert_w4a8_close(it[6].float().cpu().numpy().astype(np.float64), ref)
+
+
 # ------------------------------------------------------ failure path ----
 
 def test_bounded_wait_reports_and_context_survives():

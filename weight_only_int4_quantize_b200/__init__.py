@@ -17,6 +17,7 @@ from typing import Optional, Sequence
 __all__ = [
     "W4Error", "lib", "quantize_pack", "quantize_pack_batched", "quantize_pack_rows",
     "awq_clip_search_rows", "clip_rows_workspace_bytes", "w4a16_linear",
+    "quantize_act_int8", "w4a8_linear", "w4a8_linear_batched", "a8_items",
     "w4a16_linear_batched", "awq_scales", "awq_score_grid", "awq_score_grid_static_scratch",
     "awq_workspace_bytes", "device_error", "selftest_bounded_wait",
     "LINEAR_FORCE_GEMV", "LINEAR_FORCE_GEMM", "LINEAR_PDL", "LINEAR_STATIC_WEIGHTS",
@@ -96,6 +97,13 @@ def _declare(L: ctypes.CDLL) -> None:
     L.w4_quantize_pack_rows.restype = ctypes.c_int
     L.w4_quantize_pack_rows.argtypes = [_p, _i64, _i64, ctypes.c_int, ctypes.c_int, _p, _p, _p,
                                         _p, _p, _p]
+    L.w4_quantize_act_int8.restype = ctypes.c_int
+    L.w4_quantize_act_int8.argtypes = [_p, _i64, _i64, _p, _p, _p, _p]
+    L.w4a8_linear.restype = ctypes.c_int
+    L.w4a8_linear.argtypes = [_p, _p, _p, _i64, _p, _p, _p, _i64, _i64, ctypes.c_int, _p,
+                              ctypes.c_uint, _p]
+    L.w4a8_linear_batched.restype = ctypes.c_int
+    L.w4a8_linear_batched.argtypes = [_p, ctypes.c_int, _i64, ctypes.c_int, ctypes.c_uint, _p]
     L.w4_device_error.restype = ctypes.c_int
     L.w4_device_error.argtypes = [ctypes.c_int, _p]
     L.w4_selftest_bounded_wait.restype = ctypes.c_int
@@ -265,6 +273,71 @@ def w4a16_linear_batched(items, m: int, flags: int = 0, group: int = 128, stream
     st = lib().w4a16_linear_batched(ctypes.addressof(arr), len(arr), int(m), group, int(flags),
                                     stream if stream is not None else _stream(torch.cuda.current_device()))
     _check(st, "w4a16_linear_batched")
+
+
+def quantize_act_int8(x):
+    """Per-token int8 activations for W4A8: (xq int8 [M, K] in the library's
+    chunk channel order, xsum int32 [M, K/128], xscale float32 [M])."""
+    torch = _torch()
+    _cuda(x, torch.bfloat16, "x")
+    m, k = x.shape
+    xq = torch.empty((m, k), dtype=torch.int8, device=x.device)
+    xs = torch.empty((m, k // 128), dtype=torch.int32, device=x.device)
+    sc = torch.empty((m,), dtype=torch.float32, device=x.device)
+    with torch.cuda.device(x.device):
+        st = lib().w4_quantize_act_int8(x.data_ptr(), m, k, xq.data_ptr(), xs.data_ptr(),
+                                        sc.data_ptr(), _stream(x.device))
+    _check(st, "w4_quantize_act_int8")
+    return xq, xs, sc
+
+
+def w4a8_linear(xq, xsum, xscale, qweight, scales, zeros=None, flags: int = 0, group: int = 128,
+                out=None):
+    """y = W4A8 decode of int8 activations (from quantize_act_int8), bf16 [M, N]."""
+    torch = _torch()
+    _cuda(xq, torch.int8, "xq")
+    _cuda(xsum, torch.int32, "xsum")
+    _cuda(xscale, torch.float32, "xscale")
+    _cuda(qweight, torch.int32, "qweight")
+    _cuda(scales, torch.int16, "scales")
+    if zeros is not None:
+        _cuda(zeros, torch.int16, "zeros")
+    m, k = xq.shape
+    n = qweight.shape[0]
+    y = out if out is not None else torch.empty((m, n), dtype=torch.bfloat16, device=xq.device)
+    with torch.cuda.device(xq.device):
+        st = lib().w4a8_linear(xq.data_ptr(), xsum.data_ptr(), xscale.data_ptr(), m,
+                               qweight.data_ptr(), scales.data_ptr(),
+                               None if zeros is None else zeros.data_ptr(), n, k, group,
+                               y.data_ptr(), int(flags), _stream(xq.device))
+    _check(st, "w4a8_linear")
+    return y
+
+
+class A8Item(ctypes.Structure):
+    _fields_ = [("xq", ctypes.c_void_p), ("xsum", ctypes.c_void_p), ("xscale", ctypes.c_void_p),
+                ("qweight", ctypes.c_void_p), ("scales_f16", ctypes.c_void_p),
+                ("zeros_f16", ctypes.c_void_p), ("N", ctypes.c_int64), ("K", ctypes.c_int64),
+                ("y_bf16", ctypes.c_void_p)]
+
+
+def a8_items(items):
+    """Host array of w4a8_item from (xq, xsum, xscale, qweight, scales, zeros, y) tuples."""
+    arr = (A8Item * len(items))()
+    for i, (xq, xs, sc_x, qw, sc, zr, y) in enumerate(items):
+        arr[i] = A8Item(xq.data_ptr(), xs.data_ptr(), sc_x.data_ptr(), qw.data_ptr(),
+                        sc.data_ptr(), None if zr is None else zr.data_ptr(), qw.shape[0],
+                        xq.shape[1], y.data_ptr())
+    return arr
+
+
+def w4a8_linear_batched(items, m: int, flags: int = 0, group: int = 128, stream=None) -> None:
+    """Many independent W4A8 linears with the same token count m."""
+    torch = _torch()
+    arr = items if isinstance(items, ctypes.Array) else a8_items(items)
+    st = lib().w4a8_linear_batched(ctypes.addressof(arr), len(arr), int(m), group, int(flags),
+                                   stream if stream is not None else _stream(torch.cuda.current_device()))
+    _check(st, "w4a8_linear_batched")
 
 
 def awq_scales(x, alphas: Sequence[float]):

@@ -4,7 +4,7 @@ timing.  Inputs are seeded and generated on the device.
     python -m weight_only_int4_quantize_b200.cases quantize --n 17408 --k 5120 [--sym]
     python -m weight_only_int4_quantize_b200.cases linear --m 8 --n 17408 --k 5120 [--sym] [--gemm]
     python -m weight_only_int4_quantize_b200.cases awq --m 2048 --n 1024 --k 2048 --na 20 --nr 10
-    python -m weight_only_int4_quantize_b200.cases decode_batch --m 1 --blocks 4
+    python -m weight_only_int4_quantize_b200.cases decode_batch --m 1 --blocks 4 [--a8]
     python -m weight_only_int4_quantize_b200.cases clip_rows --m 2048 --n 6144 --k 2048 --nr 10
 
 Each case captures --iters launches in one CUDA graph (so host launch
@@ -75,6 +75,7 @@ def main():
     ap.add_argument("--iters", type=int, default=3)
     ap.add_argument("--pdl", action="store_true", help="programmatic dependent launch + static weights")
     ap.add_argument("--eager", action="store_true", help="time eager launches instead of a graph")
+    ap.add_argument("--a8", action="store_true", help="decode_batch: W4A8 (int8 activations)")
     a = ap.parse_args()
     w = _weights(a.n, a.k, 1)
     out = {"case": a.case, "m": a.m, "n": a.n, "k": a.k, "sym": a.sym}
@@ -111,10 +112,15 @@ def main():
                 y = torch.empty(a.m, n, dtype=torch.bfloat16, device="cuda")
                 items.append((x, qw, sc, zr, y))
                 byts += n * k * (0.5 + 4 / 128) + 2 * a.m * (k + n)
-        arr = w4.linear_items(items)
         flags = w4.LINEAR_PDL | w4.LINEAR_STATIC_WEIGHTS if a.pdl else 0
-        ms = _time(lambda: w4.w4a16_linear_batched(arr, a.m, flags), a.iters, not a.eager)
-        out.update(ms=ms, gbs=byts / ms / 1e6, linears=len(items))
+        if a.a8:  # W4A8: activations quantized once, outside the timed launches
+            arr = w4.a8_items([(*w4.quantize_act_int8(x), qw, sc, zr, y)
+                               for (x, qw, sc, zr, y) in items])
+            ms = _time(lambda: w4.w4a8_linear_batched(arr, a.m, flags), a.iters, not a.eager)
+        else:
+            arr = w4.linear_items(items)
+            ms = _time(lambda: w4.w4a16_linear_batched(arr, a.m, flags), a.iters, not a.eager)
+        out.update(ms=ms, gbs=byts / ms / 1e6, linears=len(items), a8=a.a8)
     elif a.case == "clip_rows":
         g = torch.Generator(device="cuda")
         g.manual_seed(3)

@@ -251,6 +251,7 @@ w4_status w4a16_linear(const void* x_bf16, int64_t M, const int32_t* qweight,
     b.count = 0;
     b.unit_start[0] = 0;
     b.M = static_cast<int>(M);
+    b.a8 = 0;
     stream_batch_add(b, x_bf16, qweight, scales_f16, zeros_f16, static_cast<int>(N),
                      static_cast<int>(K), y_bf16);
     int bundles = 0;
@@ -270,6 +271,87 @@ w4_status w4a16_linear(const void* x_bf16, int64_t M, const int32_t* qweight,
                                          zeros_f16, static_cast<int>(N), static_cast<int>(K),
                                          y_bf16, pdl, stat, s, err),
                      "prefill tcgen05 GEMM launch");
+}
+
+w4_status w4_quantize_act_int8(const void* x_bf16, int64_t M, int64_t K, int8_t* xq_out,
+                               int32_t* xsum_out, float* xscale_out, void* stream) {
+  if (!x_bf16 || !xq_out || !xsum_out || !xscale_out) return W4_ERR_INVALID_ARG;
+  if (M < 1 || M > 0x7FFFFFFF || !valid_k(K)) return W4_ERR_SHAPE;
+  if (!aligned16(x_bf16) || !aligned16(xq_out) || !aligned16(xsum_out) || !aligned16(xscale_out))
+    return W4_ERR_ALIGNMENT;
+  return cuda_status(launch_quantize_act_int8(x_bf16, M, K, xq_out, xsum_out, xscale_out,
+                                              static_cast<cudaStream_t>(stream)),
+                     "int8 activation quantize launch");
+}
+
+static w4_status check_a8_item(const w4a8_item& it, int64_t M) {
+  if (!it.xq || !it.xsum || !it.xscale || !it.qweight || !it.scales_f16 || !it.y_bf16)
+    return W4_ERR_INVALID_ARG;
+  if (M < 1 || it.N < 1 || !valid_k(it.K) || it.N > 0x7FFFFFFF || it.K > kGemvMaxK)
+    return W4_ERR_SHAPE;
+  if (!aligned16(it.xq) || !aligned16(it.xsum) || !aligned16(it.xscale) ||
+      !aligned16(it.qweight) || !aligned16(it.scales_f16) ||
+      (it.zeros_f16 && !aligned16(it.zeros_f16)) || !aligned16(it.y_bf16))
+    return W4_ERR_ALIGNMENT;
+  return W4_OK;
+}
+
+w4_status w4a8_linear_batched(const w4a8_item* items, int count, int64_t M, int group,
+                              unsigned flags, void* stream) {
+  if (!items || count < 1) return W4_ERR_INVALID_ARG;
+  if (flags & ~(W4_LINEAR_PDL | W4_LINEAR_STATIC_WEIGHTS)) return W4_ERR_INVALID_ARG;
+  if (group != 128) return W4_ERR_UNSUPPORTED;
+  if (M > 16) return W4_ERR_UNSUPPORTED;
+  const bool sym = items[0].zeros_f16 == nullptr;
+  for (int i = 0; i < count; ++i) {
+    const w4_status st = check_a8_item(items[i], M);
+    if (st != W4_OK) return st;
+    if ((items[i].zeros_f16 == nullptr) != sym) return W4_ERR_INVALID_ARG;
+  }
+  int sms = 0;
+  unsigned* err = nullptr;
+  w4_status st = device_info(&sms, &err);
+  if (st != W4_OK) return st;
+  const bool pdl = (flags & W4_LINEAR_PDL) != 0;
+  const bool stat = (flags & W4_LINEAR_STATIC_WEIGHTS) != 0;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  std::vector<int> order(count);
+  for (int i = 0; i < count; ++i) order[i] = i;
+  std::stable_sort(order.begin(), order.end(),
+                   [&](int a, int c) { return items[a].K > items[c].K; });
+  // Tokens in chunks of 8 (the kernel's mma columns), linears in launches of
+  // up to kStreamBatch, longest K first.
+  for (int64_t m0 = 0; m0 < M; m0 += 8) {
+    const int mc = static_cast<int>(M - m0 < 8 ? M - m0 : 8);
+    for (int i0 = 0; i0 < count;) {
+      StreamBatch b;
+      b.count = 0;
+      b.unit_start[0] = 0;
+      b.M = mc;
+      b.a8 = 1;
+      int j = i0;
+      for (; j < count && j < i0 + kStreamBatch; ++j) {
+        const w4a8_item& it = items[order[j]];
+        if (b.count > 0 && b.unit_start[b.count] + (it.N + 63) / 64 > (int64_t{1} << 30)) break;
+        stream_batch_add(b, it.xq + m0 * it.K, it.qweight, it.scales_f16, it.zeros_f16,
+                         static_cast<int>(it.N), static_cast<int>(it.K),
+                         static_cast<uint16_t*>(it.y_bf16) + m0 * it.N,
+                         it.xsum + m0 * (it.K / 128), it.xscale + m0);
+      }
+      st = cuda_status(launch_gemv_stream(b, sym, pdl, stat, s, sms), "W4A8 decode GEMV launch");
+      if (st != W4_OK) return st;
+      i0 = j;
+    }
+  }
+  return W4_OK;
+}
+
+w4_status w4a8_linear(const int8_t* xq, const int32_t* xsum, const float* xscale, int64_t M,
+                      const int32_t* qweight, const uint16_t* scales_f16,
+                      const uint16_t* zeros_f16, int64_t N, int64_t K, int group, void* y_bf16,
+                      unsigned flags, void* stream) {
+  const w4a8_item it{xq, xsum, xscale, qweight, scales_f16, zeros_f16, N, K, y_bf16};
+  return w4a8_linear_batched(&it, 1, M, group, flags, stream);
 }
 
 // Decodes items idx[0..n) through the per-CTA tensor-map kernel.  Launches
@@ -369,6 +451,7 @@ w4_status w4a16_linear_batched(const w4_linear_item* items, int count, int64_t M
     b.count = 0;
     b.unit_start[0] = 0;
     b.M = static_cast<int>(M);
+    b.a8 = 0;
     int j = i0;
     // (a launch's bundles are counted in int: at most 2^30 of them)
     for (; j < count && j < i0 + kStreamBatch; ++j) {

@@ -124,6 +124,38 @@ __device__ __forceinline__ void tile_group_s(float (&d)[4], const uint4 wa, cons
 }
 #undef W4S_STEP
 
+// W4A8: one 16-row tile over one group against int8 activations, 4 steps of
+// mma.m16n8k32 (u8 codes x s8 activations, exact int32 sums).  Word j of
+// each row gives two A registers by masking: low nibbles (channels 0, 4, 1,
+// 5 of the word's 8) and high nibbles (2, 6, 3, 7); the activation codes are
+// stored in the same channel order, so x words 2j and 2j+1 are the matching
+// B registers.
+#define W4A8_STEP(VA, VB, B0, B1, CIN)                                           \
+  "shr.b32 s0, " VA ", 4;\n\t"                                                   \
+  "shr.b32 s1, " VB ", 4;\n\t"                                                   \
+  "and.b32 a0, " VA ", 0x0F0F0F0F;\n\t"                                          \
+  "and.b32 a1, " VB ", 0x0F0F0F0F;\n\t"                                          \
+  "and.b32 a2, s0, 0x0F0F0F0F;\n\t"                                              \
+  "and.b32 a3, s1, 0x0F0F0F0F;\n\t"                                              \
+  "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0, %1, %2, %3}, "            \
+  "{a0, a1, a2, a3}, {" B0 ", " B1 "}, " CIN ";\n\t"
+
+__device__ __forceinline__ void tile_group_a8(int (&d)[4], const uint4 wa, const uint4 wb,
+                                              const uint4 (&x)[2]) {
+  asm("{\n\t.reg .b32 a0, a1, a2, a3, s0, s1;\n\t"
+      ".reg .s32 z;\n\tmov.b32 z, 0;\n\t"
+      W4A8_STEP("%4", "%8", "%12", "%13", "{z, z, z, z}")
+      W4A8_STEP("%5", "%9", "%14", "%15", "{%0, %1, %2, %3}")
+      W4A8_STEP("%6", "%10", "%16", "%17", "{%0, %1, %2, %3}")
+      W4A8_STEP("%7", "%11", "%18", "%19", "{%0, %1, %2, %3}")
+      "}"
+      : "=&r"(d[0]), "=&r"(d[1]), "=&r"(d[2]), "=&r"(d[3])
+      : "r"(wa.x), "r"(wa.y), "r"(wa.z), "r"(wa.w), "r"(wb.x), "r"(wb.y), "r"(wb.z), "r"(wb.w),
+        "r"(x[0].x), "r"(x[0].y), "r"(x[0].z), "r"(x[0].w), "r"(x[1].x), "r"(x[1].y),
+        "r"(x[1].z), "r"(x[1].w));
+}
+#undef W4A8_STEP
+
 __device__ __forceinline__ float half_bits_to_float(uint32_t h) {
   return __half2float(__ushort_as_half(static_cast<unsigned short>(h)));
 }
@@ -165,7 +197,9 @@ constexpr int kTiles = 4;  // 16-row mma tiles per unit (64 weight rows)
 constexpr uint32_t kSlotCodes = kTiles * 1024;
 constexpr uint32_t kSlotBytes = kSlotCodes + kTiles * 128;
 
-template <bool SYM, int S, int MIN_CTAS>
+// A8 = false: bf16 activations (W4A16).  A8 = true: int8 activation codes
+// with per-token scales and per-group code sums (W4A8).
+template <bool SYM, int S, int MIN_CTAS, bool A8>
 __global__ void __launch_bounds__(kStreamThreads, MIN_CTAS)
     gemv_w4a16_stream_kernel(const __grid_constant__ StreamBatch b, int static_weights) {
   // Partial sums of the warps of a unit: [warp][tile][lane].
@@ -267,16 +301,32 @@ __global__ void __launch_bounds__(kStreamThreads, MIN_CTAS)
   enter_bundle(b, cp, first, warp, units);
   // x fragments (token g, channels 32t .. 32t+31 of a group) are loaded one
   // group ahead of use; xq walks the compute list one group ahead of cp.
+  // W4A8: dst[0..1] hold the 32 activation codes, dst[2].x / .y the group's
+  // code sums of tokens 2t and 2t + 1 (the mma's output columns).
   UnitPos xq = cp;
   auto load_x = [&](uint4 (&dst)[4]) {
-    if (xq.bundle < units && g < M) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) dst[j] = make_uint4(0u, 0u, 0u, 0u);
+    if constexpr (A8) {
+      if (xq.bundle < units) {
+        const int K = b.K[xq.item];
+        if (g < M) {
+          const uint4* xp = reinterpret_cast<const uint4*>(
+              reinterpret_cast<const int8_t*>(b.x[xq.item]) + static_cast<size_t>(g) * K +
+              xq.g * 128 + 32 * t);
+          dst[0] = __ldg(xp);
+          dst[1] = __ldg(xp + 1);
+        }
+        const int32_t* xs = b.xsum[xq.item] + xq.g;
+        if (2 * t < M) dst[2].x = static_cast<uint32_t>(__ldg(xs + static_cast<size_t>(2 * t) * (K >> 7)));
+        if (2 * t + 1 < M)
+          dst[2].y = static_cast<uint32_t>(__ldg(xs + static_cast<size_t>(2 * t + 1) * (K >> 7)));
+      }
+    } else if (xq.bundle < units && g < M) {
       const uint4* xp = reinterpret_cast<const uint4*>(
           b.x[xq.item] + static_cast<size_t>(g) * b.K[xq.item] + xq.g * 128 + 32 * t);
 #pragma unroll
       for (int j = 0; j < 4; ++j) dst[j] = __ldg(xp + j);
-    } else {
-#pragma unroll
-      for (int j = 0; j < 4; ++j) dst[j] = make_uint4(0u, 0u, 0u, 0u);
     }
     if (xq.bundle < units && ++xq.g == xq.ge) enter_bundle(b, xq, xq.bundle + stride, warp, units);
   };
@@ -303,16 +353,18 @@ __global__ void __launch_bounds__(kStreamThreads, MIN_CTAS)
 #pragma unroll
     for (int j = 0; j < 4; ++j) xv[j] = xnext[j];
     load_x(xnext);
-    // Per-token sums of x over the group (all-ones rows), two chains.
+    // W4A16: per-token sums of x over the group (all-ones rows), two chains.
     float xs[4] = {0.f, 0.f, 0.f, 0.f};
-    float xt[4] = {0.f, 0.f, 0.f, 0.f};
+    if constexpr (!A8) {
+      float xt[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      mma_16816(xs, ones, ones, ones, ones, xv[j].x, xv[j].y);
-      mma_16816(xt, ones, ones, ones, ones, xv[j].z, xv[j].w);
+      for (int j = 0; j < 4; ++j) {
+        mma_16816(xs, ones, ones, ones, ones, xv[j].x, xv[j].y);
+        mma_16816(xt, ones, ones, ones, ones, xv[j].z, xv[j].w);
+      }
+#pragma unroll
+      for (int k = 0; k < 4; ++k) xs[k] += xt[k];
     }
-#pragma unroll
-    for (int k = 0; k < 4; ++k) xs[k] += xt[k];
     // This slot's copies (issued S groups ago) have landed; every lane reads
     // back only what it copied itself.
     cp_async_wait<S - 1>();
@@ -323,20 +375,37 @@ __global__ void __launch_bounds__(kStreamThreads, MIN_CTAS)
       const uint4 wa = lds128s(src + rt * 1024 + lane * 16);
       const uint4 wb = lds128s(src + rt * 1024 + 512 + lane * 16);
       const uint32_t v = (lds32s(src + kSlotCodes + rt * 128 + lane * 4) >> sh) & 0xFFFFu;
-      float c[4];
-      tile_group_s(c, wa, wb, xv);
       const int q0 = lane & ~3;
       const float sa = half_bits_to_float(__shfl_sync(0xffffffffu, v, q0 + 0));
       const float sb = half_bits_to_float(__shfl_sync(0xffffffffu, v, q0 + 1));
-      float za = 136.0f, zb = 136.0f;  // 128 + zero (symmetric: zero 8)
-      if (!SYM) {
-        za = 128.0f + half_bits_to_float(__shfl_sync(0xffffffffu, v, q0 + 2));
-        zb = 128.0f + half_bits_to_float(__shfl_sync(0xffffffffu, v, q0 + 3));
+      if constexpr (A8) {
+        // D = sum (q - z) x8 = sum q x8 - z * S (exact int32), then scale.
+        int c[4];
+        const uint4 x8[2] = {xv[0], xv[1]};
+        tile_group_a8(c, wa, wb, x8);
+        int za = 8, zb = 8;  // symmetric: zero 8
+        if (!SYM) {
+          za = __float2int_rn(half_bits_to_float(__shfl_sync(0xffffffffu, v, q0 + 2)));
+          zb = __float2int_rn(half_bits_to_float(__shfl_sync(0xffffffffu, v, q0 + 3)));
+        }
+        const int s0 = static_cast<int>(xv[2].x), s1 = static_cast<int>(xv[2].y);
+        acc[rt][0] = fmaf(sa, __int2float_rn(c[0] - za * s0), acc[rt][0]);
+        acc[rt][1] = fmaf(sa, __int2float_rn(c[1] - za * s1), acc[rt][1]);
+        acc[rt][2] = fmaf(sb, __int2float_rn(c[2] - zb * s0), acc[rt][2]);
+        acc[rt][3] = fmaf(sb, __int2float_rn(c[3] - zb * s1), acc[rt][3]);
+      } else {
+        float c[4];
+        tile_group_s(c, wa, wb, xv);
+        float za = 136.0f, zb = 136.0f;  // 128 + zero (symmetric: zero 8)
+        if (!SYM) {
+          za = 128.0f + half_bits_to_float(__shfl_sync(0xffffffffu, v, q0 + 2));
+          zb = 128.0f + half_bits_to_float(__shfl_sync(0xffffffffu, v, q0 + 3));
+        }
+        acc[rt][0] = fmaf(sa, fmaf(-za, xs[0], c[0]), acc[rt][0]);
+        acc[rt][1] = fmaf(sa, fmaf(-za, xs[1], c[1]), acc[rt][1]);
+        acc[rt][2] = fmaf(sb, fmaf(-zb, xs[2], c[2]), acc[rt][2]);
+        acc[rt][3] = fmaf(sb, fmaf(-zb, xs[3], c[3]), acc[rt][3]);
       }
-      acc[rt][0] = fmaf(sa, fmaf(-za, xs[0], c[0]), acc[rt][0]);
-      acc[rt][1] = fmaf(sa, fmaf(-za, xs[1], c[1]), acc[rt][1]);
-      acc[rt][2] = fmaf(sb, fmaf(-zb, xs[2], c[2]), acc[rt][2]);
-      acc[rt][3] = fmaf(sb, fmaf(-zb, xs[3], c[3]), acc[rt][3]);
     }
     // The slot's data has been consumed: refill it with the group S ahead.
     load_group(slot);
@@ -376,6 +445,18 @@ __global__ void __launch_bounds__(kStreamThreads, MIN_CTAS)
         const int N = b.N[cp.item];
         __nv_bfloat16* y = b.y[cp.item];
         const int m0 = 2 * t, m1 = 2 * t + 1;
+        if constexpr (A8) {  // y = xscale_m * sum_g scale * D
+          const float* xsc = b.xscale[cp.item];
+          const float f0 = m0 < M ? __ldg(xsc + m0) : 0.f;
+          const float f1 = m1 < M ? __ldg(xsc + m1) : 0.f;
+#pragma unroll
+          for (int rt = 0; rt < kTiles; ++rt) {
+            acc[rt][0] *= f0;
+            acc[rt][1] *= f1;
+            acc[rt][2] *= f0;
+            acc[rt][3] *= f1;
+          }
+        }
 #pragma unroll
         for (int rt = 0; rt < kTiles; ++rt) {
           const int r0 = crow + 16 * rt;
@@ -464,11 +545,11 @@ cudaError_t launch_stream_cfg(const StreamBatch& b, int grid, bool pdl, bool sta
   return cudaLaunchKernelEx(&cfg, kern, b, static_cast<int>(pdl && static_w));
 }
 
-template <bool SYM>
+template <bool SYM, bool A8>
 cudaError_t launch_stream_t(StreamBatch& b, bool pdl, bool static_w, cudaStream_t stream,
                             int num_sms) {
-  constexpr auto kWide = gemv_w4a16_stream_kernel<SYM, kDepthWide, 3>;
-  constexpr auto kDeep = gemv_w4a16_stream_kernel<SYM, kDepthDeep, 2>;
+  constexpr auto kWide = gemv_w4a16_stream_kernel<SYM, kDepthWide, 3, A8>;
+  constexpr auto kDeep = gemv_w4a16_stream_kernel<SYM, kDepthDeep, 2, A8>;
   constexpr size_t kWideBytes = ring_bytes<kDepthWide>();
   constexpr size_t kDeepBytes = ring_bytes<kDepthDeep>();
   int dev = 0;
@@ -494,9 +575,12 @@ cudaError_t launch_stream_t(StreamBatch& b, bool pdl, bool static_w, cudaStream_
 // most 4 parts, each of at least 2 groups): units of similar length keep the
 // warps' totals even when linears of different K share a launch.
 void stream_batch_add(StreamBatch& b, const void* x, const int32_t* qw, const uint16_t* sc,
-                      const uint16_t* z, int N, int K, void* y) {
+                      const uint16_t* z, int N, int K, void* y, const int32_t* xsum,
+                      const float* xscale) {
   const int i = b.count;
   b.x[i] = static_cast<const __nv_bfloat16*>(x);
+  b.xsum[i] = xsum;
+  b.xscale[i] = xscale;
   b.qw[i] = reinterpret_cast<const uint8_t*>(qw);
   b.scales[i] = sc;
   b.zeros[i] = z;
@@ -515,7 +599,7 @@ void stream_batch_add(StreamBatch& b, const void* x, const int32_t* qw, const ui
 
 template <bool SYM>
 cudaError_t plan_stream_t(StreamBatch& b, int num_sms, int* bundles) {
-  constexpr auto kWide = gemv_w4a16_stream_kernel<SYM, kDepthWide, 3>;
+  constexpr auto kWide = gemv_w4a16_stream_kernel<SYM, kDepthWide, 3, false>;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
@@ -535,8 +619,11 @@ cudaError_t plan_gemv_stream(StreamBatch& b, bool symmetric, int num_sms, int* b
 cudaError_t launch_gemv_stream(StreamBatch& b, bool symmetric, bool pdl, bool static_w,
                                cudaStream_t stream, int num_sms) {
   if (b.count < 1 || b.M < 1 || b.M > 8) return cudaErrorInvalidValue;
-  return symmetric ? launch_stream_t<true>(b, pdl, static_w, stream, num_sms)
-                   : launch_stream_t<false>(b, pdl, static_w, stream, num_sms);
+  if (b.a8)
+    return symmetric ? launch_stream_t<true, true>(b, pdl, static_w, stream, num_sms)
+                     : launch_stream_t<false, true>(b, pdl, static_w, stream, num_sms);
+  return symmetric ? launch_stream_t<true, false>(b, pdl, static_w, stream, num_sms)
+                   : launch_stream_t<false, false>(b, pdl, static_w, stream, num_sms);
 }
 
 }  // namespace w4

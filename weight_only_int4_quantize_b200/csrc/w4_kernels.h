@@ -68,19 +68,23 @@ cudaError_t launch_gemv(const void* x, int M, const int32_t* qw, const uint16_t*
 // decoded by one persistent streaming launch (kernel parameter).
 constexpr int kStreamBatch = 256;
 struct StreamBatch {
-  const __nv_bfloat16* x[kStreamBatch];  // bf16 [M, K]
+  const __nv_bfloat16* x[kStreamBatch];  // bf16 [M, K]; W4A8: int8 codes [M, K]
   const uint8_t* qw[kStreamBatch];       // packed codes, [N, K/2] bytes
   const uint16_t* scales[kStreamBatch];  // fp16 [N, K/128]
   const uint16_t* zeros[kStreamBatch];   // fp16 [N, K/128]; NULL: symmetric
   __nv_bfloat16* y[kStreamBatch];        // bf16 [M, N]
   int N[kStreamBatch];
   int K[kStreamBatch];
+  const int32_t* xsum[kStreamBatch];     // W4A8: per-group code sums [M, K/128]
+  const float* xscale[kStreamBatch];     // W4A8: per-token scales [M]
   int ks[kStreamBatch];                  // K parts of each linear (1, 2 or 4)
   int unit_start[kStreamBatch + 1];      // prefix sums of bundles (4 warp units each)
   int count, M;
+  int a8;                                // activations: 0 bf16, 1 int8 codes
 };
 void stream_batch_add(StreamBatch& b, const void* x, const int32_t* qw, const uint16_t* sc,
-                      const uint16_t* z, int N, int K, void* y);
+                      const uint16_t* z, int N, int K, void* y, const int32_t* xsum = nullptr,
+                      const float* xscale = nullptr);
 // Chooses the K split of every linear for the launch's grid; *bundles is the
 // number of 4-warp bundles the launch would deal (launch_gemv_stream plans
 // the same way, so planning first does not change the launch).
@@ -100,6 +104,11 @@ struct PrefillItem {
 // Up to 16 linears per tcgen05 launch (more in further launches).
 cudaError_t launch_prefill_gemm_group(const PrefillItem* items, int count, int M, bool pdl,
                                       bool static_w, cudaStream_t stream, unsigned* err);
+// Per-token int8 activation codes (channel order 0,4,1,5,2,6,3,7 in every
+// 8-channel chunk), per-group code sums and per-token scales.
+cudaError_t launch_quantize_act_int8(const void* x, int64_t M, int64_t K, int8_t* xq,
+                                     int32_t* xsum, float* xscale, cudaStream_t stream);
+
 cudaError_t launch_prefill_gemm(const void* x, int M, const int32_t* qw, const uint16_t* sc,
                                 const uint16_t* z, int N, int K, void* y, bool pdl,
                                 bool static_w, cudaStream_t stream, unsigned* err);
