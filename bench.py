@@ -70,6 +70,20 @@ def source_digest(name):
         return None
 
 
+def max_over_ranks(dist, t_ms, device):
+    """Replica timing: the slowest rank's time (every rank calls this once)."""
+    import torch
+    t = torch.tensor([float(t_ms)], device=device, dtype=torch.float64)
+    if dist is not None:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_gbs(world, bytes_per_rank, max_ms):
+    """Whole-job throughput of `world` replicas over the slowest rank's time."""
+    return world * bytes_per_rank / (max_ms * 1e-3) / 1e9
+
+
 def quant_bytes(n, k, sym=False):
     return n * k * (2 + 0.5 + (2 if sym else 4) / 128)
 
@@ -491,15 +505,12 @@ def main():
     if pg:
         pg.barrier()
     total_ms = start.elapsed_time(end)
-    t_local = torch.tensor([total_ms], device=dev, dtype=torch.float64)
-    if pg:
-        pg.all_reduce(t_local, op=pg.ReduceOp.MAX)
-    total_ms = float(t_local.item())
+    total_ms = max_over_ranks(pg, total_ms, dev)
     ms_step = total_ms / args.steps
     q_ms = sum(e[0].elapsed_time(e[1]) for e in ev) / args.steps
     d_ms = {m: sum(e[1 + j].elapsed_time(e[2 + j]) for e in ev) / args.steps
             for j, m in enumerate(DECODE_M)}
-    value = world * (qb + db) / (ms_step * 1e-3) / 1e9
+    value = whole_job_gbs(world, qb + db, ms_step)
     clocks = clk.summary()
 
     # ---------------------------------------------- end to end (host buffers)
@@ -542,10 +553,8 @@ def main():
         e2e_step()
     b.record()
     torch.cuda.synchronize()
-    e2e_ms = torch.tensor([a.elapsed_time(b) / n_e2e], device=dev, dtype=torch.float64)
-    if pg:
-        pg.all_reduce(e2e_ms, op=pg.ReduceOp.MAX)
-    e2e_val = world * (qb + db) / (float(e2e_ms.item()) * 1e-3) / 1e9
+    e2e_ms = max_over_ranks(pg, a.elapsed_time(b) / n_e2e, dev)
+    e2e_val = whole_job_gbs(world, qb + db, e2e_ms)
     del host_w, host_x, host_q, host_y
 
     # ---------------------------------------------- W4A8 decode (same weights)
