@@ -147,7 +147,7 @@ w4_status w4_quantize_pack_batched(const w4_quant_item* items, int count, int gr
  *           rounded once to bf16).
  * flags     bitwise OR of W4_LINEAR_* below (0 for defaults).
  *
- * M <= 16 (and K <= 81920) runs a decode GEMV (tensor-core mma over
+ * M <= 32 (and K <= 81920) runs a decode GEMV (tensor-core mma over
  * register-dequantized weight fragments, HBM-bound); larger M runs the
  * prefill GEMM (tcgen05 with TMEM accumulators, weight tiles dequantized into
  * shared memory).  There are two decode kernels: a persistent streaming
@@ -155,7 +155,9 @@ w4_status w4_quantize_pack_batched(const w4_quant_item* items, int count, int gr
  * launches with at least two of its 4-warp bundles per SM, and a per-CTA
  * tensor-map kernel (K split over a thread-block cluster) for smaller
  * launches and 9 <= M <= 64.  W4_LINEAR_DECODE_STREAM / _TILED override the
- * choice; both meet the same error bound.
+ * choice; both meet the same error bound.  A prefill launch with few tiles
+ * splits K over a thread-block cluster of up to 4 CTAs and adds the fp32
+ * partial tiles through distributed shared memory in rank order.
  */
 #define W4_LINEAR_FORCE_GEMV 0x1u  /* decode kernel at any M <= 64 (K <= 81920) */
 #define W4_LINEAR_FORCE_GEMM 0x2u  /* prefill kernel at any M */
@@ -182,10 +184,11 @@ w4_status w4a16_linear(const void* x_bf16, int64_t M, const int32_t* qweight,
  * share the token count M and the symmetry (all zeros NULL or none), for
  * example every projection of a decode step whose inputs are ready.  M <= 8
  * runs up to 256 linears per persistent streaming launch (or, for a launch
- * too small to fill the GPU, the tensor-map kernel); 9 <= M <= 64 (K <=
- * 81920) runs the tensor-map kernel with up to 32 linears per launch; larger
- * M runs grouped prefill GEMM launches, up to 16 linears each (every CTA
- * finds its linear and tile; the tile shape is chosen for the group).  flags: W4_LINEAR_PDL,
+ * too small to fill the GPU, the tensor-map kernel); 9 <= M <= 32 (K <=
+ * 81920) runs the tensor-map kernel with up to 32 linears per launch (up to
+ * M = 64 with W4_LINEAR_DECODE_TILED); larger M runs grouped prefill GEMM
+ * launches, up to 16 linears each (every CTA finds its linear and tile; the
+ * tile shape and K split are chosen for the group).  flags: W4_LINEAR_PDL,
  * W4_LINEAR_STATIC_WEIGHTS and the W4_LINEAR_DECODE_* choice only.  items: host array.  Each result meets the
  * same error bound as a per-linear call (the K split of a batch, and so the
  * binary32 summation order, may differ from a single call's).

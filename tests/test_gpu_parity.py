@@ -198,6 +198,30 @@ def test_gemv_stream_deterministic():
     assert torch.equal(y0.view(torch.int16), y1.view(torch.int16))
 
 
+@pytest.mark.parametrize("m", [24, 32])
+def test_decode_default_up_to_32_rows(m):
+    assert linear_case(m, 700, 1024, False, seed=150 + m) <= Y_RTOL
+
+
+@pytest.mark.parametrize("m,n,k", [(33, 512, 8192), (64, 300, 17408), (130, 640, 4096),
+                                   (300, 256, 6144)])
+@pytest.mark.parametrize("sym", [False, True])
+def test_prefill_split_k(m, n, k, sym):
+    """Few tiles and long K: the prefill GEMM splits K over a cluster and
+    adds the partial tiles through distributed shared memory."""
+    assert linear_case(m, n, k, sym, seed=160 + m + n) <= Y_RTOL
+
+
+def test_prefill_split_k_deterministic():
+    w = synth.normal_weight(384, 8192, 0.02, seed=171)
+    x = synth.normal_activations(48, 8192, seed=172).to(DEV)
+    qw, sc, zr = w4.quantize_pack(w.to(DEV), False)
+    y0 = w4.w4a16_linear(x, qw, sc, zr)
+    y1 = w4.w4a16_linear(x, qw, sc, zr)
+    torch.cuda.synchronize()
+    assert torch.equal(y0.view(torch.int16), y1.view(torch.int16))
+
+
 @pytest.mark.parametrize("m", [17, 40, 64])
 def test_gemv_forced_chunks(m):
     assert linear_case(m, 520, 640, False, seed=200 + m, flags=w4.LINEAR_FORCE_GEMV) <= Y_RTOL

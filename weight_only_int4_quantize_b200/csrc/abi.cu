@@ -209,6 +209,7 @@ static w4_status check_linear_item(const void* x_bf16, int64_t M, const int32_t*
 }
 
 static constexpr int64_t kGemvMaxK = 8 * 80 * 128;  // decode kernel: K slice <= 80 groups x 8
+static constexpr int64_t kDecodeMaxRows = 32;       // decode kernels up to this M by default
 
 // The persistent streaming decode kernel is chosen for launches that deal
 // at least this many 4-warp bundles per SM; smaller launches (a single
@@ -234,8 +235,11 @@ w4_status w4a16_linear(const void* x_bf16, int64_t M, const int32_t* qweight,
   // The decode kernels keep a CTA's K slice (at most 8 x 80 groups) in a
   // shared scale table; longer K goes to the prefill kernel.
   const bool gemv_ok = K <= kGemvMaxK;
+  // Measured on B200: the decode kernels beat the prefill GEMM up to 32
+  // tokens on the 27B-scale linears (two 16-token passes still read less
+  // than the GEMM's dequantized tiles cost).
   const bool gemv = (flags & (W4_LINEAR_FORCE_GEMV | kDecodeChoice)) ||
-                    (M <= 16 && gemv_ok && !(flags & W4_LINEAR_FORCE_GEMM));
+                    (M <= kDecodeMaxRows && gemv_ok && !(flags & W4_LINEAR_FORCE_GEMM));
   if (gemv && (M > 64 || !gemv_ok)) return W4_ERR_UNSUPPORTED;
   if ((flags & W4_LINEAR_DECODE_STREAM) && M > 8) return W4_ERR_UNSUPPORTED;
   if (!gemv && (M + 127) / 128 > 65535) return W4_ERR_UNSUPPORTED;
@@ -415,7 +419,8 @@ w4_status w4a16_linear_batched(const w4_linear_item* items, int count, int64_t M
                                      it.K, it.y_bf16);
     if (st != W4_OK) return st;
     if ((it.zeros_f16 == nullptr) != sym) return W4_ERR_INVALID_ARG;
-    if (M <= 64 && it.K > kGemvMaxK) return W4_ERR_UNSUPPORTED;
+    if ((M <= kDecodeMaxRows || (flags & kDecodeChoice)) && it.K > kGemvMaxK)
+      return W4_ERR_UNSUPPORTED;
   }
   int sms = 0;
   unsigned* err = nullptr;
@@ -424,7 +429,8 @@ w4_status w4a16_linear_batched(const w4_linear_item* items, int count, int64_t M
   const bool pdl = (flags & W4_LINEAR_PDL) != 0;
   const bool stat = (flags & W4_LINEAR_STATIC_WEIGHTS) != 0;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (M > 64) {  // prefill: grouped tcgen05 launches (up to 16 linears each)
+  if (M > kDecodeMaxRows && !(flags & kDecodeChoice)) {
+    // prefill: grouped tcgen05 launches (up to 16 linears each)
     if ((M + 127) / 128 > 65535) return W4_ERR_UNSUPPORTED;
     std::vector<PrefillItem> pi(count);
     for (int i = 0; i < count; ++i) {

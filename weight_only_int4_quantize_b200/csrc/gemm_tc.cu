@@ -23,6 +23,7 @@
 // Every mbarrier wait is bounded (w4_common.cuh); a CTA that gives up sets
 // the device error word, drains its own TMA loads and MMAs, frees its TMEM
 // and returns.  No TMA multicast.
+#include <cooperative_groups.h>
 #include <cudaTypedefs.h>
 
 #include <cmath>
@@ -31,6 +32,8 @@
 #include "w4_kernels.h"
 
 namespace w4 {
+
+namespace cg = cooperative_groups;
 
 namespace {
 
@@ -206,11 +209,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   __nv_bfloat16* __restrict__ y = nullptr;
   int N = N_arg, K = K_arg;
   int tile_n = blockIdx.x, tile_m = blockIdx.y;
+  // Split K over a thread-block cluster (prefill launches with few tiles):
+  // CTA `rank` of the cluster takes its share of the k-blocks, and the
+  // partial accumulators are added through distributed shared memory.
+  int ks = 1, rank = 0;
   if constexpr (BSRC == kBDequant) {
+    asm("mov.u32 %0, %%cluster_nctarank;" : "=r"(ks));
+    asm("mov.u32 %0, %%cluster_ctarank;" : "=r"(rank));
+  }
+  if constexpr (BSRC == kBDequant) {
+    const int cta_tile = static_cast<int>(blockIdx.x) / ks;
     int lo = 0, hi = grp.count - 1;
     while (lo < hi) {
       const int mid = (lo + hi + 1) >> 1;
-      if (grp.tile_start[mid] <= static_cast<int>(blockIdx.x)) lo = mid; else hi = mid - 1;
+      if (grp.tile_start[mid] <= cta_tile) lo = mid; else hi = mid - 1;
     }
     ta = &grp.ta[lo];
     qw = grp.qw[lo];
@@ -219,7 +231,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     y = grp.y[lo];
     N = grp.N[lo];
     K = grp.K[lo];
-    const int local = static_cast<int>(blockIdx.x) - grp.tile_start[lo];
+    const int local = cta_tile - grp.tile_start[lo];
     const int n_tiles = (N + NB - 1) / NB;
     tile_n = local % n_tiles;
     tile_m = local / n_tiles;
@@ -227,7 +239,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int n0 = tile_n * NB;
   const int m0 = tile_m * (MT * BM);
   const int cand = blockIdx.z;
-  const int num_kb = K / BK;
+  // This CTA's k-blocks: [kb_begin, kb_begin + num_kb); every loop below runs
+  // over local indices (stages and phases count from the first local block).
+  const int kb_begin = rank * (K / BK) / ks;
+  const int num_kb = (rank + 1) * (K / BK) / ks - kb_begin;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -264,11 +279,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!mbar_wait(empty(s), ph ^ 1u, abort_flag, err, kKernelIdGemm)) break;
         if (BSRC == kBTma) {
           mbar_arrive_expect_tx(full_a(s), kTileABytes + kTileBBytes);
-          tma_load_2d(sA + s * kTileABytes, ta, kb * BK, m0, full_a(s));
-          tma_load_3d(sB + s * kTileBBytes, &tmap_b, kb * BK, n0, cand, full_a(s));
+          tma_load_2d(sA + s * kTileABytes, ta, (kb_begin + kb) * BK, m0, full_a(s));
+          tma_load_3d(sB + s * kTileBBytes, &tmap_b, (kb_begin + kb) * BK, n0, cand, full_a(s));
         } else {
           mbar_arrive_expect_tx(full_a(s), kTileABytes);
-          tma_load_2d(sA + s * kTileABytes, ta, kb * BK, m0, full_a(s));
+          tma_load_2d(sA + s * kTileABytes, ta, (kb_begin + kb) * BK, m0, full_a(s));
         }
         kb_stop = kb + 1;
       }
@@ -349,9 +364,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           q[it] = make_uint4(0, 0, 0, 0);
           sz[it] = 0x48000000u;  // scale 0, zero 8
           if (valid[it] && kb < num_kb) {
-            q[it] = __ldg(reinterpret_cast<const uint4*>(qrow[it] + kb * 8));
-            sz[it] = srow[it][kb >> 1];
-            sz[it] |= SYM ? 0x48000000u : (static_cast<uint32_t>(zrow[it][kb >> 1]) << 16);
+            const int ka = kb_begin + kb;  // absolute k-block
+            q[it] = __ldg(reinterpret_cast<const uint4*>(qrow[it] + ka * 8));
+            sz[it] = srow[it][ka >> 1];
+            sz[it] |= SYM ? 0x48000000u : (static_cast<uint32_t>(zrow[it][ka >> 1]) << 16);
           }
         }
       };
@@ -402,7 +418,27 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool ok = mbar_wait(acc_full, 0, abort_flag, err, kKernelIdGemm);
     tc_fence_after();
     if (ok) {
-      if (EPI == kEpiStoreBf16) {
+      if (EPI == kEpiStoreBf16 && ks > 1) {
+        // Split K: this CTA's fp32 partial tile into its own shared memory
+        // (the stage buffers are idle once the accumulator is complete),
+        // rows padded by 4 words so a warp's 16-byte stores hit distinct
+        // banks.  The cluster adds the partials below.
+        float* part = reinterpret_cast<float*>(base_ptr + SL::a);
+        for (int mt = 0; mt < MT; ++mt)
+          for (int c = 0; c < NB / 32; ++c) {
+            const int row = 128 * mt + 32 * q + lane;
+            const int col = (NB / 2) * ch + 16 * c;
+            uint32_t r[16];
+            tmem_ld_32x32b_x16(tmem_base + (static_cast<uint32_t>(32 * q) << 16) + NB * mt + col,
+                               r);
+            tmem_ld_wait();
+            float4* dst = reinterpret_cast<float4*>(part + row * (NB + 4) + col);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              dst[i] = make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
+                                   __uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3]));
+          }
+      } else if (EPI == kEpiStoreBf16) {
         for (int mt = 0; mt < MT; ++mt)
         for (int c = 0; c < NB / 32; ++c) {
           const int m = m0 + 128 * mt + 32 * q + lane;
@@ -536,6 +572,70 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
 
+  if constexpr (BSRC == kBDequant && EPI == kEpiStoreBf16) {
+    if (ks > 1) {
+      // Every thread of every CTA of the cluster passes both barriers, also
+      // after a timeout (the waits above are bounded), so none is left waiting.
+      cg::cluster_group cluster = cg::this_cluster();
+      cluster.sync();  // all partial tiles written
+      if (warp >= 2 && !*abort_flag) {
+        // CTA `rank` adds rows [r0, r1) of the tile over the cluster's CTAs
+        // in rank order and stores them (consecutive threads: consecutive
+        // columns).
+        // Four consecutive columns per thread and four such pieces in flight
+        // (distributed shared memory loads have a long latency).
+        constexpr int kRows = MT * BM;
+        constexpr int kN4 = NB / 4;
+        const int r0 = rank * kRows / ks, r1 = (rank + 1) * kRows / ks;
+        const int total = (r1 - r0) * kN4;
+        float* part = reinterpret_cast<float*>(base_ptr + SL::a);
+        for (int e0 = threadIdx.x - 64; e0 < total; e0 += 4 * 256) {
+          float4 v[4];
+          int off[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int e = e0 + 256 * u;
+            off[u] = e < total ? (r0 + e / kN4) * (NB + 4) + 4 * (e % kN4) : -1;
+            v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+          }
+          for (int p = 0; p < ks; ++p) {  // rank order: the sum is deterministic
+            const float* peer = cluster.map_shared_rank(part, p);
+            float4 t[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+              if (off[u] >= 0) t[u] = *reinterpret_cast<const float4*>(peer + off[u]);
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+              if (off[u] >= 0) {
+                v[u].x += t[u].x;
+                v[u].y += t[u].y;
+                v[u].z += t[u].z;
+                v[u].w += t[u].w;
+              }
+          }
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            if (off[u] < 0) continue;
+            const int row = off[u] / (NB + 4), col = off[u] % (NB + 4);
+            const int m = m0 + row, n = n0 + col;
+            if (m >= M || n >= N) continue;
+            __nv_bfloat16* dst = y + static_cast<size_t>(m) * N + n;
+            const __nv_bfloat162 lo = __floats2bfloat162_rn(v[u].x, v[u].y);
+            const __nv_bfloat162 hi = __floats2bfloat162_rn(v[u].z, v[u].w);
+            if (n + 4 <= N && (N & 3) == 0) {
+              *reinterpret_cast<uint2*>(dst) =
+                  make_uint2(*reinterpret_cast<const uint32_t*>(&lo),
+                             *reinterpret_cast<const uint32_t*>(&hi));
+            } else {
+              const float f[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+              for (int i = 0; i < 4 && n + i < N; ++i) dst[i] = __float2bfloat16_rn(f[i]);
+            }
+          }
+        }
+      }
+      cluster.sync();  // peers keep their partials until every reader is done
+    }
+  }
   tc_fence_before();
   __syncthreads();
   if (threadIdx.x == 0) pdl_launch_dependents();
@@ -572,7 +672,7 @@ const GemmGroup kNoGroup = {};
 template <auto kern, size_t kSmemBytes>
 cudaError_t launch_gemm(dim3 grid, bool pdl, cudaStream_t stream, const CUtensorMap& ta,
                         const CUtensorMap& tb, const GemmGroup& grp, const SumSqArgs& ss, int M,
-                        int N, int K, int pdl_static, unsigned* err) {
+                        int N, int K, int pdl_static, unsigned* err, int cluster = 1) {
   // The opt-in shared-memory size is a per-device function attribute; set it
   // once per device and kernel instantiation.
   static unsigned long long attr_done = 0;  // bit d: device d
@@ -590,13 +690,22 @@ cudaError_t launch_gemm(dim3 grid, bool pdl, cudaStream_t stream, const CUtensor
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = kSmemBytes;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
+  int na = 0;
   if (pdl) {
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
   }
+  if (cluster > 1) {
+    attr[na].id = cudaLaunchAttributeClusterDimension;
+    attr[na].val.clusterDim.x = cluster;
+    attr[na].val.clusterDim.y = 1;
+    attr[na].val.clusterDim.z = 1;
+    ++na;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = na;
   return cudaLaunchKernelEx(&cfg, kern, ta, tb, grp, ss, M, N, K, pdl_static, err);
 }
 
@@ -627,11 +736,25 @@ cudaError_t launch_prefill_gemm_group(const PrefillItem* items_in, int count, in
     // dequantization scales with NB and the MMAs with MT x NB.  The group's
     // tiles count in units of its longest K; the shape with the smallest
     // waves x wave time wins, on equal cost the earlier (larger) one.
-    struct Shape { int mt, nb, cost; };
-    const Shape shapes[4] = {{2, 256, 132}, {1, 256, 100}, {2, 128, 80}, {1, 128, 68}};
+    //
+    // A group whose best unsplit launch fills less than half the SMs also
+    // considers splitting K over a cluster of ks CTAs (ks <= 4, at least 2
+    // k-blocks each, the fp32 partial tile fitting the stage buffers): ks x
+    // the CTAs, each 1/ks of the K loop, plus about 15 % for writing and
+    // adding the partials through distributed shared memory.
+    struct Shape { int mt, nb, cost; size_t stage_bytes; };
+    const Shape shapes[4] = {
+        {2, 256, 132, SmemLayout<2, 256>::kStages * size_t(Tile<2, 256>::kTileABytes + Tile<2, 256>::kTileBBytes)},
+        {1, 256, 100, SmemLayout<1, 256>::kStages * size_t(Tile<1, 256>::kTileABytes + Tile<1, 256>::kTileBBytes)},
+        {2, 128, 80, SmemLayout<2, 128>::kStages * size_t(Tile<2, 128>::kTileABytes + Tile<2, 128>::kTileBBytes)},
+        {1, 128, 68, SmemLayout<1, 128>::kStages * size_t(Tile<1, 128>::kTileABytes + Tile<1, 128>::kTileBBytes)}};
     const int k_max = items[0].K;
-    int best = -1;
-    long best_cost = 0;
+    int kb_min = 1 << 30;
+    for (int i = 0; i < n; ++i) kb_min = items[i].K / BK < kb_min ? items[i].K / BK : kb_min;
+    int best = -1, best_ks = 1;
+    double best_cost = 0.0;
+    bool allow_split = false;
+    for (int pass = 0; pass < 2; ++pass) {
     for (int si = 0; si < 4; ++si) {
       const Shape sh = shapes[si];
       if (sh.mt == 2 && M < 2 * BM) continue;  // 256-row tiles only when rows fill them
@@ -639,14 +762,22 @@ cudaError_t launch_prefill_gemm_group(const PrefillItem* items_in, int count, in
       for (int i = 0; i < n; ++i)
         eq += static_cast<double>((items[i].N + sh.nb - 1) / sh.nb) *
               ((M + sh.mt * BM - 1) / (sh.mt * BM)) * items[i].K / k_max;
-      const long cost = static_cast<long>(std::ceil(eq / sms - 1e-9)) * sh.cost;
-      if (best < 0 || cost < best_cost) {
-        best = si;
-        best_cost = cost;
+      const size_t part_bytes = static_cast<size_t>(sh.mt) * BM * (sh.nb + 4) * 4;
+      for (int ks = pass == 0 ? 1 : 2; ks <= (pass == 0 ? 1 : 4); ++ks) {
+        if (ks > 1 && (!allow_split || part_bytes > sh.stage_bytes || kb_min < 2 * ks)) break;
+        const double cost = std::ceil(eq * ks / sms - 1e-9) * sh.cost / ks * (ks > 1 ? 1.15 : 1.0);
+        if (best < 0 || cost < best_cost - 1e-9) {
+          best = si;
+          best_ks = ks;
+          best_cost = cost;
+          if (pass == 0) allow_split = eq * 2 < sms;
+        }
       }
+    }
     }
     if (best < 0) best = 1;
     const int mt = shapes[best].mt, nb = shapes[best].nb;
+    const int ks = best_ks;
     const int bm = mt * BM;
     GemmGroup grp;
     grp.count = n;
@@ -671,16 +802,17 @@ cudaError_t launch_prefill_gemm_group(const PrefillItem* items_in, int count, in
     }
     CUtensorMap none = grp.ta[0];  // unused by the dequantizing variant
     SumSqArgs ss = {};
-    dim3 grid(grp.tile_start[n], 1, 1);
+    if (static_cast<long>(grp.tile_start[n]) * ks > 0x7FFFFFFFL) return cudaErrorInvalidValue;
+    dim3 grid(grp.tile_start[n] * ks, 1, 1);
     const int ps = (pdl && static_w) ? 1 : 0;
     cudaError_t e;
 #define W4_PREFILL_LAUNCH(MT_, NB_)                                                           \
   (sym ? launch_gemm<gemm_tc_kernel<kBDequant, kEpiStoreBf16, true, MT_, NB_>,                \
                      SmemLayout<MT_, NB_>::bytes>(grid, pdl, stream, none, none, grp, ss, M, 0, \
-                                                  0, ps, err)                                 \
+                                                  0, ps, err, ks)                             \
        : launch_gemm<gemm_tc_kernel<kBDequant, kEpiStoreBf16, false, MT_, NB_>,               \
                      SmemLayout<MT_, NB_>::bytes>(grid, pdl, stream, none, none, grp, ss, M, 0, \
-                                                  0, ps, err))
+                                                  0, ps, err, ks))
     if (mt == 2 && nb == 256) e = W4_PREFILL_LAUNCH(2, 256);
     else if (mt == 2) e = W4_PREFILL_LAUNCH(2, 128);
     else if (nb == 256) e = W4_PREFILL_LAUNCH(1, 256);
