@@ -588,3 +588,51 @@ def test_linear_batched_qwen_block(m, sym, kernel):
     torch.cuda.synchronize()
     for (x, qw, sc, zr, y), ref in zip(items, refs):
         assert max_rel_err(y, ref) <= Y_RTOL
+
+
+# --------------------------------------------- bench configuration ----
+
+def test_bench_configuration_sampled():
+    """The bench's launch configuration at full size: 28 Qwen3-1.7B-shaped
+    blocks (196 linears, bf16 N(0, 0.02)), one batched quantize+pack and one
+    batched decode per token count (M = 1, 4, 8) with programmatic dependent
+    launch and static weights, as bench.py times them.  Sampled rows of
+    sampled linears are checked against the oracle: codes, scales and zeros
+    bit-exact, y within the linear bound."""
+    rng = np.random.default_rng(2024)
+    g = torch.Generator(device=DEV)
+    lin = []
+    for b in range(28):
+        for i, (_name, k, n) in enumerate(synth.QWEN3_1P7B_BLOCK):
+            g.manual_seed(5000 + 7 * b + i)
+            w = (torch.randn(n, k, generator=g, device=DEV) * 0.02).to(torch.bfloat16)
+            qw = torch.empty(n, k // 8, dtype=torch.int32, device=DEV)
+            sc = torch.empty(n, k // 128, dtype=torch.int16, device=DEV)
+            zr = torch.empty(n, k // 128, dtype=torch.int16, device=DEV)
+            lin.append((k, n, w, qw, sc, zr))
+    w4.quantize_pack_batched([(w, None, 1.0, qw, sc, zr) for (k, n, w, qw, sc, zr) in lin], False)
+    flags = w4.LINEAR_PDL | w4.LINEAR_STATIC_WEIGHTS
+    xs = {}
+    ys = {}
+    for m in (1, 4, 8):
+        for k in {k for k, *_ in lin}:
+            g.manual_seed(77 + 10 * m + k)
+            xs[(m, k)] = torch.randn(m, k, generator=g, device=DEV).to(torch.bfloat16)
+        ys[m] = [torch.empty(m, n, dtype=torch.bfloat16, device=DEV) for (k, n, *_r) in lin]
+        w4.w4a16_linear_batched([(xs[(m, k)], qw, sc, zr, y) for (k, n, w, qw, sc, zr), y in
+                                 zip(lin, ys[m])], m, flags)
+    torch.cuda.synchronize()
+    for j in rng.choice(len(lin), 12, replace=False):
+        k, n, w, qw, sc, zr = lin[j]
+        rows = np.sort(rng.choice(n, 16, replace=False))
+        rt = torch.as_tensor(rows, device=DEV)
+        wb = synth.bits(w[rt].cpu())
+        oq, os_, oz = O.quantize_pack(wb, False)
+        assert np.array_equal(qw[rt].cpu().numpy(), oq)
+        assert np.array_equal(u16(sc[rt]), os_)
+        assert np.array_equal(u16(zr[rt]), oz)
+        what = O.dequantize(*O.quantize_rtn(wb, False))
+        for m in (1, 4, 8):
+            ref = O.linear(synth.bits(xs[(m, k)].cpu()), what)
+            y = ys[m][j][:, rt]
+            assert max_rel_err(y, ref) <= Y_RTOL, (j, m)
