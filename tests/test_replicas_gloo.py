@@ -37,7 +37,7 @@ def _rank(rank, world, port, out):
 
 def test_two_replicas_take_the_slowest_rank():
     world = 2
-    out = mp.Manager().dict()
+    out = mp.get_context("spawn").Manager().dict()  # no fork of this process
     mp.start_processes(_rank, args=(world, _free_port(), out), nprocs=world, join=True,
                        start_method="spawn")
     assert out[0] == out[1]
