@@ -634,7 +634,10 @@ def main():
     }
     if rank == 0 and world == 1 and not args.no_cpu:
         out["cpu_baseline"] = cpu_baseline()
-    if rank == 0 and not args.no_breakdown:
+    # The breakdown (about a minute of single-GPU measurements) runs only at
+    # N = 1: under torchrun the other ranks would wait for it at the final
+    # barrier against the process group's timeout.
+    if rank == 0 and world == 1 and not args.no_breakdown:
         del g_q, g_d, model
         torch.cuda.empty_cache()
         out["breakdown"] = breakdown(torch, dev, hbm, bf16_peak, bf16_sus)
