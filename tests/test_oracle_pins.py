@@ -523,3 +523,18 @@ def test_act_int8_ties_to_even_hand_case():
     q, sc = O.quantize_act_int8(f32_bits_to_bf16_exact(vals))
     assert sc[0] == np.float32(1.0)
     assert q[0, :8].tolist() == [127, 0, 2, 2, 0, -2, 4, -127]
+
+
+def test_storage_accounting():
+    """Stored bytes per weight of the packed format: 4 bits of code plus an
+    fp16 scale (and an fp16 zero when asymmetric) per 128 weights, i.e.
+    0.53125 B/weight asymmetric and 0.515625 symmetric; the symmetric rate
+    applied to the 27B card's 12.56 GB of int4 linears gives about 24.4e9
+    parameters (a plausibility check of a 27B-class model, not a pin of the
+    card's own packing, which it does not state)."""
+    w = synth.bits(synth.normal_weight(16, 384, 0.02, seed=81))
+    for sym, rate in ((False, 0.53125), (True, 0.515625)):
+        qw, s16, z16 = O.quantize_pack(w, sym)
+        stored = qw.nbytes + s16.nbytes + (0 if z16 is None else z16.nbytes)
+        assert stored == rate * w.size
+    assert 24.0e9 < 12.56e9 / 0.515625 < 24.8e9
