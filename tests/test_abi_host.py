@@ -164,3 +164,48 @@ def test_w4a8_validation(L):
     it = (w4.A8Item * 2)(w4.A8Item(A, A, A, A, A, None, 8, 128, B),
                          w4.A8Item(A, A, A, A, A, A, 8, 128, B))
     assert L.w4a8_linear_batched(it, 2, 1, 128, 0, None) == 1             # mixed symmetry
+
+
+def test_binding_refuses_missized_companion_tensors(monkeypatch):
+    """The C ABI takes bare pointers; the binding checks the shapes of every
+    companion tensor before any call (CPU tensors here: the C library is
+    replaced by a stub that must not be reached)."""
+    import torch
+    import weight_only_int4_quantize_b200 as w4
+
+    class NoCall:
+        def __getattr__(self, name):
+            raise AssertionError(f"{name} reached with mis-sized inputs")
+
+    monkeypatch.setattr(w4, "_cuda", lambda t, dtype, name: t)
+    monkeypatch.setattr(w4, "lib", lambda: NoCall())
+    x = torch.zeros(4, 256, dtype=torch.bfloat16)
+    qw = torch.zeros(8, 32, dtype=torch.int32)
+    sc = torch.zeros(8, 2, dtype=torch.int16)
+    with pytest.raises(ValueError):
+        w4.w4a16_linear(x, qw, torch.zeros(8, 3, dtype=torch.int16))
+    with pytest.raises(ValueError):
+        w4.w4a16_linear(x, qw, sc, torch.zeros(7, 2, dtype=torch.int16))
+    with pytest.raises(ValueError):
+        w4.w4a16_linear(x, qw, sc, out=torch.zeros(4, 9, dtype=torch.bfloat16))
+    with pytest.raises(ValueError):
+        w4.linear_items([(x, qw, sc, None, torch.zeros(4, 8, dtype=torch.bfloat16))], m=5)
+    with pytest.raises(ValueError):
+        w4.linear_items([(x, qw, sc, None, torch.zeros(3, 8, dtype=torch.bfloat16))])
+    xq = torch.zeros(4, 256, dtype=torch.int8)
+    with pytest.raises(ValueError):
+        w4.w4a8_linear(xq, torch.zeros(4, 3, dtype=torch.int32), torch.zeros(4), qw, sc)
+    with pytest.raises(ValueError):
+        w4.w4a8_linear(xq, torch.zeros(4, 2, dtype=torch.int32), torch.zeros(5), qw, sc)
+    with pytest.raises(ValueError):
+        w4.a8_items([(xq, torch.zeros(4, 2, dtype=torch.int32), torch.zeros(4), qw,
+                      torch.zeros(8, 1, dtype=torch.int16), None,
+                      torch.zeros(4, 8, dtype=torch.bfloat16))])
+    with pytest.raises(ValueError):
+        w4.quantize_pack_items([(torch.zeros(8, 256, dtype=torch.bfloat16), torch.zeros(255),
+                                 1.0, qw, sc, None)])
+    with pytest.raises(ValueError):
+        w4.quantize_pack(torch.zeros(8, 256, dtype=torch.bfloat16), False,
+                         awq_s=torch.zeros(128))
+    with pytest.raises(ValueError):
+        w4.awq_clip_search_rows(x, torch.zeros(8, 128, dtype=torch.bfloat16), [1.0], False)

@@ -150,6 +150,13 @@ def _cuda(t, dtype, name):
     return t
 
 
+def _expect(t, shape, name):
+    """Shape check of a companion tensor: the C ABI takes bare pointers and
+    cannot see a mis-sized buffer, so the binding refuses it here."""
+    if t is not None and tuple(t.shape) != tuple(int(v) for v in shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
 def quantize_pack(w, symmetric: bool, awq_s=None, shrink: float = 1.0, group: int = 128):
     """RTN int4 g128 quantize+pack of a bf16 [N, K] weight on its device.
 
@@ -160,6 +167,7 @@ def quantize_pack(w, symmetric: bool, awq_s=None, shrink: float = 1.0, group: in
     n, k = w.shape
     if awq_s is not None:
         _cuda(awq_s, torch.float32, "awq_s")
+        _expect(awq_s, (k,), "awq_s")
     qw = torch.empty((n, k // 8), dtype=torch.int32, device=w.device)
     sc = torch.empty((n, k // group), dtype=torch.int16, device=w.device)
     zr = None if symmetric else torch.empty((n, k // group), dtype=torch.int16, device=w.device)
@@ -183,6 +191,7 @@ def quantize_pack_rows(w, symmetric: bool, shrink_rows, awq_s=None, group: int =
         raise ValueError("shrink_rows needs one ratio per output row")
     if awq_s is not None:
         _cuda(awq_s, torch.float32, "awq_s")
+        _expect(awq_s, (k,), "awq_s")
     qw = torch.empty((n, k // 8), dtype=torch.int32, device=w.device)
     sc = torch.empty((n, k // group), dtype=torch.int16, device=w.device)
     zr = None if symmetric else torch.empty((n, k // group), dtype=torch.int16, device=w.device)
@@ -207,6 +216,11 @@ def w4a16_linear(x, qweight, scales, zeros=None, flags: int = 0, group: int = 12
     n = qweight.shape[0]
     if qweight.shape[1] * 8 != k:
         raise ValueError("qweight does not match x's K")
+    _expect(scales, (n, k // group), "scales")
+    _expect(zeros, (n, k // group), "zeros")
+    if out is not None:
+        _cuda(out, torch.bfloat16, "out")
+        _expect(out, (m, n), "out")
     y = out if out is not None else torch.empty((m, n), dtype=torch.bfloat16, device=x.device)
     with torch.cuda.device(x.device):
         st = lib().w4a16_linear(x.data_ptr(), m, qweight.data_ptr(), scales.data_ptr(),
@@ -234,6 +248,11 @@ def quantize_pack_items(items):
     (w, awq_s or None, shrink, qweight, scales, zeros or None) tuples."""
     arr = (QuantItem * len(items))()
     for a, (w, s, r, qw, sc, zr) in zip(arr, items):
+        n, k = w.shape
+        _expect(s, (k,), "awq_s")
+        _expect(qw, (n, k // 8), "qweight")
+        _expect(sc, (n, k // 128), "scales")
+        _expect(zr, (n, k // 128), "zeros")
         a.w_bf16, a.N, a.K = w.data_ptr(), w.shape[0], w.shape[1]
         a.awq_s = None if s is None else s.data_ptr()
         a.shrink = float(r)
@@ -254,10 +273,19 @@ def quantize_pack_batched(items, symmetric: bool, group: int = 128, stream=None)
     _check(st, "w4_quantize_pack_batched")
 
 
-def linear_items(items):
-    """ctypes array of LinearItem from (x, qweight, scales, zeros or None, y) tuples."""
+def linear_items(items, m=None):
+    """ctypes array of LinearItem from (x, qweight, scales, zeros or None, y)
+    tuples (x [M, K], y [M, N]; with m given, M must equal it)."""
     arr = (LinearItem * len(items))()
     for a, (x, qw, sc, zr, y) in zip(arr, items):
+        mm, k = x.shape
+        n = qw.shape[0]
+        if m is not None and mm != m:
+            raise ValueError(f"x has {mm} rows, the call has {m}")
+        _expect(qw, (n, k // 8), "qweight")
+        _expect(sc, (n, k // 128), "scales")
+        _expect(zr, (n, k // 128), "zeros")
+        _expect(y, (mm, n), "y")
         a.x_bf16, a.qweight, a.scales_f16 = x.data_ptr(), qw.data_ptr(), sc.data_ptr()
         a.zeros_f16 = None if zr is None else zr.data_ptr()
         a.N, a.K, a.y_bf16 = qw.shape[0], x.shape[1], y.data_ptr()
@@ -269,7 +297,7 @@ def w4a16_linear_batched(items, m: int, flags: int = 0, group: int = 128, stream
     items are (x, qweight, scales, zeros or None, y) tuples of CUDA tensors or
     a prepared linear_items() array."""
     torch = _torch()
-    arr = items if isinstance(items, ctypes.Array) else linear_items(items)
+    arr = items if isinstance(items, ctypes.Array) else linear_items(items, m)
     st = lib().w4a16_linear_batched(ctypes.addressof(arr), len(arr), int(m), group, int(flags),
                                     stream if stream is not None else _stream(torch.cuda.current_device()))
     _check(st, "w4a16_linear_batched")
@@ -304,6 +332,14 @@ def w4a8_linear(xq, xsum, xscale, qweight, scales, zeros=None, flags: int = 0, g
         _cuda(zeros, torch.int16, "zeros")
     m, k = xq.shape
     n = qweight.shape[0]
+    _expect(xsum, (m, k // 128), "xsum")
+    _expect(xscale, (m,), "xscale")
+    _expect(qweight, (n, k // 8), "qweight")
+    _expect(scales, (n, k // group), "scales")
+    _expect(zeros, (n, k // group), "zeros")
+    if out is not None:
+        _cuda(out, torch.bfloat16, "out")
+        _expect(out, (m, n), "out")
     y = out if out is not None else torch.empty((m, n), dtype=torch.bfloat16, device=xq.device)
     with torch.cuda.device(xq.device):
         st = lib().w4a8_linear(xq.data_ptr(), xsum.data_ptr(), xscale.data_ptr(), m,
@@ -321,10 +357,20 @@ class A8Item(ctypes.Structure):
                 ("y_bf16", ctypes.c_void_p)]
 
 
-def a8_items(items):
+def a8_items(items, m=None):
     """Host array of w4a8_item from (xq, xsum, xscale, qweight, scales, zeros, y) tuples."""
     arr = (A8Item * len(items))()
     for i, (xq, xs, sc_x, qw, sc, zr, y) in enumerate(items):
+        mm, k = xq.shape
+        n = qw.shape[0]
+        if m is not None and mm != m:
+            raise ValueError(f"xq has {mm} rows, the call has {m}")
+        _expect(xs, (mm, k // 128), "xsum")
+        _expect(sc_x, (mm,), "xscale")
+        _expect(qw, (n, k // 8), "qweight")
+        _expect(sc, (n, k // 128), "scales")
+        _expect(zr, (n, k // 128), "zeros")
+        _expect(y, (mm, n), "y")
         arr[i] = A8Item(xq.data_ptr(), xs.data_ptr(), sc_x.data_ptr(), qw.data_ptr(),
                         sc.data_ptr(), None if zr is None else zr.data_ptr(), qw.shape[0],
                         xq.shape[1], y.data_ptr())
@@ -334,7 +380,7 @@ def a8_items(items):
 def w4a8_linear_batched(items, m: int, flags: int = 0, group: int = 128, stream=None) -> None:
     """Many independent W4A8 linears with the same token count m."""
     torch = _torch()
-    arr = items if isinstance(items, ctypes.Array) else a8_items(items)
+    arr = items if isinstance(items, ctypes.Array) else a8_items(items, m)
     st = lib().w4a8_linear_batched(ctypes.addressof(arr), len(arr), int(m), group, int(flags),
                                    stream if stream is not None else _stream(torch.cuda.current_device()))
     _check(st, "w4a8_linear_batched")
@@ -369,6 +415,7 @@ def awq_score_grid(x, w, alphas, shrinks, symmetric: bool, seg_offsets=None, wor
     _cuda(w, torch.bfloat16, "w")
     m, k = x.shape
     n = w.shape[0]
+    _expect(w, (n, k), "w")
     a = np.ascontiguousarray(np.asarray(alphas, dtype=np.float32))
     r = np.ascontiguousarray(np.asarray(shrinks, dtype=np.float32))
     if seg_offsets is None:
@@ -409,6 +456,8 @@ def awq_clip_search_rows(x, w, shrinks, symmetric: bool, awq_s=None, workspace=N
         _cuda(awq_s, torch.float32, "awq_s")
     m, k = x.shape
     n = w.shape[0]
+    _expect(w, (n, k), "w")
+    _expect(awq_s, (k,), "awq_s")
     r = np.ascontiguousarray(np.asarray(shrinks, dtype=np.float32))
     if workspace is None:
         workspace = torch.empty(clip_rows_workspace_bytes(m, n, k, len(r)), dtype=torch.uint8,
@@ -440,6 +489,7 @@ def awq_score_grid_static_scratch(x, w, alphas, shrinks, symmetric: bool, seg_of
     _cuda(w, torch.bfloat16, "w")
     m, k = x.shape
     n = w.shape[0]
+    _expect(w, (n, k), "w")
     a = np.ascontiguousarray(np.asarray(alphas, dtype=np.float32))
     r = np.ascontiguousarray(np.asarray(shrinks, dtype=np.float32))
     seg = None if seg_offsets is None else np.ascontiguousarray(np.asarray(seg_offsets, dtype=np.int64))
