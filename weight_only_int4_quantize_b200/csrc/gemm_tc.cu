@@ -22,7 +22,7 @@
 //
 // Every mbarrier wait is bounded (w4_common.cuh); a CTA that gives up sets
 // the device error word, drains its own TMA loads and MMAs, frees its TMEM
-// and returns.  No TMA multicast.
+// and returns.  Every TMA load feeds only its own CTA.
 #include <cooperative_groups.h>
 #include <cudaTypedefs.h>
 

@@ -26,7 +26,8 @@
 // consecutive bf16 pairs and needs no permutation.
 //
 // Every wait is bounded; a CTA that gives up records it in the device error
-// word, drains its own TMA loads and returns.  No TMA multicast.
+// word, drains its own TMA loads and returns.  Every TMA load feeds only its
+// own CTA.
 #include <cooperative_groups.h>
 #include <cudaTypedefs.h>
 
