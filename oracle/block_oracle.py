@@ -33,7 +33,10 @@ the pages; these are the published Qwen3 conventions):
     output for q, k, v (shared), the attention output for o, the second norm
     output for gate, up (shared), the SwiGLU product for down;
   * loss = mean over tokens and hidden units of (candidate path - reference
-    path)^2; everything in binary64 here (the pages fix no precision).
+    path)^2; everything in binary64 here (the pages fix no precision);
+  * the search: alpha per linear group at no clipping, then one shrink ratio
+    per linear with the rest of the group unclipped, each group scored with
+    the rest of block i unquantized; the caller supplies block i's input.
 """
 from __future__ import annotations
 
@@ -123,14 +126,17 @@ def candidate_linear(w_bits: np.ndarray, s: np.ndarray, shrink: float, symmetric
 
 
 def scoring_losses(x: np.ndarray, bits_i: dict, norms_i: dict, next_block, group: str,
-                   alphas, shrinks, symmetric: bool, cfg: dict) -> np.ndarray:
+                   alphas, shrinks, symmetric: bool, cfg: dict, only: str | None = None
+                   ) -> np.ndarray:
     """loss[a, r] for every (alpha_a, shrink_r) candidate of one linear group
     of block i ([rebuttal] 'Search' row; look-ahead paragraph).
 
     x: block i's input [T, hidden] (binary64).  next_block: (bits, norms) of
     block i+1 for the look-ahead loss at its output, or None for the loss at
     block i's own output (the d=0 arm, and block 27's fallback).  Every
-    linear of the group takes the same alpha and shrink."""
+    linear of the group takes the same alpha; the shrink goes to every
+    linear of the group, or with `only` to that linear alone (the others
+    unclipped)."""
     w_ref = block_weights_f64(bits_i, norms_i)
     acts: dict = {}
     out_i = block_forward(x, w_ref, cfg, acts)
@@ -148,7 +154,33 @@ def scoring_losses(x: np.ndarray, bits_i: dict, norms_i: dict, next_block, group
         for j, r in enumerate(shrinks):
             wc = dict(w_ref)
             for name in GROUPS[group]:
-                wc[name] = candidate_linear(bits_i[name], s_all[a], float(r), symmetric)
+                ratio = float(r) if only is None or name == only else 1.0
+                wc[name] = candidate_linear(bits_i[name], s_all[a], ratio, symmetric)
             diff = path(wc) - ref
             losses[a, j] = np.mean(diff * diff)
     return losses
+
+
+def search_block(x: np.ndarray, bits_i: dict, norms_i: dict, next_block, alphas, shrinks,
+                 symmetric: bool, cfg: dict) -> dict:
+    """The search of one block ([rebuttal] 'Search' row, 'Clipping
+    granularity'): for each linear group, alpha* = the least loss over the
+    alpha grid at no clipping (shrink 1.0); then for each linear of the group
+    its own ratio r* = the least loss over the shrink grid with the group at
+    alpha* and the group's other linears unclipped.  Groups are scored one at
+    a time with the rest of block i unquantized (a candidate swaps only its
+    own weights).  Ties go to the lowest grid index.  Returns {group:
+    (alpha index, {linear: shrink index})}."""
+    one = np.array([1.0], np.float32)
+    out = {}
+    for group, names in GROUPS.items():
+        col = scoring_losses(x, bits_i, norms_i, next_block, group, alphas, one, symmetric, cfg)
+        a_star = int(np.argmin(col[:, 0]))
+        al = np.asarray(alphas, np.float32)[a_star:a_star + 1]
+        r_star = {}
+        for name in names:
+            row = scoring_losses(x, bits_i, norms_i, next_block, group, al, shrinks, symmetric,
+                                 cfg, only=name)
+            r_star[name] = int(np.argmin(row[0]))
+        out[group] = (a_star, r_star)
+    return out

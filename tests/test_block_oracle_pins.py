@@ -243,3 +243,39 @@ def test_scoring_candidate_is_the_scale_rewrite():
     wc = B.candidate_linear(bits["up"], s, 0.9, True)
     codes, s16, z16 = W4.quantize_rtn(bits["up"], True, s, 0.9)
     assert np.array_equal(wc, W4.dequantize(codes, s16, z16).astype(np.float64) / s[None, :])
+
+
+def test_search_picks_rtn_for_weights_on_the_grid():
+    """Weights already on the int4 grid are reproduced exactly only by alpha 0
+    at shrink 1.0, so the search must pick those for every group and linear,
+    with or without a next block."""
+    cfg = dict(SMALL, hidden=128, heads=4, kv_heads=2, head_dim=32, ffn=128)
+    bits, norms = _block(cfg, 20, std=0.05)
+    shapes = {"q": (128, 128), "k": (64, 128), "v": (64, 128), "o": (128, 128),
+              "gate": (128, 128), "up": (128, 128), "down": (128, 128)}
+    for i, name in enumerate(B.LINEARS):
+        bits[name] = _on_grid_bits(*shapes[name], 30 + i)
+    x = _rng(21).normal(size=(5, 128))
+    al = np.array([0.0, 0.25, 0.5], np.float32)
+    sh = np.array([0.9, 1.0, 0.8], np.float32)  # 1.0 not first: the index is checked
+    for next_block in (None, _block(cfg, 22, std=0.05)):
+        res = B.search_block(x, bits, norms, next_block, al, sh, False, cfg)
+        assert set(res) == set(B.GROUPS)
+        for group, (a_star, r_star) in res.items():
+            assert a_star == 0, group
+            assert set(r_star) == set(B.GROUPS[group])
+            assert all(j == 1 for j in r_star.values()), (group, r_star)
+
+
+def test_per_linear_shrink_touches_only_that_linear():
+    """With `only`, the other linears of the group stay unclipped: a ratio on
+    k alone gives the loss of the group with k clipped, which differs from
+    clipping the whole group and, at ratio 1.0, equals no clipping."""
+    bits, norms = _block(SMALL, 23)
+    x = _rng(24).normal(size=(4, SMALL["hidden"]))
+    al = np.array([0.5], np.float32)
+    sh = np.array([1.0, 0.7], np.float32)
+    whole = B.scoring_losses(x, bits, norms, None, "qkv", al, sh, False, SMALL)
+    k_only = B.scoring_losses(x, bits, norms, None, "qkv", al, sh, False, SMALL, only="k")
+    assert k_only[0, 0] == whole[0, 0]
+    assert k_only[0, 1] != whole[0, 1]
