@@ -1,7 +1,9 @@
 /*
  * w4.h -- C ABI of libw4: weight-only int4 group-128 quantization, the W4A16
- * linear that consumes it, and AWQ alpha/shrink candidate scoring, as
- * hand-written CUDA kernels for B200 (sm_100a).
+ * linear that consumes it (decode and prefill), the W4A8 decode over the
+ * same stored weights, AWQ alpha/shrink candidate scoring and the
+ * per-output-channel clipping search, as hand-written CUDA kernels for B200
+ * (sm_100a).
  *
  * Sources (model-card pages, cited by title and section):
  *   [rebuttal] "ghostchoir/rebuttal_w4g128_awq_w2": 'Model Details' table
@@ -10,14 +12,16 @@
  *              grid, clipping as a 10-point global shrink grid); the
  *              scale-rewrite paragraph (prev_op /= s, W *= s equals
  *              Q(W diag(s)) diag(1/s)); 'Clipping granularity' (one shrink
- *              ratio per linear); the table note defining RTN.
+ *              ratio per linear); the table note defining RTN; the
+ *              'Comparability caveat' (stock per-output-channel clipping).
  *   [qwen27b]  "GotoAI-Inc/Qwen3.6-27B-W4A16": opening paragraph (int4, group
  *              size 128, symmetric, weight-only, activations stay 16-bit).
  *   [awq-ppl]  "AWQ INT4-g128 WikiText-2 perplexity delta vs fp16, Llama-2
  *              7B": 'Methodology' (grid size 20 for the alpha search).
  *   [qsrt]     "malaiwah/GLM-5.2-QSRT-Fruit-Instruct": 'Reproducible runtime'
  *              (decode-sized batches of at most 16 rows take a separate
- *              path from prefill).
+ *              path from prefill, W4A8 there); 'What is included' and the
+ *              storage paragraph (W4A8 decode over the same stored weights).
  *
  * Conventions shared by every entry point
  *   - Device pointers are caller-owned device memory (any allocator).  Host
@@ -31,7 +35,8 @@
  *     has been synchronized.
  *   - Arguments are validated on the host before anything is launched.  A
  *     call that returns anything but W4_OK has launched nothing.
- *   - Every device base pointer must be 16-byte aligned.
+ *   - Every device base pointer must be 16-byte aligned (per-row shrink
+ *     ratios: 4-byte), unless an entry point states otherwise.
  *   - bf16 / fp16 buffers are passed as raw 16-bit patterns (void* /
  *     uint16_t*).  Inputs must be finite.
  *   - No C++ exception crosses the ABI; CUDA failures return W4_ERR_CUDA.
