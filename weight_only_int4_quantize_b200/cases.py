@@ -76,7 +76,11 @@ def main():
     ap.add_argument("--pdl", action="store_true", help="programmatic dependent launch + static weights")
     ap.add_argument("--eager", action="store_true", help="time eager launches instead of a graph")
     ap.add_argument("--a8", action="store_true", help="decode_batch: W4A8 (int8 activations)")
+    ap.add_argument("--kernel", choices=["auto", "stream", "tiled"], default="auto",
+                    help="decode kernel (linear, decode_batch)")
     a = ap.parse_args()
+    kflag = {"auto": 0, "stream": w4.LINEAR_DECODE_STREAM,
+             "tiled": w4.LINEAR_DECODE_TILED}[a.kernel]
     w = _weights(a.n, a.k, 1)
     out = {"case": a.case, "m": a.m, "n": a.n, "k": a.k, "sym": a.sym}
     if a.case == "quantize":
@@ -91,11 +95,13 @@ def main():
         x = torch.randn(a.m, a.k, generator=g, device="cuda").to(torch.bfloat16)
         y = torch.empty(a.m, a.n, dtype=torch.bfloat16, device="cuda")
         flags = (w4.LINEAR_FORCE_GEMM if a.gemm else 0) | (w4.LINEAR_FORCE_GEMV if a.gemv else 0)
+        flags |= kflag
         if a.pdl:
             flags |= w4.LINEAR_PDL | w4.LINEAR_STATIC_WEIGHTS
         ms = _time(lambda: w4.w4a16_linear(x, qw, sc, zr, flags=flags, out=y), a.iters, not a.eager)
         b = a.n * a.k * (0.5 + (2 if a.sym else 4) / 128) + 2 * a.m * (a.k + a.n)
-        out.update(ms=ms, gbs=b / ms / 1e6, tflops=2.0 * a.m * a.n * a.k / ms / 1e9)
+        out.update(ms=ms, gbs=b / ms / 1e6, tflops=2.0 * a.m * a.n * a.k / ms / 1e9,
+                   kernel=a.kernel)
     elif a.case == "decode_batch":
         # a.blocks x 7 independent linears at a.m tokens through
         # w4a16_linear_batched (asymmetric), as one decode step would run them.
@@ -112,15 +118,18 @@ def main():
                 y = torch.empty(a.m, n, dtype=torch.bfloat16, device="cuda")
                 items.append((x, qw, sc, zr, y))
                 byts += n * k * (0.5 + 4 / 128) + 2 * a.m * (k + n)
-        flags = w4.LINEAR_PDL | w4.LINEAR_STATIC_WEIGHTS if a.pdl else 0
+        flags = (w4.LINEAR_PDL | w4.LINEAR_STATIC_WEIGHTS if a.pdl else 0) | kflag
         if a.a8:  # W4A8: activations quantized once, outside the timed launches
-            arr = w4.a8_items([(*w4.quantize_act_int8(x), qw, sc, zr, y)
-                               for (x, qw, sc, zr, y) in items])
+            # (the activation tensors stay referenced: the item array holds
+            # raw pointers only)
+            acts = [w4.quantize_act_int8(x) for (x, *_r) in items]
+            arr = w4.a8_items([(*q8, qw, sc, zr, y)
+                               for q8, (x, qw, sc, zr, y) in zip(acts, items)])
             ms = _time(lambda: w4.w4a8_linear_batched(arr, a.m, flags), a.iters, not a.eager)
         else:
             arr = w4.linear_items(items)
             ms = _time(lambda: w4.w4a16_linear_batched(arr, a.m, flags), a.iters, not a.eager)
-        out.update(ms=ms, gbs=byts / ms / 1e6, linears=len(items), a8=a.a8)
+        out.update(ms=ms, gbs=byts / ms / 1e6, linears=len(items), a8=a.a8, kernel=a.kernel)
     elif a.case == "clip_rows":
         g = torch.Generator(device="cuda")
         g.manual_seed(3)

@@ -49,11 +49,10 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool v
                "r"(valid ? 16 : 0)
                : "memory");
 }
-// 4-byte asynchronous copy global -> shared (cached in L1), zero-filled when
-// `valid` is false.
-__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src, bool valid) {
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst), "l"(src),
-               "r"(valid ? 4 : 0)
+// 4-byte asynchronous copy global -> shared (cached in L1) of which the
+// first `bytes` (0, 2 or 4) are read and the rest is zero-filled.
+__device__ __forceinline__ void cp_async4_part(uint32_t dst, const void* src, uint32_t bytes) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst), "l"(src), "r"(bytes)
                : "memory");
 }
 __device__ __forceinline__ uint32_t lds32s(uint32_t addr) {
@@ -220,18 +219,19 @@ __global__ void __launch_bounds__(kStreamThreads, MIN_CTAS)
 
   // ---- load side: S groups ahead of the compute side -------------------
   // Per group lane t copies 16 bytes of rows g and g + 8 of each tile, and
-  // per tile one 4-byte word holding t = 0: scale of row g, 1: scale of row
-  // g + 8, 2: zero of row g, 3: zero of row g + 8 (the aligned word around
-  // the 2-byte value: it lies inside the tensor's 16-byte aligned storage).
-  // Rows beyond N copy nothing (zero fill) from row 0's address.
+  // per tile the aligned 4-byte word holding t = 0: the scale of row g, 1:
+  // the scale of row g + 8, 2: the zero of row g, 3: the zero of row g + 8
+  // (only the value's own two bytes are read: from an even element index the
+  // word's first two, from an odd one all four).  Rows beyond N copy nothing
+  // (zero fill) from row 0's address.
   UnitPos lp{0, 0, 1, 0, 0, 0, 0};
   const uint8_t* lw = nullptr;   // this lane's bytes of row 16*0 + g at group lp.g
   const uint8_t* lw0 = nullptr;  // the same bytes of row 0 (source of skipped copies)
-  const uint16_t* ls = nullptr;  // this lane's scale/zero value (tile 0) at group lp.g
-  const uint16_t* ls0 = nullptr;
+  const uint8_t* lsp[kTiles];    // per tile: the aligned word holding this lane's value
+  uint32_t lsv = 0;              // bit rt: this lane's value row of tile rt in range
+  uint32_t lpar = 0;             // parity of the element index of this lane's values
   size_t lrow8 = 0;              // 8 rows of codes, in bytes
-  int lsrow16 = 0;               // 16 rows of scales, in elements
-  uint32_t lvalid = 0;           // bit 2*rt+h: row 16rt + 8h + g in range; bit 8+rt: value row
+  uint32_t lvalid = 0;           // bit 2*rt+h: row 16rt + 8h + g in range
   auto load_enter = [&](int bundle) {
     enter_bundle(b, lp, bundle, warp, units);
     if (lp.bundle >= units) return;
@@ -239,23 +239,27 @@ __global__ void __launch_bounds__(kStreamThreads, MIN_CTAS)
     const int N = b.N[lp.item];
     const int G = K >> 7;
     const int row = lp.rb * (16 * kTiles) + g;
+    const int vrow = row + 8 * (t & 1);  // the row of this lane's value
     lvalid = 0;
+    lsv = 0;
 #pragma unroll
     for (int rt = 0; rt < kTiles; ++rt) {
       if (row + 16 * rt < N) lvalid |= 1u << (2 * rt);
       if (row + 16 * rt + 8 < N) lvalid |= 2u << (2 * rt);
-      if (row + 16 * rt + 8 * (t & 1) < N && (t < 2 || !SYM)) lvalid |= 256u << rt;
+      if (vrow + 16 * rt < N && (t < 2 || !SYM)) lsv |= 1u << rt;
     }
     lrow8 = static_cast<size_t>(K) * 4;
     lw0 = b.qw[lp.item] + lp.g * 64 + 16 * t;
     lw = lw0 + static_cast<size_t>(row) * (K >> 1);
     const uint16_t* base = (t < 2 || SYM) ? b.scales[lp.item] : b.zeros[lp.item];
-    ls0 = base + lp.g;
-    ls = ls0 + static_cast<size_t>(row + 8 * (t & 1)) * G;
-    lsrow16 = 16 * G;
-  };
-  auto align4 = [](const uint16_t* p) {
-    return reinterpret_cast<const void*>(reinterpret_cast<uintptr_t>(p) & ~uintptr_t{3});
+    const size_t e0 = static_cast<size_t>(vrow) * G + lp.g;  // tile 0 (rows 16 G apart)
+    lpar = static_cast<uint32_t>(e0 & 1);
+#pragma unroll
+    for (int rt = 0; rt < kTiles; ++rt) {
+      const size_t e = ((lsv >> rt) & 1u) ? e0 + static_cast<size_t>(16 * rt) * G
+                                          : static_cast<size_t>(lp.g);
+      lsp[rt] = reinterpret_cast<const uint8_t*>(base + (e & ~size_t{1}));
+    }
   };
   // Requests the next group into ring slot `slot` (one commit group per
   // call, empty once the warp's list is exhausted).
@@ -273,16 +277,18 @@ __global__ void __launch_bounds__(kStreamThreads, MIN_CTAS)
           cp_async16(dst + p * 512 + lane * 16, v ? lw + p * lrow8 : lw0, v);
         }
       }
+      const uint32_t sz = 2u << lpar;  // bytes of an in-range value word
+      const uint32_t adv = lpar << 2;  // the next group's value is in the next word after an odd one
 #pragma unroll
       for (int rt = 0; rt < kTiles; ++rt) {
-        const bool v = (lvalid >> (8 + rt)) & 1u;
-        cp_async4(dst + kSlotCodes + rt * 128 + lane * 4, align4(v ? ls + rt * lsrow16 : ls0), v);
+        cp_async4_part(dst + kSlotCodes + rt * 128 + lane * 4, lsp[rt],
+                       ((lsv >> rt) & 1u) ? sz : 0u);
+        lsp[rt] += adv;
       }
+      lpar ^= 1u;
       ++lp.g;
       lw += 64;
       lw0 += 64;
-      ++ls;
-      ++ls0;
       if (lp.g == lp.ge) load_enter(lp.bundle + stride);
     }
     cp_async_commit();
@@ -303,34 +309,53 @@ __global__ void __launch_bounds__(kStreamThreads, MIN_CTAS)
   // group ahead of use; xq walks the compute list one group ahead of cp.
   // W4A8: dst[0..1] hold the 32 activation codes, dst[2].x / .y the group's
   // code sums of tokens 2t and 2t + 1 (the mma's output columns).
+  // A lane whose token is beyond M reads token M - 1 instead: its mma
+  // columns are never stored, so no zero fill and no predicate are needed.
+  // The lane's x pointer runs on through a unit and is set at unit entry.
   UnitPos xq = cp;
-  auto load_x = [&](uint4 (&dst)[4]) {
-#pragma unroll
-    for (int j = 0; j < 4; ++j) dst[j] = make_uint4(0u, 0u, 0u, 0u);
+  const int xtok = g < M ? g : M - 1;
+  const int xt0 = 2 * t < M ? 2 * t : M - 1;
+  const int xt1 = 2 * t + 1 < M ? 2 * t + 1 : M - 1;
+  const uint4* xptr = nullptr;     // this lane's x chunk of group xq.g
+  const int32_t* xsp0 = nullptr;   // W4A8: group code sums of tokens xt0, xt1 at group xq.g
+  const int32_t* xsp1 = nullptr;
+  auto x_enter = [&]() {
+    if (xq.bundle >= units) return;
+    const int K = b.K[xq.item];
     if constexpr (A8) {
-      if (xq.bundle < units) {
-        const int K = b.K[xq.item];
-        if (g < M) {
-          const uint4* xp = reinterpret_cast<const uint4*>(
-              reinterpret_cast<const int8_t*>(b.x[xq.item]) + static_cast<size_t>(g) * K +
-              xq.g * 128 + 32 * t);
-          dst[0] = __ldg(xp);
-          dst[1] = __ldg(xp + 1);
-        }
-        const int32_t* xs = b.xsum[xq.item] + xq.g;
-        if (2 * t < M) dst[2].x = static_cast<uint32_t>(__ldg(xs + static_cast<size_t>(2 * t) * (K >> 7)));
-        if (2 * t + 1 < M)
-          dst[2].y = static_cast<uint32_t>(__ldg(xs + static_cast<size_t>(2 * t + 1) * (K >> 7)));
-      }
-    } else if (xq.bundle < units && g < M) {
-      const uint4* xp = reinterpret_cast<const uint4*>(
-          b.x[xq.item] + static_cast<size_t>(g) * b.K[xq.item] + xq.g * 128 + 32 * t);
-#pragma unroll
-      for (int j = 0; j < 4; ++j) dst[j] = __ldg(xp + j);
+      xptr = reinterpret_cast<const uint4*>(reinterpret_cast<const int8_t*>(b.x[xq.item]) +
+                                            static_cast<size_t>(xtok) * K + xq.g * 128 + 32 * t);
+      xsp0 = b.xsum[xq.item] + static_cast<size_t>(xt0) * (K >> 7) + xq.g;
+      xsp1 = b.xsum[xq.item] + static_cast<size_t>(xt1) * (K >> 7) + xq.g;
+    } else {
+      xptr = reinterpret_cast<const uint4*>(b.x[xq.item] + static_cast<size_t>(xtok) * K +
+                                            xq.g * 128 + 32 * t);
     }
-    if (xq.bundle < units && ++xq.g == xq.ge) enter_bundle(b, xq, xq.bundle + stride, warp, units);
+  };
+  auto load_x = [&](uint4 (&dst)[4]) {
+    if (xq.bundle >= units) return;
+    if constexpr (A8) {
+      dst[0] = __ldg(xptr);
+      dst[1] = __ldg(xptr + 1);
+      dst[2].x = static_cast<uint32_t>(__ldg(xsp0));
+      dst[2].y = static_cast<uint32_t>(__ldg(xsp1));
+      xptr += 8;  // 128 int8 codes
+      ++xsp0;
+      ++xsp1;
+    } else {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) dst[j] = __ldg(xptr + j);
+      xptr += 16;  // 128 bf16 values
+    }
+    if (++xq.g == xq.ge) {
+      enter_bundle(b, xq, xq.bundle + stride, warp, units);
+      x_enter();
+    }
   };
   uint4 xnext[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) xnext[j] = make_uint4(0u, 0u, 0u, 0u);
+  x_enter();
   load_x(xnext);
   float acc[kTiles][4];
 #pragma unroll
