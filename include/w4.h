@@ -318,10 +318,9 @@ w4_status awq_score_grid(const void* x_bf16, int64_t M, const void* w_bf16, int6
 /*
  * awq_score_grid_static_scratch -- awq_score_grid without a caller-supplied
  * workspace: its scratch is a fixed device array inside the library of
- * W4_AWQ_STATIC_SCRATCH_BYTES (32 MiB).  The pages have no counterpart; the
- * candidates, SSE table and argmins are those of awq_score_grid
- * ([rebuttal] 'Search' and the scale-rewrite paragraph), bit-identical for
- * the same inputs.
+ * W4_AWQ_STATIC_SCRATCH_BYTES (32 MiB).  The pages have no counterpart.  The
+ * candidates, SSE table and argmins are those of awq_score_grid,
+ * bit-identical for the same inputs (every reduction runs in a fixed order).
  *
  * It is for callers that cannot allocate device memory when they score: a
  * serving process whose caching allocator already holds the free HBM (for
@@ -334,13 +333,16 @@ w4_status awq_score_grid(const void* x_bf16, int64_t M, const void* w_bf16, int6
  * n_shrink, n_seg) exceeds W4_AWQ_STATIC_SCRATCH_BYTES is refused with
  * W4_ERR_WORKSPACE, nothing launched; w4_last_error() then names the needed
  * and available sizes.  Any other invalid argument returns the same status
- * as awq_score_grid would.
+ * as awq_score_grid would, checked before anything else (the scratch is
+ * not looked up then).
  *
  * Set-up: the first call on each device, with that device current, looks up
  * the scratch's device address (cudaGetSymbolAddress) and caches it; under
  * CUDA's default lazy module loading this is also when the driver reserves
  * the 32 MiB on that device.  Make that first call before any stream capture
- * begins.
+ * begins.  The cached address (like the device error word's, see
+ * w4_device_error) belongs to the device's primary context: do not use the
+ * library across cudaDeviceReset or another teardown of that context.
  *
  * Nothing in the scratch needs to start at zero: every word a kernel of the
  * call reads is written earlier in the same call, so nothing is cleared.

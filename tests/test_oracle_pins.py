@@ -280,6 +280,30 @@ def test_awq_scale_stat_and_pow_brute_force():
     assert np.all(s[0] == 1.0)
 
 
+def test_awq_scales_closed_forms():
+    """s = float32(stat ** alpha) where the power has an exact closed form:
+    alpha = 1/2 on perfect squares (s = k), alpha = 1/4 and 3/4 on 2^(4k)
+    (s = 2^k, 2^(3k)), and two roots exactly halfway between binary32
+    neighbours, which the final rounding must send to the even one:
+    sqrt((1 + 2^-24)^2) = 1 + 2^-24 -> 1.0 and
+    sqrt((1 + 3 2^-24)^2) = 1 + 3 2^-24 -> 1 + 2^-22 (both squares are exact in
+    binary64).  A stat below the floor 1e-8 takes the floor."""
+    ks = np.array([1.0, 3.0, 7.0, 12.0, 255.0, 4096.0, 0.5, 0.125])
+    s = O.awq_scales(ks * ks, [0.5])[0]
+    assert np.array_equal(s, ks.astype(np.float32))
+    p = np.array([-6, -3, 0, 1, 5, 9], dtype=np.float64)  # 2^-24 stays above the floor
+    s = O.awq_scales(2.0 ** (4 * p), [0.25, 0.75])
+    assert np.array_equal(s[0], (2.0 ** p).astype(np.float32))
+    assert np.array_equal(s[1], (2.0 ** (3 * p)).astype(np.float32))
+    t1, t3 = 1.0 + 2.0 ** -24, 1.0 + 3 * 2.0 ** -24
+    assert Fraction(t1 * t1) == Fraction(t1) ** 2 and Fraction(t3 * t3) == Fraction(t3) ** 2
+    s = O.awq_scales(np.array([t1 * t1, t3 * t3]), [0.5])[0]
+    assert s[0] == np.float32(1.0)
+    assert s[1] == np.float32(1.0 + 2.0 ** -22)
+    s = O.awq_scales(np.array([1e-12, 0.0]), [0.5])[0]
+    assert np.all(s == np.float32(1e-4))
+
+
 def _sse_exact(x_bits, w_bits, s, shrink, sym):
     codes, s16, z16 = O.quantize_rtn(w_bits, sym, s, shrink)
     what = O.dequantize(codes, s16, z16)

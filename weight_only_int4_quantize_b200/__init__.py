@@ -139,6 +139,14 @@ def _stream(device) -> int:
     return torch.cuda.current_stream(device).cuda_stream
 
 
+def _same_device(ref, **tensors):
+    """The kernels run on ref's device and write through every pointer they
+    get: all tensors of a call must live on that device."""
+    for name, t in tensors.items():
+        if t is not None and t.device != ref.device:
+            raise ValueError(f"{name} is on {t.device}, the call runs on {ref.device}")
+
+
 def _cuda(t, dtype, name):
     torch = _torch()
     if not isinstance(t, torch.Tensor) or not t.is_cuda:
@@ -413,6 +421,7 @@ def awq_score_grid(x, w, alphas, shrinks, symmetric: bool, seg_offsets=None, wor
     import numpy as np
     _cuda(x, torch.bfloat16, "x")
     _cuda(w, torch.bfloat16, "w")
+    _same_device(x, w=w)
     m, k = x.shape
     n = w.shape[0]
     _expect(w, (n, k), "w")
@@ -452,6 +461,7 @@ def awq_clip_search_rows(x, w, shrinks, symmetric: bool, awq_s=None, workspace=N
     import numpy as np
     _cuda(x, torch.bfloat16, "x")
     _cuda(w, torch.bfloat16, "w")
+    _same_device(x, w=w)
     if awq_s is not None:
         _cuda(awq_s, torch.float32, "awq_s")
     m, k = x.shape
@@ -487,6 +497,7 @@ def awq_score_grid_static_scratch(x, w, alphas, shrinks, symmetric: bool, seg_of
     import numpy as np
     _cuda(x, torch.bfloat16, "x")
     _cuda(w, torch.bfloat16, "w")
+    _same_device(x, w=w)
     m, k = x.shape
     n = w.shape[0]
     _expect(w, (n, k), "w")
@@ -502,6 +513,7 @@ def awq_score_grid_static_scratch(x, w, alphas, shrinks, symmetric: bool, seg_of
     _cuda(argmin_out, torch.int32, "argmin_out")
     if tuple(sse_out.shape) != (n_seg, len(a), len(r)) or tuple(argmin_out.shape) != (n_seg + 1, 4):
         raise ValueError("sse_out / argmin_out have the wrong shape")
+    _same_device(x, w=w, sse_out=sse_out, argmin_out=argmin_out)
     with torch.cuda.device(x.device):
         st = lib().awq_score_grid_static_scratch(
             x.data_ptr(), m, w.data_ptr(), n, k, group, int(bool(symmetric)), a.ctypes.data,

@@ -677,19 +677,20 @@ w4_status awq_score_grid_static_scratch(const void* x_bf16, int64_t M, const voi
                                         const float* alphas, int n_alpha, const float* shrinks,
                                         int n_shrink, const int64_t* seg_offsets, int n_seg,
                                         double* sse_out, int32_t* argmin_out, void* stream) {
+  // Without a workspace the shared validation checks every argument and
+  // launches nothing: any status but W4_ERR_WORKSPACE is an argument error,
+  // reported before the scratch is looked up (and reserved).
+  const w4_status pre = awq_score_grid(x_bf16, M, w_bf16, N, K, group, symmetric, alphas,
+                                       n_alpha, shrinks, n_shrink, seg_offsets, n_seg, sse_out,
+                                       argmin_out, nullptr, 0, stream);
+  if (pre != W4_ERR_WORKSPACE) return pre;
   const size_t need = w4_awq_workspace_bytes(M, N, K, n_alpha, n_shrink, n_seg);
   if (need > W4_AWQ_STATIC_SCRATCH_BYTES) {
-    // Without a workspace the shared validation reports any earlier argument
-    // error first and launches nothing; W4_ERR_WORKSPACE means only the size.
-    const w4_status st = awq_score_grid(x_bf16, M, w_bf16, N, K, group, symmetric, alphas,
-                                        n_alpha, shrinks, n_shrink, seg_offsets, n_seg, sse_out,
-                                        argmin_out, nullptr, 0, stream);
-    if (st == W4_ERR_WORKSPACE)
-      snprintf(g_last_error, sizeof(g_last_error),
-               "awq_score_grid_static_scratch: the problem needs %zu bytes of scratch, the "
-               "static scratch holds %zu; use awq_score_grid with a workspace",
-               need, static_cast<size_t>(W4_AWQ_STATIC_SCRATCH_BYTES));
-    return st;
+    snprintf(g_last_error, sizeof(g_last_error),
+             "awq_score_grid_static_scratch: the problem needs %zu bytes of scratch, the "
+             "static scratch holds %zu; use awq_score_grid with a workspace",
+             need, static_cast<size_t>(W4_AWQ_STATIC_SCRATCH_BYTES));
+    return W4_ERR_WORKSPACE;
   }
   void* scratch = nullptr;
   const w4_status st = cuda_status(awq_static_scratch_address(&scratch), "static scratch address");
