@@ -73,39 +73,64 @@ w4_status device_info(int* num_sms, unsigned** err_ptr) {
 
 bool valid_k(int64_t K) { return K >= 128 && K % 128 == 0 && K <= (int64_t{1} << 30); }
 
-// Workspace of awq_score_grid: every region 256-byte aligned.
-struct AwqWs {
-  size_t s, a, e, partials, total;
-};
-
 size_t round256(size_t b) { return (b + 255) & ~size_t{255}; }
+
+// Workspace of awq_score_grid: every region 256-byte aligned.  xpart, wpart:
+// partial column maxima of |x| and |w|; fe: the operand exponents per alpha.
+struct AwqWs {
+  size_t s, xpart, wpart, fe, a, e, partials, list, rowsum, total;
+};
 
 AwqWs awq_layout(int64_t M, int64_t N, int64_t K, int n_alpha, int n_shrink, int n_seg) {
   AwqWs w;
   w.s = 0;
-  w.a = w.s + round256(sizeof(float) * n_alpha * K);
+  w.xpart = w.s + round256(sizeof(float) * n_alpha * K);
+  w.wpart = w.xpart + round256(sizeof(float) * colmax_chunks(M) * K);
+  w.fe = w.wpart + round256(sizeof(float) * colmax_chunks(N) * K);
+  w.a = w.fe + round256(sizeof(int) * 2 * n_alpha);
   w.e = w.a + round256(sizeof(uint16_t) * M * K);
   w.partials = w.e + round256(sizeof(uint16_t) * static_cast<size_t>(n_shrink) * N * K);
   const size_t tiles = static_cast<size_t>(sumsq_tiles(static_cast<int>(M), static_cast<int>(N)));
-  w.total = w.partials + round256(sizeof(double) * n_alpha * n_shrink * n_seg * tiles);
+  w.list = w.partials + round256(sizeof(double) * n_alpha * n_shrink * n_seg * tiles);
+  w.rowsum = w.list + round256(sizeof(int) * (kExactCap + 1));
+  w.total = w.rowsum + round256(sizeof(double) * kExactCap *
+                                static_cast<size_t>(exact_token_chunks(static_cast<int>(M))) * N);
   return w;
 }
 
 // Workspace of awq_clip_search_rows: every region 256-byte aligned.
 struct ClipWs {
-  size_t ones, a, e, partials, total;
+  size_t ones, xpart, wpart, fe, a, e, partials, flags, list, rows, rowsum, total;
 };
 
 ClipWs clip_layout(int64_t M, int64_t N, int64_t K, int n_shrink) {
   ClipWs w;
   w.ones = 0;
-  w.a = w.ones + round256(sizeof(float) * K);
+  w.xpart = w.ones + round256(sizeof(float) * K);
+  w.wpart = w.xpart + round256(sizeof(float) * colmax_chunks(M) * K);
+  w.fe = w.wpart + round256(sizeof(float) * colmax_chunks(N) * K);
+  w.a = w.fe + round256(sizeof(int) * 2);
   w.e = w.a + round256(sizeof(uint16_t) * M * K);
   w.partials = w.e + round256(sizeof(uint16_t) * static_cast<size_t>(n_shrink) * N * K);
-  w.total = w.partials + round256(sizeof(double) * n_shrink *
-                                  static_cast<size_t>(colsumsq_row_tiles(static_cast<int>(M))) * N);
+  w.flags = w.partials + round256(sizeof(double) * n_shrink *
+                                   static_cast<size_t>(colsumsq_row_tiles(static_cast<int>(M))) * N);
+  w.list = w.flags + round256(static_cast<size_t>(n_shrink) * N);
+  w.rows = w.list + round256(sizeof(unsigned long long) + sizeof(int) * (2 * kMaxGrid + 1));
+  w.rowsum = w.rows + round256(sizeof(int) * static_cast<size_t>(n_shrink) * N);
+  w.total = w.rowsum + round256(sizeof(double) * n_shrink *
+                                static_cast<size_t>(exact_token_chunks(static_cast<int>(M))) * N);
   return w;
 }
+
+// Selections whose fp16 values put candidates within this relative distance
+// of the least are decided again in binary64.  Against a binary64
+// recomputation the fp16 scores differ by at most 2.9e-5 (relative) for a
+// table of 256 or more rows and 6.4e-4 for a single row (2048 tokens,
+// K = 2048, Gaussian and per-channel-scaled heavy-tailed activations); the
+// tolerances are 17x and 8x those, so that two candidates whose order the
+// fp16 values could invert are always both decided in binary64.
+constexpr double kGridTieTol = 5e-4;
+constexpr double kRowTieTol = 5e-3;
 
 }  // namespace
 }  // namespace w4
@@ -565,13 +590,23 @@ w4_status awq_score_grid(const void* x_bf16, int64_t M, const void* w_bf16, int6
   double* partials = reinterpret_cast<double*>(ws + L.partials);
   const int tiles = sumsq_tiles(static_cast<int>(M), static_cast<int>(N));
 
+  float* xpart = reinterpret_cast<float*>(ws + L.xpart);
+  float* wpart = reinterpret_cast<float*>(ws + L.wpart);
+  int* fe = reinterpret_cast<int*>(ws + L.fe);
   cudaError_t e = launch_awq_scales(x_bf16, M, K, al, s_all, s);
   if (e != cudaSuccess) return cuda_status(e, "awq scales");
+  e = launch_colmax_abs(x_bf16, M, K, xpart, s);
+  if (e != cudaSuccess) return cuda_status(e, "awq column maxima of x");
+  e = launch_colmax_abs(w_bf16, N, K, wpart, s);
+  if (e != cudaSuccess) return cuda_status(e, "awq column maxima of w");
+  e = launch_awq_exponents(xpart, colmax_chunks(M), wpart, colmax_chunks(N), s_all, n_alpha, K, fe,
+                           s);
+  if (e != cudaSuccess) return cuda_status(e, "awq operand exponents");
   for (int i = 0; i < n_alpha; ++i) {
     const float* si = s_all + static_cast<size_t>(i) * K;
-    e = launch_awq_xs(x_bf16, si, M, K, a_buf, s, sms);
+    e = launch_awq_xs(x_bf16, si, M, K, fe + 2 * i, a_buf, s, sms);
     if (e != cudaSuccess) return cuda_status(e, "awq x/s operand");
-    e = launch_awq_err(w_bf16, si, N, K, symmetric != 0, sl, e_buf, s, sms);
+    e = launch_awq_err(w_bf16, si, N, K, symmetric != 0, sl, fe + 2 * i + 1, e_buf, s, sms);
     if (e != cudaSuccess) return cuda_status(e, "awq error operand");
     e = launch_sumsq_gemm(a_buf, static_cast<int>(M), e_buf, static_cast<int>(N),
                           static_cast<int>(K), n_shrink,
@@ -579,8 +614,24 @@ w4_status awq_score_grid(const void* x_bf16, int64_t M, const void* w_bf16, int6
                           s, err);
     if (e != cudaSuccess) return cuda_status(e, "awq tcgen05 sum-of-squares GEMM");
   }
-  e = launch_awq_reduce(partials, n_alpha * n_shrink, n_seg, tiles, sse_out, s);
+  e = launch_awq_reduce(partials, n_alpha * n_shrink, n_seg, tiles, n_shrink, fe, sse_out, s);
   if (e != cudaSuccess) return cuda_status(e, "awq reduce");
+  // Near ties of any selection: those candidates' SSE again in binary64.
+  int* list = reinterpret_cast<int*>(ws + L.list);
+  int* count = list + kExactCap;
+  double* rowsum = reinterpret_cast<double*>(ws + L.rowsum);
+  e = launch_awq_flag(sse_out, n_seg, n_alpha, n_shrink, c1, kGridTieTol, kExactCap, list, count,
+                      s);
+  if (e != cudaSuccess) return cuda_status(e, "awq near-tie flags");
+  e = launch_exact_rowsse(x_bf16, static_cast<int>(M), w_bf16, static_cast<int>(N),
+                          static_cast<int>(K), s_all, sl, n_shrink, symmetric != 0, list, count,
+                          kExactCap, nullptr, nullptr, rowsum, s);
+  if (e != cudaSuccess) return cuda_status(e, "awq binary64 near-tie scores");
+  SegOffsets so;
+  for (int i = 0; i <= n_seg; ++i) so.off[i] = seg[i];
+  e = launch_awq_exact_merge(rowsum, static_cast<int>(M), static_cast<int>(N), list, count,
+                             kExactCap, n_seg, so, n_alpha * n_shrink, sse_out, s);
+  if (e != cudaSuccess) return cuda_status(e, "awq binary64 merge");
   return cuda_status(launch_awq_argmin(sse_out, n_seg, n_alpha, n_shrink, c1, argmin_out, s),
                      "awq argmin");
 }
@@ -631,17 +682,37 @@ w4_status awq_clip_search_rows(const void* x_bf16, int64_t M, const void* w_bf16
   void* a_buf = ws + L.a;
   void* e_buf = ws + L.e;
   double* partials = reinterpret_cast<double*>(ws + L.partials);
-  e = launch_awq_xs(x_bf16, sv, M, K, a_buf, s, sms);
+  float* xpart = reinterpret_cast<float*>(ws + L.xpart);
+  float* wpart = reinterpret_cast<float*>(ws + L.wpart);
+  int* fe = reinterpret_cast<int*>(ws + L.fe);
+  e = launch_colmax_abs(x_bf16, M, K, xpart, s);
+  if (e != cudaSuccess) return cuda_status(e, "clip search column maxima of x");
+  e = launch_colmax_abs(w_bf16, N, K, wpart, s);
+  if (e != cudaSuccess) return cuda_status(e, "clip search column maxima of w");
+  e = launch_awq_exponents(xpart, colmax_chunks(M), wpart, colmax_chunks(N), sv, 1, K, fe, s);
+  if (e != cudaSuccess) return cuda_status(e, "clip search operand exponents");
+  e = launch_awq_xs(x_bf16, sv, M, K, fe, a_buf, s, sms);
   if (e != cudaSuccess) return cuda_status(e, "clip search x/s operand");
-  e = launch_awq_err(w_bf16, sv, N, K, symmetric != 0, sl, e_buf, s, sms);
+  e = launch_awq_err(w_bf16, sv, N, K, symmetric != 0, sl, fe + 1, e_buf, s, sms);
   if (e != cudaSuccess) return cuda_status(e, "clip search error operand");
   e = launch_colsumsq_gemm(a_buf, static_cast<int>(M), e_buf, static_cast<int>(N),
                            static_cast<int>(K), n_shrink, partials, s, err);
   if (e != cudaSuccess) return cuda_status(e, "clip search tcgen05 column sum-of-squares GEMM");
-  return cuda_status(launch_clip_rows_select(partials, n_shrink,
-                                             colsumsq_row_tiles(static_cast<int>(M)), N, sl,
-                                             sse_rows_out, choice_out, shrink_rows_out, s),
-                     "clip search row selection");
+  e = launch_clip_rows_select(partials, n_shrink, colsumsq_row_tiles(static_cast<int>(M)), N, sl,
+                              fe, sse_rows_out, choice_out, shrink_rows_out, s);
+  if (e != cudaSuccess) return cuda_status(e, "clip search row selection");
+  // Rows with near ties: those ratios' row errors again in binary64.
+  uint8_t* flags = ws + L.flags;
+  unsigned long long* mask = reinterpret_cast<unsigned long long*>(ws + L.list);
+  int* list = reinterpret_cast<int*>(ws + L.list + sizeof(unsigned long long));
+  int* count = list + kMaxGrid;
+  int* row_counts = count + 1;  // [kMaxGrid]
+  return cuda_status(launch_clip_exact(x_bf16, static_cast<int>(M), w_bf16, static_cast<int>(N),
+                                       static_cast<int>(K), sv, sl, symmetric != 0, kRowTieTol,
+                                       sse_rows_out, choice_out, shrink_rows_out, flags, mask,
+                                       list, count, reinterpret_cast<int*>(ws + L.rows),
+                                       row_counts, reinterpret_cast<double*>(ws + L.rowsum), s),
+                     "clip search binary64 near ties");
 }
 
 w4_status w4_quantize_pack_rows(const void* w_bf16, int64_t N, int64_t K, int group,

@@ -126,19 +126,52 @@ int colsumsq_row_tiles(int M);
 
 cudaError_t launch_awq_scales(const void* x, int64_t M, int64_t K, const AlphaList& alphas,
                               float* s_out, cudaStream_t stream);
-cudaError_t launch_awq_xs(const void* x, const float* s, int64_t M, int64_t K, void* a,
-                          cudaStream_t stream, int num_sms);
+// Operand exponents (awq.cu): partial column maxima of |x| and |w| over
+// colmax_chunks(R) row chunks, then per alpha fe[2i] = f_i, fe[2i+1] = e_i.
+int colmax_chunks(int64_t R);
+cudaError_t launch_colmax_abs(const void* a, int64_t R, int64_t K, float* part,
+                              cudaStream_t stream);
+cudaError_t launch_awq_exponents(const float* xpart, int xchunks, const float* wpart, int wchunks,
+                                 const float* s_all, int n_alpha, int64_t K, int* fe,
+                                 cudaStream_t stream);
+cudaError_t launch_awq_xs(const void* x, const float* s, int64_t M, int64_t K, const int* fexp,
+                          void* a, cudaStream_t stream, int num_sms);
 cudaError_t launch_awq_err(const void* w, const float* s, int64_t N, int64_t K, bool symmetric,
-                           const ShrinkList& shrinks, void* e, cudaStream_t stream, int num_sms);
-cudaError_t launch_awq_reduce(const double* partials, int n_cand, int n_seg, int tiles,
-                              double* sse, cudaStream_t stream);
+                           const ShrinkList& shrinks, const int* eexp, void* e,
+                           cudaStream_t stream, int num_sms);
+cudaError_t launch_awq_reduce(const double* partials, int n_cand, int n_seg, int tiles, int n_r,
+                              const int* fe, double* sse, cudaStream_t stream);
 cudaError_t launch_awq_argmin(const double* sse, int n_seg, int n_a, int n_r, int c1,
                               int32_t* out, cudaStream_t stream);
 
 cudaError_t launch_clip_rows_select(const double* partials, int n_cand, int row_tiles, int64_t N,
-                                    const ShrinkList& shrinks, double* sse_rows, int32_t* choice,
-                                    float* shrink_rows, cudaStream_t stream);
+                                    const ShrinkList& shrinks, const int* fe, double* sse_rows,
+                                    int32_t* choice, float* shrink_rows, cudaStream_t stream);
 cudaError_t launch_fill_ones(float* p, int64_t n, cudaStream_t stream);
+
+// Exact (binary64) decision of near ties (awq.cu).  At most kExactCap
+// candidates of an awq_score_grid call are decided again.
+constexpr int kExactCap = 64;
+struct SegOffsets {
+  int off[17];
+};
+cudaError_t launch_exact_rowsse(const void* x, int M, const void* w, int N, int K,
+                                const float* s_all, const ShrinkList& shrinks, int n_r,
+                                bool symmetric, const int* list, const int* count, int cap,
+                                const int* rowlist, const int* rowcount, double* rowsum,
+                                cudaStream_t stream);
+cudaError_t launch_awq_flag(const double* sse, int n_seg, int n_a, int n_r, int c1, double tol,
+                            int cap, int* list, int* count, cudaStream_t stream);
+// Token chunks of the binary64 kernel: its row sums are [cap][chunks][N].
+int exact_token_chunks(int M);
+cudaError_t launch_awq_exact_merge(const double* rowsum, int M, int N, const int* list,
+                                   const int* count, int cap, int n_seg, const SegOffsets& seg,
+                                   int n_c, double* sse, cudaStream_t stream);
+cudaError_t launch_clip_exact(const void* x, int M, const void* w, int N, int K, const float* s,
+                              const ShrinkList& shrinks, bool symmetric, double tol,
+                              double* sse_rows, int32_t* choice, float* shrink_rows,
+                              uint8_t* flags, unsigned long long* mask, int* list, int* count,
+                              int* rows, int* row_counts, double* rowsum, cudaStream_t stream);
 
 // Device address of the fixed scratch behind awq_score_grid_static_scratch
 // on the current device (looked up once per device, then cached).
