@@ -2,8 +2,8 @@
  * w4.h -- C ABI of libw4: weight-only int4 group-128 quantization, the W4A16
  * linear that consumes it (decode and prefill), the W4A8 decode over the
  * same stored weights, AWQ alpha/shrink candidate scoring and the
- * per-output-channel clipping search, as hand-written CUDA kernels for B200
- * (sm_100a).
+ * per-output-channel clipping search, the block-level (look-ahead) candidate
+ * loss and search, as hand-written CUDA kernels for B200 (sm_100a).
  *
  * Sources (model-card pages, cited by title and section):
  *   [rebuttal] "ghostchoir/rebuttal_w4g128_awq_w2": 'Model Details' table
@@ -22,6 +22,8 @@
  *              (decode-sized batches of at most 16 rows take a separate
  *              path from prefill, W4A8 there); 'What is included' and the
  *              storage paragraph (W4A8 decode over the same stored weights).
+ *   [q326]     "ariacompute/qwen3-1.7b_q326_channel": the Qwen3-1.7B block
+ *              shapes used by the block-level scoring.
  *
  * Conventions shared by every entry point
  *   - Device pointers are caller-owned device memory (any allocator).  Host
@@ -399,6 +401,118 @@ w4_status awq_clip_search_rows(const void* x_bf16, int64_t M, const void* w_bf16
                                const float* shrinks, int n_shrink, double* sse_rows_out,
                                int32_t* choice_out, float* shrink_rows_out, void* workspace,
                                size_t workspace_bytes, void* stream);
+
+/*
+ * Block-level candidate scoring (binary64).
+ *
+ * [rebuttal] 'Model Details' table, row 'Search', and the paragraph under
+ * it: a candidate (alpha, shrink) for a linear group of decoder block i is
+ * scored by the mean squared difference, over tokens and hidden units,
+ * between the output of block i+1 (kept in original precision) with the
+ * candidate's quantized linears swapped into block i and the same path with
+ * block i unquantized; block i's own output when there is no successor (the
+ * last block, and the perplexity table's d=0 arm).  A candidate swaps only
+ * its linears' weights for Q_r(W diag(s)) diag(1/s) (scale-rewrite
+ * paragraph; the codes of w4_quantize_pack), s = fp32(max(stat, 1e-8)^alpha)
+ * with stat the mean |input| over tokens of the activation entering the
+ * group on the unquantized path.  Block shapes: [q326] "ariacompute/
+ * qwen3-1.7b_q326_channel" (16 query heads, 8 key/value heads of width 128,
+ * SwiGLU width 6144).  The decoder block follows the Qwen3 conventions (the
+ * pages do not give it): pre-norm RMSNorm, per-head RMSNorm of q and k, then
+ * a rotate-half rotary embedding at positions 0..T-1, causal softmax
+ * attention scaled by 1/sqrt(head_dim), query head h reading key/value head
+ * h / (heads / kv_heads), SwiGLU MLP (silu(gate) * up), residual adds.
+ *
+ * Every step runs in binary64 (the contractions on the fp64 MMA); results
+ * depend on nothing but the inputs (fixed order of every sum).
+ *
+ * Linears are numbered q 0, k 1, v 2, o 3, gate 4, up 5, down 6; groups are
+ * qkv 0 (q, k, v), o 1, gate_up 2 (gate, up), down 3.
+ */
+typedef struct {
+  int32_t hidden;     /* multiple of 128 */
+  int32_t heads;      /* query heads */
+  int32_t kv_heads;   /* key/value heads, divides heads */
+  int32_t head_dim;   /* 64 or 128; heads * head_dim a multiple of 128 */
+  int32_t ffn;        /* SwiGLU width, multiple of 128 */
+  double eps;         /* RMSNorm epsilon, > 0 */
+  double rope_theta;  /* rotary base, > 0 */
+} w4_block_config;
+
+typedef struct {
+  /* device bf16 [out, in] row-major: q [heads*head_dim, hidden], k and v
+   * [kv_heads*head_dim, hidden], o [hidden, heads*head_dim], gate and up
+   * [ffn, hidden], down [hidden, ffn] */
+  const void* q;
+  const void* k;
+  const void* v;
+  const void* o;
+  const void* gate;
+  const void* up;
+  const void* down;
+  const double* ln1;     /* device float64 [hidden]: the attention norm gain */
+  const double* ln2;     /* device float64 [hidden]: the MLP norm gain */
+  const double* q_norm;  /* device float64 [head_dim] */
+  const double* k_norm;  /* device float64 [head_dim] */
+} w4_block_weights;
+
+/* Workspace of awq_block_scoring_losses and awq_block_search for T tokens
+ * (about (2 heads T^2 + 24 T max(hidden, ffn)) * 8 bytes plus the largest
+ * group's binary64 candidate weights); 0 if cfg is NULL or T < 1. */
+size_t w4_block_workspace_bytes(const w4_block_config* cfg, int64_t T);
+
+/*
+ * awq_block_scoring_losses -- loss[a, j] of every candidate (alphas[a],
+ * shrinks[j]) of one linear group.  The shrink applies to every linear of
+ * the group, or with only >= 0 to that linear alone (the group's other
+ * linears quantized at the same alpha, unclipped).
+ *
+ * cfg            host, the block shape.
+ * x, T           device float64 [T, hidden]: block i's input; 1 <= T <= 8192.
+ * block          host struct of device pointers: block i.
+ * next           host struct: block i+1 (loss at its output), or NULL (loss
+ *                at block i's output).
+ * group          0..3.   only: -1, or a linear of the group.
+ * alphas         host float32 [n_alpha], finite; 1 <= n_alpha <= 64.
+ * shrinks        host float32 [n_shrink], each in (0, 1]; 1 <= n_shrink <= 64.
+ * symmetric      0: asymmetric with zero point; 1: symmetric.
+ * losses_out     device float64 [n_alpha, n_shrink] out.
+ * workspace      device scratch of at least w4_block_workspace_bytes(cfg, T)
+ *                bytes, 256-byte aligned.
+ * Errors: W4_ERR_INVALID_ARG (NULL pointer, group / only / grid value out of
+ * range), W4_ERR_SHAPE (a size outside the ranges above),
+ * W4_ERR_UNSUPPORTED (head_dim, grid sizes), W4_ERR_ALIGNMENT,
+ * W4_ERR_WORKSPACE, W4_ERR_CUDA.  Nothing is launched unless every check
+ * passes.  Stream-ordered; no host synchronization.
+ */
+w4_status awq_block_scoring_losses(const w4_block_config* cfg, const double* x, int64_t T,
+                                   const w4_block_weights* block, const w4_block_weights* next,
+                                   int group, const float* alphas, int n_alpha,
+                                   const float* shrinks, int n_shrink, int symmetric, int only,
+                                   double* losses_out, void* workspace, size_t workspace_bytes,
+                                   void* stream);
+
+/*
+ * awq_block_search -- the search of one block ([rebuttal] 'Search' row,
+ * 'Clipping granularity'): for each group in order, alpha* = the least loss
+ * over the alpha grid at shrink 1 (every linear of the group quantized with
+ * that alpha); then for each linear of the group its own ratio r* = the
+ * least loss over the shrink grid with the group at alpha* and its other
+ * linears unclipped.  Groups are scored one at a time with the rest of
+ * block i unquantized.  Ties go to the lowest index.
+ *
+ * choice_out     device int32 [11] out: alpha index per group (4), then
+ *                shrink index per linear (7).
+ * losses_out     device float64 [4 * n_alpha + 7 * n_shrink] out (the alpha
+ *                losses per group, then the shrink losses per linear), or
+ *                NULL.
+ * Other arguments and errors as awq_block_scoring_losses.
+ */
+w4_status awq_block_search(const w4_block_config* cfg, const double* x, int64_t T,
+                           const w4_block_weights* block, const w4_block_weights* next,
+                           const float* alphas, int n_alpha, const float* shrinks, int n_shrink,
+                           int symmetric, int32_t* choice_out, double* losses_out,
+                           void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * w4_quantize_pack_rows -- w4_quantize_pack with one shrink ratio per output

@@ -1,0 +1,119 @@
+"""Block-level candidate scoring on the GPU against oracle/block_oracle.py
+("ghostchoir/rebuttal_w4g128_awq_w2" model card: the 'Search' row and the
+paragraph under the 'Model Details' table; the perplexity table's d=0 row):
+the losses of every candidate at the output of block i+1 (look-ahead) and at
+block i's own output, and the whole search of one block, on a
+Qwen3-1.7B-shaped block (hidden 2048, 16 / 8 heads of width 128, SwiGLU
+6144) at T = 256 tokens.
+
+Both sides compute in binary64; they differ only in the order of the sums
+(the GPU's fp64 MMA against numpy's BLAS).  Rounding of the order is about
+1e-16 of an activation; the loss is the mean square of (path - reference),
+a difference about 1e-2 of the activations, so its relative error is at most
+about 1e-16 * 1e2 * (a few steps) ~ 1e-13.  The tests allow 1e-9.  Chosen
+indices must match; two different indices are accepted only if the oracle's
+own losses at them agree within that tolerance (a genuine tie).
+"""
+import numpy as np
+import pytest
+
+from oracle import block_oracle as B
+from weight_only_int4_quantize_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+LOSS_RTOL = 1e-9
+T = 256
+CFG = dict(B.QWEN3_1P7B)
+
+
+def _torch():
+    import torch
+    return torch
+
+
+@pytest.fixture(scope="module")
+def blocks():
+    """Block i, block i+1 and block i's input, on the GPU and as the oracle's
+    inputs (bf16 bit patterns, binary64 gains and input)."""
+    torch = _torch()
+    dev = "cuda"
+    out = []
+    for b in (3, 4):
+        cpu = synth.qwen_block(b)
+        bits = {n: synth.bits(cpu[n]) for n in synth.BLOCK_LINEAR_NAMES}
+        norms = {n: cpu[n].numpy() for n in ("ln1", "ln2", "q_norm", "k_norm")}
+        gpu = {n: v.to(dev) for n, v in cpu.items()}
+        out.append((gpu, bits, norms))
+    x = synth.block_input(T, 2048, seed=77)
+    return out[0], out[1], x.to(dev), x.numpy()
+
+
+def _same_pick(got: int, ref_losses: np.ndarray, what: str):
+    want = int(np.argmin(ref_losses))
+    if got != want:
+        a, b = ref_losses[got], ref_losses[want]
+        assert abs(a - b) <= LOSS_RTOL * abs(b), (what, got, want, a, b)
+
+
+def _check_losses(got, ref, what):
+    rel = np.abs(got - ref) / np.abs(ref)
+    assert rel.max() <= LOSS_RTOL, (what, float(rel.max()))
+    return float(rel.max())
+
+
+@pytest.mark.parametrize("ahead", [True, False], ids=["lookahead", "own_output"])
+def test_block_losses_qkv_alpha_grid(blocks, ahead):
+    import weight_only_int4_quantize_b200 as w4
+    (gi, bi, ni), (gn, bn, nn), x, xh = blocks
+    al = synth.alpha_grid(20)
+    one = np.array([1.0], np.float32)
+    got = w4.awq_block_scoring_losses(x, gi, gn if ahead else None, "qkv", al, one, False)
+    ref = B.scoring_losses(xh, bi, ni, (bn, nn) if ahead else None, "qkv", al, one, False, CFG)
+    got = got.cpu().numpy()
+    _check_losses(got, ref, "qkv alpha grid")
+    _same_pick(int(np.argmin(got[:, 0])), ref[:, 0], "alpha*")
+
+
+@pytest.mark.parametrize("group,only,sym", [("o", None, True), ("gate_up", "up", False),
+                                            ("down", None, False)])
+def test_block_losses_groups_and_single_linear(blocks, group, only, sym):
+    import weight_only_int4_quantize_b200 as w4
+    (gi, bi, ni), (gn, bn, nn), x, xh = blocks
+    al = synth.alpha_grid(20)[[0, 5, 10, 15]]
+    sh = synth.shrink_grid(10)[[0, 2, 4]]
+    got = w4.awq_block_scoring_losses(x, gi, gn, group, al, sh, sym, only=only).cpu().numpy()
+    ref = B.scoring_losses(xh, bi, ni, (bn, nn), group, al, sh, sym, CFG, only=only)
+    _check_losses(got, ref, f"{group} {only}")
+
+
+@pytest.mark.parametrize("ahead", [True, False], ids=["lookahead", "own_output"])
+def test_block_search_matches_oracle(blocks, ahead):
+    """The whole search of one block: alpha* per group, then r* per linear."""
+    import weight_only_int4_quantize_b200 as w4
+    (gi, bi, ni), (gn, bn, nn), x, xh = blocks
+    al = synth.alpha_grid(20)[::4]
+    sh = synth.shrink_grid(10)[:4]
+    choice, losses = w4.awq_block_search(x, gi, gn if ahead else None, al, sh, False)
+    choice = choice.cpu().numpy()
+    losses = losses.cpu().numpy()
+    ref = B.search_block(xh, bi, ni, (bn, nn) if ahead else None, al, sh, False, CFG)
+    na, nr = len(al), len(sh)
+    for gidx, group in enumerate(B.GROUPS):
+        a_star, r_star = ref[group]
+        if choice[gidx] != a_star:
+            one = np.array([1.0], np.float32)
+            col = B.scoring_losses(xh, bi, ni, (bn, nn) if ahead else None, group, al, one,
+                                   False, CFG)[:, 0]
+            _same_pick(int(choice[gidx]), col, f"{group} alpha*")
+            continue  # the shrink phase then ran at another (tied) alpha
+        for name, r in r_star.items():
+            li = B.LINEARS.index(name)
+            got_r = int(choice[4 + li])
+            if got_r != r:
+                row = B.scoring_losses(xh, bi, ni, (bn, nn) if ahead else None, group,
+                                       al[a_star:a_star + 1], sh, False, CFG, only=name)[0]
+                _same_pick(got_r, row, f"{name} r*")
+        # the reported alpha losses are the group's column
+        assert np.all(np.isfinite(losses[gidx * na:(gidx + 1) * na]))
+    assert np.all(losses[4 * na:] > 0)

@@ -104,6 +104,15 @@ def _declare(L: ctypes.CDLL) -> None:
                               ctypes.c_uint, _p]
     L.w4a8_linear_batched.restype = ctypes.c_int
     L.w4a8_linear_batched.argtypes = [_p, ctypes.c_int, _i64, ctypes.c_int, ctypes.c_uint, _p]
+    L.w4_block_workspace_bytes.restype = ctypes.c_size_t
+    L.w4_block_workspace_bytes.argtypes = [_p, _i64]
+    L.awq_block_scoring_losses.restype = ctypes.c_int
+    L.awq_block_scoring_losses.argtypes = [_p, _p, _i64, _p, _p, ctypes.c_int, _p, ctypes.c_int,
+                                           _p, ctypes.c_int, ctypes.c_int, ctypes.c_int, _p, _p,
+                                           ctypes.c_size_t, _p]
+    L.awq_block_search.restype = ctypes.c_int
+    L.awq_block_search.argtypes = [_p, _p, _i64, _p, _p, _p, ctypes.c_int, _p, ctypes.c_int,
+                                   ctypes.c_int, _p, _p, _p, ctypes.c_size_t, _p]
     L.w4_device_error.restype = ctypes.c_int
     L.w4_device_error.argtypes = [ctypes.c_int, _p]
     L.w4_selftest_bounded_wait.restype = ctypes.c_int
@@ -523,6 +532,113 @@ def awq_score_grid_static_scratch(x, w, alphas, shrinks, symmetric: bool, seg_of
         raise W4Error(st, "awq_score_grid_static_scratch: " + lib().w4_last_error().decode())
     _check(st, "awq_score_grid_static_scratch")
     return sse_out, argmin_out
+
+
+class BlockConfig(ctypes.Structure):
+    """w4_block_config: a decoder block's shape (Qwen3 conventions)."""
+    _fields_ = [("hidden", ctypes.c_int32), ("heads", ctypes.c_int32),
+                ("kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+                ("ffn", ctypes.c_int32), ("eps", ctypes.c_double),
+                ("rope_theta", ctypes.c_double)]
+
+
+class _BlockWeights(ctypes.Structure):
+    _fields_ = [(name, ctypes.c_void_p) for name in
+                ("q", "k", "v", "o", "gate", "up", "down", "ln1", "ln2", "q_norm", "k_norm")]
+
+
+QWEN3_1P7B_BLOCK = dict(hidden=2048, heads=16, kv_heads=8, head_dim=128, ffn=6144, eps=1e-6,
+                        rope_theta=1e6)
+BLOCK_LINEARS = ("q", "k", "v", "o", "gate", "up", "down")
+BLOCK_GROUPS = ("qkv", "o", "gate_up", "down")
+
+
+def _block_cfg(cfg):
+    return BlockConfig(**(cfg or QWEN3_1P7B_BLOCK))
+
+
+def _block_weights(blk, ref):
+    """Checks one block's tensors (dict: the seven bf16 linears, the four
+    float64 gains) and returns the C struct of their pointers."""
+    if blk is None:
+        return None
+    torch = _torch()
+    for name in BLOCK_LINEARS:
+        _cuda(blk[name], torch.bfloat16, name)
+    for name in ("ln1", "ln2", "q_norm", "k_norm"):
+        _cuda(blk[name], torch.float64, name)
+    _same_device(ref, **{k: blk[k] for k in BLOCK_LINEARS + ("ln1", "ln2", "q_norm", "k_norm")})
+    return _BlockWeights(**{f[0]: blk[f[0]].data_ptr() for f in _BlockWeights._fields_})
+
+
+def block_workspace_bytes(t: int, cfg=None) -> int:
+    c = _block_cfg(cfg)
+    return int(lib().w4_block_workspace_bytes(ctypes.byref(c), int(t)))
+
+
+def _block_common(x, block, next_block, alphas, shrinks, cfg, workspace):
+    import numpy as np
+    torch = _torch()
+    _cuda(x, torch.float64, "x")
+    c = _block_cfg(cfg)
+    t = x.shape[0]
+    if x.dim() != 2 or x.shape[1] != c.hidden:
+        raise ValueError("x must be float64 [T, hidden]")
+    bi = _block_weights(block, x)
+    bn = _block_weights(next_block, x)
+    al = np.ascontiguousarray(np.asarray(alphas, dtype=np.float32))
+    sh = np.ascontiguousarray(np.asarray(shrinks, dtype=np.float32))
+    need = int(lib().w4_block_workspace_bytes(ctypes.byref(c), t))
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=x.device)
+    _same_device(x, workspace=workspace)
+    return c, t, bi, bn, al, sh, workspace
+
+
+def awq_block_scoring_losses(x, block, next_block, group, alphas, shrinks, symmetric: bool,
+                             only=None, cfg=None, workspace=None):
+    """loss[a, j] of every (alphas[a], shrinks[j]) candidate of one linear
+    group of a decoder block, at the output of next_block (look-ahead) or of
+    the block itself (next_block None), in binary64 on the device.
+
+    x: float64 [T, hidden] block input on the device; block / next_block:
+    dicts of the seven bf16 linears ("q" .. "down", [out, in]) and the float64
+    gains "ln1", "ln2", "q_norm", "k_norm"; group: "qkv", "o", "gate_up",
+    "down" (or 0..3); only: None or the name of one linear of the group."""
+    torch = _torch()
+    c, t, bi, bn, al, sh, ws = _block_common(x, block, next_block, alphas, shrinks, cfg,
+                                             workspace)
+    g = BLOCK_GROUPS.index(group) if isinstance(group, str) else int(group)
+    o = -1 if only is None else (BLOCK_LINEARS.index(only) if isinstance(only, str) else int(only))
+    losses = torch.empty((len(al), len(sh)), dtype=torch.float64, device=x.device)
+    with torch.cuda.device(x.device):
+        st = lib().awq_block_scoring_losses(
+            ctypes.byref(c), x.data_ptr(), t, ctypes.byref(bi),
+            None if bn is None else ctypes.byref(bn), g, al.ctypes.data, len(al),
+            sh.ctypes.data, len(sh), int(bool(symmetric)), o, losses.data_ptr(),
+            ws.data_ptr(), ws.numel(), _stream(x.device))
+    _check(st, "awq_block_scoring_losses")
+    return losses
+
+
+def awq_block_search(x, block, next_block, alphas, shrinks, symmetric: bool, cfg=None,
+                     workspace=None):
+    """The search of one block on the device: returns (choice int32 [11]:
+    alpha index per group qkv, o, gate_up, down, then shrink index per
+    linear q .. down; losses float64 [4 * n_alpha + 7 * n_shrink])."""
+    torch = _torch()
+    c, t, bi, bn, al, sh, ws = _block_common(x, block, next_block, alphas, shrinks, cfg,
+                                             workspace)
+    choice = torch.empty(11, dtype=torch.int32, device=x.device)
+    losses = torch.empty(4 * len(al) + 7 * len(sh), dtype=torch.float64, device=x.device)
+    with torch.cuda.device(x.device):
+        st = lib().awq_block_search(
+            ctypes.byref(c), x.data_ptr(), t, ctypes.byref(bi),
+            None if bn is None else ctypes.byref(bn), al.ctypes.data, len(al), sh.ctypes.data,
+            len(sh), int(bool(symmetric)), choice.data_ptr(), losses.data_ptr(), ws.data_ptr(),
+            ws.numel(), _stream(x.device))
+    _check(st, "awq_block_search")
+    return choice, losses
 
 
 def device_error(clear: bool = True) -> int:

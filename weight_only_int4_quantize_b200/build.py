@@ -19,7 +19,7 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libw4.so")
 
-SOURCES = ["abi.cu", "quantize.cu", "gemv.cu", "gemv_stream.cu", "act_int8.cu", "gemm_tc.cu", "awq.cu", "noalloc.cu"]
+SOURCES = ["abi.cu", "quantize.cu", "gemv.cu", "gemv_stream.cu", "act_int8.cu", "gemm_tc.cu", "awq.cu", "block.cu", "noalloc.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-Wall",
          "--expt-relaxed-constexpr", f"-I{INCLUDE}", f"-I{CSRC}"]

@@ -715,6 +715,123 @@ w4_status awq_clip_search_rows(const void* x_bf16, int64_t M, const void* w_bf16
                      "clip search binary64 near ties");
 }
 
+namespace {
+
+bool valid_block_config(const w4_block_config* c) {
+  if (!c) return false;
+  if (c->hidden < 128 || c->hidden % 128 != 0 || c->hidden > (1 << 16)) return false;
+  if (c->heads < 1 || c->kv_heads < 1 || c->heads % c->kv_heads != 0 || c->heads > 256)
+    return false;
+  if (c->head_dim != 64 && c->head_dim != 128) return false;
+  if ((c->heads * c->head_dim) % 128 != 0) return false;
+  if (c->ffn < 128 || c->ffn % 128 != 0 || c->ffn > (1 << 17)) return false;
+  return std::isfinite(c->eps) && c->eps > 0.0 && std::isfinite(c->rope_theta) &&
+         c->rope_theta > 0.0;
+}
+
+// A block's pointers: the seven bf16 linears and the four binary64 gains.
+bool block_ptrs(const w4_block_weights* b, BlockLinears* out, bool* aligned) {
+  if (!b) return false;
+  const void* w[7] = {b->q, b->k, b->v, b->o, b->gate, b->up, b->down};
+  const double* g[4] = {b->ln1, b->ln2, b->q_norm, b->k_norm};
+  *aligned = true;
+  for (int i = 0; i < 7; ++i) {
+    if (!w[i]) return false;
+    *aligned = *aligned && aligned16(w[i]);
+    out->w[i] = w[i];
+  }
+  for (int i = 0; i < 4; ++i) {
+    if (!g[i]) return false;
+    *aligned = *aligned && aligned16(g[i]);
+  }
+  out->norms = BlockNorms{b->ln1, b->ln2, b->q_norm, b->k_norm};
+  return true;
+}
+
+// Shared checks of the block entry points; fills the internal forms.
+w4_status check_block_call(const w4_block_config* cfg, const double* x, int64_t T,
+                           const w4_block_weights* block, const w4_block_weights* next,
+                           const float* alphas, int n_alpha, const float* shrinks, int n_shrink,
+                           void* workspace, size_t workspace_bytes, BlockConfig* c,
+                           BlockLinears* bi, BlockLinears* bn) {
+  if (!cfg || !x || !block || !alphas || !shrinks) return W4_ERR_INVALID_ARG;
+  if (!valid_block_config(cfg)) return W4_ERR_SHAPE;
+  if (T < 1 || T > 8192) return W4_ERR_SHAPE;
+  if (n_alpha < 1 || n_alpha > kMaxGrid || n_shrink < 1 || n_shrink > kMaxGrid)
+    return W4_ERR_UNSUPPORTED;
+  for (int i = 0; i < n_alpha; ++i)
+    if (!std::isfinite(alphas[i])) return W4_ERR_INVALID_ARG;
+  for (int j = 0; j < n_shrink; ++j)
+    if (!(shrinks[j] > 0.0f && shrinks[j] <= 1.0f)) return W4_ERR_INVALID_ARG;
+  bool al_i = true, al_n = true;
+  if (!block_ptrs(block, bi, &al_i)) return W4_ERR_INVALID_ARG;
+  if (next && !block_ptrs(next, bn, &al_n)) return W4_ERR_INVALID_ARG;
+  if (!al_i || !al_n || !aligned16(x)) return W4_ERR_ALIGNMENT;
+  *c = BlockConfig{cfg->hidden, cfg->heads, cfg->kv_heads, cfg->head_dim, cfg->ffn, cfg->eps,
+                   cfg->rope_theta};
+  if (!workspace || workspace_bytes < block_workspace_bytes(*c, T)) return W4_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return W4_ERR_ALIGNMENT;
+  return W4_OK;
+}
+
+}  // namespace
+
+size_t w4_block_workspace_bytes(const w4_block_config* cfg, int64_t T) {
+  if (!valid_block_config(cfg) || T < 1 || T > 8192) return 0;
+  const BlockConfig c{cfg->hidden, cfg->heads, cfg->kv_heads, cfg->head_dim, cfg->ffn, cfg->eps,
+                      cfg->rope_theta};
+  return block_workspace_bytes(c, T);
+}
+
+w4_status awq_block_scoring_losses(const w4_block_config* cfg, const double* x, int64_t T,
+                                   const w4_block_weights* block, const w4_block_weights* next,
+                                   int group, const float* alphas, int n_alpha,
+                                   const float* shrinks, int n_shrink, int symmetric, int only,
+                                   double* losses_out, void* workspace, size_t workspace_bytes,
+                                   void* stream) {
+  if (!losses_out) return W4_ERR_INVALID_ARG;
+  if (group < 0 || group > 3) return W4_ERR_INVALID_ARG;
+  static const int first[5] = {0, 3, 4, 6, 7};
+  if (only != -1 && (only < first[group] || only >= first[group + 1])) return W4_ERR_INVALID_ARG;
+  BlockConfig c;
+  BlockLinears bi{}, bn{};
+  w4_status st = check_block_call(cfg, x, T, block, next, alphas, n_alpha, shrinks, n_shrink,
+                                  workspace, workspace_bytes, &c, &bi, &bn);
+  if (st != W4_OK) return st;
+  if (!aligned16(losses_out)) return W4_ERR_ALIGNMENT;
+  int sms = 0;
+  unsigned* err = nullptr;
+  st = device_info(&sms, &err);
+  if (st != W4_OK) return st;
+  return cuda_status(block_scoring_losses(&c, x, T, bi, next ? &bn : nullptr, group, alphas,
+                                          n_alpha, shrinks, n_shrink, symmetric != 0, only,
+                                          losses_out, workspace,
+                                          static_cast<cudaStream_t>(stream)),
+                     "block-level candidate losses");
+}
+
+w4_status awq_block_search(const w4_block_config* cfg, const double* x, int64_t T,
+                           const w4_block_weights* block, const w4_block_weights* next,
+                           const float* alphas, int n_alpha, const float* shrinks, int n_shrink,
+                           int symmetric, int32_t* choice_out, double* losses_out,
+                           void* workspace, size_t workspace_bytes, void* stream) {
+  if (!choice_out) return W4_ERR_INVALID_ARG;
+  BlockConfig c;
+  BlockLinears bi{}, bn{};
+  w4_status st = check_block_call(cfg, x, T, block, next, alphas, n_alpha, shrinks, n_shrink,
+                                  workspace, workspace_bytes, &c, &bi, &bn);
+  if (st != W4_OK) return st;
+  if (!aligned16(choice_out) || (losses_out && !aligned16(losses_out))) return W4_ERR_ALIGNMENT;
+  int sms = 0;
+  unsigned* err = nullptr;
+  st = device_info(&sms, &err);
+  if (st != W4_OK) return st;
+  return cuda_status(block_search(&c, x, T, bi, next ? &bn : nullptr, alphas, n_alpha, shrinks,
+                                  n_shrink, symmetric != 0, choice_out, losses_out, workspace,
+                                  static_cast<cudaStream_t>(stream)),
+                     "block-level search");
+}
+
 w4_status w4_quantize_pack_rows(const void* w_bf16, int64_t N, int64_t K, int group,
                                 int symmetric, const float* awq_s, const float* shrink_rows,
                                 int32_t* qweight, uint16_t* scales_f16, uint16_t* zeros_f16,

@@ -173,6 +173,34 @@ cudaError_t launch_clip_exact(const void* x, int M, const void* w, int N, int K,
                               uint8_t* flags, unsigned long long* mask, int* list, int* count,
                               int* rows, int* row_counts, double* rowsum, cudaStream_t stream);
 
+// Block-level candidate scoring in binary64 (block.cu).  Linears in the
+// order q, k, v, o, gate, up, down (bf16 [out, in]); groups 0 qkv, 1 o,
+// 2 gate_up, 3 down.
+struct BlockConfig {
+  int hidden, heads, kv_heads, head_dim, ffn;
+  double eps, rope_theta;
+};
+struct BlockNorms {
+  const double* ln1;
+  const double* ln2;
+  const double* q_norm;
+  const double* k_norm;
+};
+struct BlockLinears {
+  const void* w[7];
+  BlockNorms norms;
+};
+size_t block_workspace_bytes(const BlockConfig& c, int64_t T);
+cudaError_t block_scoring_losses(const BlockConfig* c, const double* x, int64_t T,
+                                 const BlockLinears& blk, const BlockLinears* next, int group,
+                                 const float* alphas, int n_alpha, const float* shrinks,
+                                 int n_shrink, bool sym, int only, double* losses,
+                                 void* workspace, cudaStream_t st);
+cudaError_t block_search(const BlockConfig* c, const double* x, int64_t T, const BlockLinears& blk,
+                         const BlockLinears* next, const float* alphas, int n_alpha,
+                         const float* shrinks, int n_shrink, bool sym, int32_t* choice,
+                         double* losses, void* workspace, cudaStream_t st);
+
 // Device address of the fixed scratch behind awq_score_grid_static_scratch
 // on the current device (looked up once per device, then cached).
 cudaError_t awq_static_scratch_address(void** ptr);

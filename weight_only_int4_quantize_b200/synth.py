@@ -109,3 +109,27 @@ def qwen_block_weights(block: int, seed_base: int = 1000):
     for i, (name, k, n) in enumerate(QWEN3_1P7B_BLOCK):
         out.append((name, normal_weight(n, k, 0.02, seed_base + 7 * block + i)))
     return out
+
+
+# Linear names of one decoder block in the block-level scoring's order.
+BLOCK_LINEAR_NAMES = ("q", "k", "v", "o", "gate", "up", "down")
+
+
+def qwen_block(block: int, seed_base: int = 1000, std: float = 0.02):
+    """One Qwen3-1.7B-shaped decoder block for the block-level scoring: the
+    seven bf16 linears (N(0, std), keyed "q" .. "down", [out, in]) and the
+    float64 norm gains "ln1", "ln2" [2048] and "q_norm", "k_norm" [128], each
+    1 + 0.1 N(0, 1)."""
+    out = {}
+    for i, (name, k, n) in enumerate(QWEN3_1P7B_BLOCK):
+        out[BLOCK_LINEAR_NAMES[i]] = normal_weight(n, k, std, seed_base + 7 * block + i)
+    g = _gen(seed_base + 7 * block + 1000)
+    for name, width in (("ln1", 2048), ("ln2", 2048), ("q_norm", 128), ("k_norm", 128)):
+        out[name] = 1.0 + 0.1 * torch.randn(width, generator=g, dtype=torch.float64)
+    return out
+
+
+def block_input(t: int, hidden: int, seed: int, std: float = 1.0) -> torch.Tensor:
+    """float64 [t, hidden] hidden states entering a block ~ N(0, std)."""
+    g = _gen(seed)
+    return torch.randn(t, hidden, generator=g, dtype=torch.float64) * std
