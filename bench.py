@@ -14,8 +14,10 @@ weights N(0, 0.02), int4 asymmetric g128.  A step runs
       in one persistent launch, with programmatic dependent launch.
 value = algorithmic bytes of the step / step time (GB/s): 2.53125 B/weight
 for quantize, 0.53125 B/weight + 2MK + 2MN bytes per decode linear.  The step
-is one CUDA graph; its working set (2.8 GB bf16 weights, 0.75 GB packed) is
-far larger than L2, so no flush is needed between steps.
+is two CUDA graphs: the quantize launches, then the three decode launches
+chained with programmatic dependent launch; its working set (2.8 GB bf16
+weights, 0.75 GB packed) is far larger than L2, so no flush is needed between
+steps.
 
 Multi-GPU: every rank runs its own replica (the path has no exchange step);
 value sums the ranks' bytes over the slowest rank's time ("weak" scaling).
@@ -50,15 +52,37 @@ FALLBACK_BF16_TFLOPS = 1590.0
 # summaries under profiles/ give the commands), with the digest of the kernel
 # source the capture was taken on.  A changed source reports traffic null.
 TRAFFIC_CAPTURES = {
-    # decode_batch --m 1 --blocks 4 (streaming kernel): 110.44 MB over 107.27 MB algorithmic
-    "gemv_w4a16": {"source": "gemv_stream.cu", "digest": "abce4dea2872e4f3",
-                   "ratio": 110.44 / 107.27},
+    # decode_batch --m 1 --blocks 4 (streaming kernel, 28 linears): 110.43 MB
+    # (107.27 read + 3.16 written back from the preceding quantize) over
+    # 107.27 MB algorithmic
+    "gemv_w4a16": {"source": "gemv_stream.cu", "digest": "094c567067a0bb3b",
+                   "ratio": (107269888 + 3163904) / 107266048},
     # quantize 17408 x 5120: 202.47 MB over 225.67 MB (part of the written codes
     # is still in the write-back L2 when the kernel ends)
     "quantize_pack": {"source": "quantize.cu", "digest": "f3061dcc5ac9fd85", "ratio": 202.47 / 225.67},
+    # linear --m 2048 --k 4096 --n 4096 --sym --gemm: 25.51 MB read (weights +
+    # x once; y still in L2 at the end) over 42.21 MB algorithmic
+    "gemm_tc": {"source": "gemm_tc.cu", "digest": "012479ae0a5800c8",
+                "ratio": (25499648 + 5888) / 42205184},
 }
 
+LLAMA2_LINEARS = ((4096, 4096, 4), (4096, 11008, 2), (11008, 4096, 1))
+
 # --------------------------------------------------------------------------
+
+
+def roofline_entry(kernel, bound, achieved, peak, unit, peak_kind, bytes_per_launch, share,
+                   flops_per_launch=None):
+    cap = TRAFFIC_CAPTURES.get(kernel)
+    traffic = None
+    if cap and source_digest(cap["source"]) == cap["digest"]:
+        traffic = cap["ratio"] * bytes_per_launch
+    e = {"kernel": kernel, "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
+         "frac": achieved / peak, "peak_kind": peak_kind, "traffic": traffic,
+         "algorithmic_bytes_per_launch": bytes_per_launch, "step_share": share}
+    if flops_per_launch is not None:
+        e["algorithmic_flops_per_launch"] = flops_per_launch
+    return e
 
 
 def source_digest(name):
@@ -198,17 +222,77 @@ def oracle_sample(step_index: int):
     return nbytes, dt
 
 
+def cpu_model():
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
+
+
+def _timed(fn, min_s):
+    """Calls fn until min_s seconds have passed (at least once); returns
+    (calls, seconds)."""
+    n, t0 = 0, time.perf_counter()
+    while True:
+        fn()
+        n += 1
+        dt = time.perf_counter() - t0
+        if dt >= min_s:
+            return n, dt
+
+
+def cpu_parts(threads, min_s=1.5):
+    """The oracle's pieces on this host at a given BLAS thread count:
+    quantize+pack GB/s (2048 x 2048, asymmetric), binary64 GEMV (M = 1) and
+    GEMM (M = 512) GFLOP/s on a 4096 x 4096 dequantized weight, and AWQ grid
+    candidates/s on k_proj (2048 calibration tokens, 2048 -> 1024, 2 x 2
+    grid)."""
+    from threadpoolctl import threadpool_limits
+    from oracle import w4_oracle as O
+    from weight_only_int4_quantize_b200 import synth
+    out = {"threads": threads}
+    with threadpool_limits(limits=threads):
+        w = synth.bits(synth.normal_weight(2048, 2048, 0.02, seed=9300, n_outliers=8,
+                                           outlier_scale=20.0))
+        n, dt = _timed(lambda: O.pack_codes(O.quantize_rtn(w, False)[0]), min_s)
+        out["quantize_gbs"] = n * quant_bytes(2048, 2048) / dt / 1e9
+        wb = synth.bits(synth.normal_weight(4096, 4096, 0.02, seed=9301))
+        codes, s16, _ = O.quantize_rtn(wb, True)
+        what = O.dequantize(codes, s16, None)
+        for m, key in ((1, "gemv_f64_gflops"), (512, "gemm_f64_gflops")):
+            x = synth.bits(synth.normal_activations(m, 4096, seed=9302 + m))
+            n, dt = _timed(lambda: O.linear(x, what), min_s)
+            out[key] = n * 2.0 * m * 4096 * 4096 / dt / 1e9
+        xk = synth.bits(synth.student_t_calibration(2048, 2048, seed=9304))
+        wk = synth.bits(synth.normal_weight(1024, 2048, 0.02, seed=9305))
+        al, sh = synth.alpha_grid(20)[[5, 10]], synth.shrink_grid(10)[:2]
+        n, dt = _timed(lambda: O.awq_score_grid(xk, wk, al, sh, False), min_s)
+        out["awq_kproj_candidates_per_s"] = n * len(al) * len(sh) / dt
+    return out
+
+
 def cpu_baseline(target_s=12.0):
-    """The oracle as it stands, timed on this host on a bounded sample."""
+    """The oracle as it stands, timed on this host on a bounded sample (the
+    headline figure), plus its pieces at one BLAS thread and at all."""
     tot_b, tot_t, i = 0.0, 0.0, 0
     while tot_t < target_s and i < 196:
         b, t = oracle_sample(i)
         tot_b += b
         tot_t += t
         i += 1
-    return {"value": tot_b / tot_t / 1e9, "unit": "GB/s", "cores": cpu_threads(), "kind": "oracle",
-            "sample": f"{i} linears of the Qwen3-1.7B-shaped blocks (rotating shapes): numpy binary32 "
-                      f"quantize+pack, then binary64 decode at M=1,4,8; {tot_t:.1f} s"}
+    out = {"value": tot_b / tot_t / 1e9, "unit": "GB/s", "cores": cpu_threads(), "kind": "oracle",
+           "sample": f"{i} linears of the Qwen3-1.7B-shaped blocks (rotating shapes): numpy binary32 "
+                     f"quantize+pack, then binary64 decode at M=1,4,8; {tot_t:.1f} s",
+           "nproc": os.cpu_count(), "cpu_model": cpu_model(),
+           "omp_num_threads": os.environ.get("OMP_NUM_THREADS")}
+    try:
+        out["parts"] = [cpu_parts(1), cpu_parts(cpu_threads())]
+    except Exception as e:  # threadpoolctl missing or a BLAS it cannot limit
+        out["parts_error"] = f"{type(e).__name__}: {e}"
+    return out
 
 
 def run_reference(args):
@@ -333,36 +417,84 @@ def breakdown(torch, dev, hbm, bf16_peak, bf16_sus):
             w[:, ch] *= scale
         return w.to(torch.bfloat16)
 
+    pdl_static = w4.LINEAR_PDL | w4.LINEAR_STATIC_WEIGHTS
+
+    # Single linear K = N = 2048, 8 input channels x20, asymmetric g128:
+    # quantize+pack and decode at M = 1 and 16.  120 copies (264 MB of bf16
+    # weights, 264 MB packed) are used in turn, more than twice the 126 MB L2,
+    # so the figures are HBM figures.
+    copies = 120
+    ws_bf = [weights(2048, 2048, 0.02, 9000 + c, 8, 20.0) for c in range(copies)]
+    packed1 = [w4.quantize_pack(wb, False) for wb in ws_bf]
+    q_items = w4.quantize_pack_items([(wb, None, 1.0, qw, sc, zr)
+                                      for wb, (qw, sc, zr) in zip(ws_bf, packed1)])
+
+    def run_q():
+        w4.quantize_pack_batched(q_items, False, stream=torch.cuda.current_stream(dev).cuda_stream)
+    gq = capture(torch, run_q)
+    t = time_graph(torch, gq, 10)
+    out["cfg1_quantize_2048x2048_outliers"] = {
+        "ms_per_weight": t / copies, "gbs": copies * quant_bytes(2048, 2048) / t / 1e6,
+        "frac_hbm": copies * quant_bytes(2048, 2048) / t / 1e6 / hbm, "copies": copies}
+    del gq, q_items, ws_bf
+    for m in (1, 16):
+        x1 = torch.randn(m, 2048, generator=g, device=dev).to(torch.bfloat16)
+        y1 = torch.empty(m, 2048, dtype=torch.bfloat16, device=dev)
+
+        def run_l(x1=x1, y1=y1):
+            for qw, sc, zr in packed1:
+                w4.w4a16_linear(x1, qw, sc, zr, flags=pdl_static, out=y1)
+        gl = capture(torch, run_l)
+        t = time_graph(torch, gl, 10) / copies
+        byts = gemv_bytes(m, 2048, 2048)
+        out[f"cfg1_decode_2048x2048_M{m}"] = {
+            "ms_per_linear": t, "gbs": byts / t / 1e6, "frac_hbm": byts / t / 1e6 / hbm,
+            "copies": copies, "launches": "one w4a16_linear per copy, PDL, one CUDA graph"}
+        del gl
+    del packed1
+    torch.cuda.empty_cache()
+
     # Prefill / M-sweep on the Llama-2-7B- and 27B-shaped linears (symmetric).
     lin_sets = {
         "llama2_7b": [(k, n, c) for k, n, c in synth.LLAMA2_7B_LINEARS],
         "27b": [(k, n, 1) for k, n in synth.SCALE27B_LINEARS],
     }
     for tag, shapes in lin_sets.items():
-        packed = []
-        for i, (k, n, cnt) in enumerate(shapes):
-            w = weights(n, k, 0.02 if tag == "llama2_7b" else 0.015, 500 + i,
-                        0 if tag == "llama2_7b" else k // 100, 10.0)
-            qw, sc, _ = w4.quantize_pack(w, True)
-            packed.append((k, n, cnt, qw, sc))
-            del w
+        # The 27B-scale trio (119 MB packed) fits L2: three copies of it are
+        # used in turn (357 MB), so the decode sizes read HBM.
+        n_copies = 3 if tag == "27b" else 1
+        sets = []
+        for c in range(n_copies):
+            packed = []
+            for i, (k, n, cnt) in enumerate(shapes):
+                w = weights(n, k, 0.02 if tag == "llama2_7b" else 0.015, 500 + i + 31 * c,
+                            0 if tag == "llama2_7b" else k // 100, 10.0)
+                qw, sc, _ = w4.quantize_pack(w, True)
+                packed.append((k, n, cnt, qw, sc))
+                del w
+            sets.append(packed)
+        packed = sets[0]
         ms = (512, 2048) if tag == "llama2_7b" else (1, 8, 64, 512, 4096)
         for m in ms:
             xs = {k: torch.randn(m, k, generator=g, device=dev).to(torch.bfloat16)
                   for k in {p[0] for p in packed}}
             ys = [torch.empty(m, p[1], dtype=torch.bfloat16, device=dev) for p in packed]
+            fl = pdl_static if m <= 8 else 0
 
             def run():
-                for (k, n, cnt, qw, sc), y in zip(packed, ys):
-                    for _ in range(cnt):
-                        w4.w4a16_linear(xs[k], qw, sc, None, out=y)
+                for pk in sets:
+                    for (k, n, cnt, qw, sc), y in zip(pk, ys):
+                        for _ in range(cnt):
+                            w4.w4a16_linear(xs[k], qw, sc, None, flags=fl, out=y)
             gr = capture(torch, run)
-            t = time_graph(torch, gr, 20 if m >= 512 else 50)
+            t = time_graph(torch, gr, 20 if m >= 512 else 50) / n_copies
             flops = sum(2.0 * m * n * k * cnt for k, n, cnt, *_ in packed)
             byts = sum(gemv_bytes(m, n, k, True) * cnt for k, n, cnt, *_ in packed)
             rec = {"ms": t, "tflops": flops / t / 1e9, "gbs": byts / t / 1e6}
             rec["frac_bf16_peak"] = rec["tflops"] / bf16_peak
             rec["frac_hbm"] = rec["gbs"] / hbm
+            if n_copies > 1:
+                rec["copies"] = n_copies
             out[f"{tag}_M{m}"] = rec
             if m >= 512:
                 # The same linears as one batched call (independent problems):
@@ -377,7 +509,7 @@ def breakdown(torch, dev, hbm, bf16_peak, bf16_sus):
                                               "frac_bf16_peak": flops / t2 / 1e9 / bf16_peak}
                 del gr2, arr, ys_g
             del gr, xs, ys
-        del packed
+        del packed, sets
     torch.cuda.empty_cache()
 
     # AWQ grid, one Qwen3-1.7B block (q,k,v,o,gate,up share K=2048), 20 x 10 grid.
@@ -442,6 +574,30 @@ def breakdown(torch, dev, hbm, bf16_peak, bf16_sus):
         "rows_per_ratio": torch.bincount(choice.long(), minlength=10).tolist()}
     del cws, wg, x
     torch.cuda.empty_cache()
+
+    # Block-level (look-ahead) search of one Qwen3-1.7B-shaped block in
+    # binary64: T = 2048 tokens entering block i, block i+1 unquantized, the
+    # 20 x 10 grid (alpha* per group: 4 x 20 candidates, then a ratio per
+    # linear: 7 x 10), every candidate two block forwards from the group on.
+    gi = {k: v.to(dev) for k, v in synth.qwen_block(3).items()}
+    gn = {k: v.to(dev) for k, v in synth.qwen_block(4).items()}
+    xb = synth.block_input(2048, 2048, seed=77).to(dev)
+    wsb = torch.empty(w4.block_workspace_bytes(2048), dtype=torch.uint8, device=dev)
+    al, sh = synth.alpha_grid(20), synth.shrink_grid(10)
+    w4.awq_block_scoring_losses(xb, gi, gn, "down", al[:1], sh[:1], False, workspace=wsb)
+    torch.cuda.synchronize()
+    a_ev, b_ev = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a_ev.record()
+    choice, _ = w4.awq_block_search(xb, gi, gn, al, sh, False, workspace=wsb)
+    b_ev.record()
+    torch.cuda.synchronize()
+    t = a_ev.elapsed_time(b_ev)
+    out["block_search_qwen_T2048_20x10_lookahead"] = {
+        "ms": t, "candidates": 4 * 20 + 7 * 10, "candidates_per_s": 150 / (t * 1e-3),
+        "workspace_gb": wsb.numel() / 1e9, "choice": choice.tolist(),
+        "precision": "binary64 (fp64 MMA GEMMs)"}
+    del gi, gn, xb, wsb
+    torch.cuda.empty_cache()
     return out
 
 
@@ -480,6 +636,12 @@ def main():
     model = Model(dev, seed_base=1000 + 97 * rank)
     flags = w4.LINEAR_PDL | w4.LINEAR_STATIC_WEIGHTS
     g_q = capture(torch, model.quantize_all)
+    # The decode phase: the three token counts' launches chained in one graph
+    # (programmatic dependent launch: each launch's weight stream starts while
+    # the previous one drains, as consecutive decode steps run in serving).
+    # The weights were written by the quantize graph, which has completed.
+    g_dc = capture(torch, lambda: [model.decode_all(m, flags) for m in DECODE_M])
+    # The same launches one per graph (isolated: ramp and tail exposed).
     g_d = {m: capture(torch, lambda m=m: model.decode_all(m, flags)) for m in DECODE_M}
     launches_per_step = model.launches["quantize"] + model.launches["gemv"]
     qb, db = step_bytes()
@@ -487,16 +649,14 @@ def main():
 
     def step():
         g_q.replay()
-        for m in DECODE_M:
-            g_d[m].replay()
+        g_dc.replay()
 
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
     if pg:
         pg.barrier()
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2 + len(DECODE_M))]
-          for _ in range(args.steps)]
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local) as clk:
         torch.cuda.synchronize()
@@ -506,9 +666,8 @@ def main():
             e[0].record()
             g_q.replay()
             e[1].record()
-            for j, m in enumerate(DECODE_M):
-                g_d[m].replay()
-                e[2 + j].record()
+            g_dc.replay()
+            e[2].record()
         end.record()
         torch.cuda.synchronize()
     if pg:
@@ -517,10 +676,24 @@ def main():
     total_ms = max_over_ranks(pg, total_ms, dev)
     ms_step = total_ms / args.steps
     q_ms = sum(e[0].elapsed_time(e[1]) for e in ev) / args.steps
-    d_ms = {m: sum(e[1 + j].elapsed_time(e[2 + j]) for e in ev) / args.steps
-            for j, m in enumerate(DECODE_M)}
+    gemv_ms = sum(e[1].elapsed_time(e[2]) for e in ev) / args.steps
     value = whole_job_gbs(world, qb + db, ms_step)
     clocks = clk.summary()
+    # Per token count: each launch alone in its graph, after the quantize
+    # graph as in the step (outside the timed region).
+    n_iso = max(10, min(50, args.steps))
+    iso = {m: [] for m in DECODE_M}
+    for _ in range(n_iso):
+        g_q.replay()
+        for m in DECODE_M:
+            a_i, b_i = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a_i.record()
+            g_d[m].replay()
+            b_i.record()
+            iso[m].append((a_i, b_i))
+    torch.cuda.synchronize()
+    d_ms = {m: sum(a_i.elapsed_time(b_i) for a_i, b_i in iso[m]) / n_iso for m in DECODE_M}
+    del g_d
 
     # ---------------------------------------------- end to end (host buffers)
     # Per step: H2D of every bf16 weight and x from pinned memory, the same
@@ -591,24 +764,19 @@ def main():
                          "frac_hbm": db_m[m] / (t8 * 1e-3) / 1e9 / hbm}
         del g8, a8, qx
 
-    # ---------------------------------------------- roofline (dominant kernel)
-    gemv_ms = sum(d_ms.values())
-    if q_ms >= gemv_ms:
-        dom = ("quantize_pack", qb / (q_ms * 1e-3) / 1e9, model.launches["quantize"])
-    else:
-        dom = ("gemv_w4a16", db / (gemv_ms * 1e-3) / 1e9, model.launches["gemv"])
-    bytes_per_launch = (qb if dom[0] == "quantize_pack" else db) / dom[2]
-    cap = TRAFFIC_CAPTURES.get(dom[0])
-    traffic = None
-    if cap and cap["digest"] and source_digest(cap["source"]) == cap["digest"]:
-        traffic = cap["ratio"] * bytes_per_launch
-    roofline = {"kernel": dom[0], "bound": "hbm", "achieved": dom[1], "peak": hbm, "unit": "GB/s",
-                "frac": dom[1] / hbm, "peak_kind": peak_kind, "traffic": traffic,
-                "algorithmic_bytes_per_launch": bytes_per_launch,
-                "note": "achieved = algorithmic bytes of the kernel's launches in the timed region "
-                        "/ their CUDA-event time (graph phase, launch gaps included); traffic = "
-                        "the ncu capture's DRAM bytes / algorithmic bytes, times this launch's "
-                        "algorithmic bytes (null once the kernel source differs from the capture's)"}
+    # ---------------------------------------------- roofline (per kernel)
+    # One entry per hot kernel, the step's dominant one first: achieved =
+    # algorithmic bytes (FLOPs) of its launches in the timed region / their
+    # CUDA-event time; traffic = the ncu capture's DRAM bytes / algorithmic
+    # bytes of the captured launch, times this launch's algorithmic bytes
+    # (null once the kernel source differs from the capture's).
+    roofline = [
+        roofline_entry("quantize_pack", "hbm", qb / (q_ms * 1e-3) / 1e9, hbm, "GB/s", peak_kind,
+                       qb / model.launches["quantize"], q_ms / (q_ms + gemv_ms)),
+        roofline_entry("gemv_w4a16", "hbm", db / (gemv_ms * 1e-3) / 1e9, hbm, "GB/s", peak_kind,
+                       db / model.launches["gemv"], gemv_ms / (q_ms + gemv_ms)),
+    ]
+    roofline.sort(key=lambda r: -r["step_share"])
 
     out = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
@@ -622,9 +790,13 @@ def main():
                             "problems, batched: 4 quantize launches + 1 decode launch per M",
                    "l2_note": "inputs (3.6 GB) exceed L2; no flush"},
         "phases": {"quantize_ms": q_ms, "quantize_gbs": qb / (q_ms * 1e-3) / 1e9,
-                   **{f"decode_M{m}_ms": d_ms[m] for m in DECODE_M},
-                   **{f"decode_M{m}_gbs": db_m[m] / (d_ms[m] * 1e-3) / 1e9 for m in DECODE_M},
-                   "decode_gbs": db / (gemv_ms * 1e-3) / 1e9},
+                   "decode_ms": gemv_ms, "decode_gbs": db / (gemv_ms * 1e-3) / 1e9,
+                   "decode_note": "decode_ms: the M = 1, 4, 8 launches chained (PDL) in one "
+                                  "graph, as timed in the step; decode_M*_isolated: each "
+                                  "launch alone in its graph after the quantize graph",
+                   **{f"decode_M{m}_isolated_ms": d_ms[m] for m in DECODE_M},
+                   **{f"decode_M{m}_isolated_gbs": db_m[m] / (d_ms[m] * 1e-3) / 1e9
+                      for m in DECODE_M}},
         "roofline": roofline,
         "w4a8_decode": w4a8,
         "clocks": clocks,
@@ -638,9 +810,19 @@ def main():
     # N = 1: under torchrun the other ranks would wait for it at the final
     # barrier against the process group's timeout.
     if rank == 0 and world == 1 and not args.no_breakdown:
-        del g_q, g_d, model
+        del g_q, g_dc, model
         torch.cuda.empty_cache()
         out["breakdown"] = breakdown(torch, dev, hbm, bf16_peak, bf16_sus)
+        pf = out["breakdown"].get("llama2_7b_M2048")
+        if pf:
+            # Prefill (tcgen05) on the Llama-2-7B-shaped linears at M = 2048:
+            # 7 launches per graph replay, timed burst-length.
+            flops_l = 2.0 * 2048 * sum(n * k * c for k, n, c in LLAMA2_LINEARS) / 7
+            byts_l = sum((n * k * (0.5 + 2 / 128) + 2 * 2048 * (k + n)) * c
+                         for k, n, c in LLAMA2_LINEARS) / 7
+            out["roofline"].append(roofline_entry(
+                "gemm_tc", "tensor", pf["tflops"], bf16_peak, "TFLOP/s", peak_kind, byts_l, None,
+                flops_per_launch=flops_l))
     err = w4.device_error(clear=True)
     if err:
         out["device_error"] = err

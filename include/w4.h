@@ -285,8 +285,15 @@ w4_status w4_awq_scales(const void* x_bf16, int64_t M, int64_t K, const float* a
  *
  * The candidate's codes are bit-identical to w4_quantize_pack(W, s, shrink).
  * The error product runs on tcgen05 tensor cores in fp16 in the s-domain,
- * (x/s) . (W s - w_hat)^T, accumulated in binary32 and squared and summed in
- * binary64; requires |x/s| < 65504.
+ * (x/s) . (W s - w_hat)^T, each operand scaled by an exact power of two
+ * chosen from its column maxima (its largest values near the top of fp16's
+ * range), accumulated in binary32, squared and summed in binary64 with the
+ * scaling removed exactly.  Every selection of argmin_out whose fp16 values
+ * put two or more candidates within 5e-4 (relative) of its least value is
+ * decided again on values recomputed from scratch in binary64 (fp64 MMA)
+ * for those candidates (at most 64 per call), whose sse_out entries are then
+ * the binary64 values: the selections are those of the binary64 definition,
+ * up to the order of its sums.
  *
  * x_bf16       device, bf16 [M, K] calibration activations.
  * w_bf16       device, bf16 [N, K] weight of one linear, or of several
@@ -378,7 +385,9 @@ w4_status awq_score_grid_static_scratch(const void* x_bf16, int64_t M, const voi
  * The linear's output error is the sum of its rows' errors, so the choices
  * minimise it jointly over all per-row ratio assignments.  Scored in the
  * s-domain on fp16 tensor-core operands with binary64 sums, like
- * awq_score_grid (same codes as w4_quantize_pack).
+ * awq_score_grid (same codes as w4_quantize_pack); a row whose fp16 values
+ * put two or more ratios within 5e-3 (relative) of its least value has
+ * those ratios' errors recomputed in binary64 and chooses on them.
  *
  * x_bf16, M      device bf16 [M, K] calibration activations, 1 <= M <= 2^24.
  * w_bf16, N, K   device bf16 [N, K] weight, 1 <= N <= 2^24, K % 128 == 0.

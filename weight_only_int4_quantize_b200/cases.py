@@ -6,6 +6,7 @@ timing.  Inputs are seeded and generated on the device.
     python -m weight_only_int4_quantize_b200.cases awq --m 2048 --n 1024 --k 2048 --na 20 --nr 10
     python -m weight_only_int4_quantize_b200.cases decode_batch --m 1 --blocks 4 [--a8]
     python -m weight_only_int4_quantize_b200.cases clip_rows --m 2048 --n 6144 --k 2048 --nr 10
+    python -m weight_only_int4_quantize_b200.cases block --t 512 --na 2 [--group qkv] [--own]
 
 Each case captures --iters launches in one CUDA graph (so host launch
 overhead does not count), replays it once to warm up, times one replay with
@@ -61,7 +62,12 @@ def _time(fn, iters, graph=True):
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("case", choices=["quantize", "linear", "awq", "decode_batch", "clip_rows"])
+    ap.add_argument("case", choices=["quantize", "linear", "awq", "decode_batch", "clip_rows",
+                                     "block"])
+    ap.add_argument("--t", type=int, default=512, help="block: tokens entering the block")
+    ap.add_argument("--group", default="qkv", help="block: linear group scored")
+    ap.add_argument("--own", action="store_true",
+                    help="block: loss at the block's own output (no look-ahead)")
     ap.add_argument("--blocks", type=int, default=4,
                     help="decode_batch: Qwen3-1.7B-shaped blocks (7 linears each) in one batch")
     ap.add_argument("--m", type=int, default=8)
@@ -73,12 +79,29 @@ def main():
     ap.add_argument("--na", type=int, default=20)
     ap.add_argument("--nr", type=int, default=10)
     ap.add_argument("--iters", type=int, default=3)
+    ap.add_argument("--copies", type=int, default=1,
+                    help="linear: weight copies used in turn (working set above L2)")
     ap.add_argument("--pdl", action="store_true", help="programmatic dependent launch + static weights")
     ap.add_argument("--eager", action="store_true", help="time eager launches instead of a graph")
     ap.add_argument("--a8", action="store_true", help="decode_batch: W4A8 (int8 activations)")
     ap.add_argument("--kernel", choices=["auto", "stream", "tiled"], default="auto",
                     help="decode kernel (linear, decode_batch)")
     a = ap.parse_args()
+    if a.case == "block":
+        # Block-level losses of a.na alphas (shrink 1) of one group of a
+        # Qwen3-1.7B-shaped block, binary64 (two block forwards per candidate).
+        import numpy as np
+        gi = {k: v.cuda() for k, v in synth.qwen_block(3).items()}
+        gn = None if a.own else {k: v.cuda() for k, v in synth.qwen_block(4).items()}
+        x = synth.block_input(a.t, 2048, seed=77).cuda()
+        ws = torch.empty(w4.block_workspace_bytes(a.t), dtype=torch.uint8, device="cuda")
+        al = synth.alpha_grid(20)[: a.na]
+        one = np.array([1.0], np.float32)
+        ms = _time(lambda: w4.awq_block_scoring_losses(x, gi, gn, a.group, al, one, False,
+                                                       workspace=ws), a.iters, False)
+        print(json.dumps({"case": "block", "t": a.t, "group": a.group, "candidates": a.na,
+                          "lookahead": not a.own, "ms": ms, "ms_per_candidate": ms / a.na}))
+        return
     kflag = {"auto": 0, "stream": w4.LINEAR_DECODE_STREAM,
              "tiled": w4.LINEAR_DECODE_TILED}[a.kernel]
     w = _weights(a.n, a.k, 1)
@@ -88,7 +111,11 @@ def main():
         b = a.n * a.k * (2.5 + (2 if a.sym else 4) / 128)
         out.update(ms=ms, gbs=b / ms / 1e6)
     elif a.case == "linear":
-        qw, sc, zr = w4.quantize_pack(w, a.sym)
+        # --copies C: C packed copies of the weight, used in turn, so that a
+        # working set above L2 is read from HBM.
+        packs = [w4.quantize_pack(w, a.sym)]
+        for c in range(1, a.copies):
+            packs.append(w4.quantize_pack(_weights(a.n, a.k, 1 + c), a.sym))
         del w
         g = torch.Generator(device="cuda")
         g.manual_seed(2)
@@ -98,7 +125,14 @@ def main():
         flags |= kflag
         if a.pdl:
             flags |= w4.LINEAR_PDL | w4.LINEAR_STATIC_WEIGHTS
-        ms = _time(lambda: w4.w4a16_linear(x, qw, sc, zr, flags=flags, out=y), a.iters, not a.eager)
+        turn = [0]
+
+        def run():
+            qw, sc, zr = packs[turn[0] % len(packs)]
+            turn[0] += 1
+            w4.w4a16_linear(x, qw, sc, zr, flags=flags, out=y)
+        ms = _time(run, a.iters * len(packs), not a.eager)
+        out["copies"] = len(packs)
         b = a.n * a.k * (0.5 + (2 if a.sym else 4) / 128) + 2 * a.m * (a.k + a.n)
         out.update(ms=ms, gbs=b / ms / 1e6, tflops=2.0 * a.m * a.n * a.k / ms / 1e9,
                    kernel=a.kernel)
