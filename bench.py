@@ -694,6 +694,19 @@ def main():
     torch.cuda.synchronize()
     d_ms = {m: sum(a_i.elapsed_time(b_i) for a_i, b_i in iso[m]) / n_iso for m in DECODE_M}
     del g_d
+    # Steady-state decode: the chained decode graph replayed back to back, as
+    # consecutive decode steps run (no quantize in between: the quantize
+    # graph leaves dirty packed weights in the write-back L2, which the step's
+    # decode phase writes back to HBM).
+    g_dc.replay()
+    torch.cuda.synchronize()
+    a_s, b_s = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a_s.record()
+    for _ in range(n_iso):
+        g_dc.replay()
+    b_s.record()
+    torch.cuda.synchronize()
+    steady_ms = a_s.elapsed_time(b_s) / n_iso
 
     # ---------------------------------------------- end to end (host buffers)
     # Per step: H2D of every bf16 weight and x from pinned memory, the same
@@ -794,6 +807,10 @@ def main():
                    "decode_note": "decode_ms: the M = 1, 4, 8 launches chained (PDL) in one "
                                   "graph, as timed in the step; decode_M*_isolated: each "
                                   "launch alone in its graph after the quantize graph",
+                   "decode_steady_ms": steady_ms,
+                   "decode_steady_gbs": db / (steady_ms * 1e-3) / 1e9,
+                   "decode_steady_note": "the chained decode graph replayed back to back "
+                                         "(consecutive decode steps, no quantize between)",
                    **{f"decode_M{m}_isolated_ms": d_ms[m] for m in DECODE_M},
                    **{f"decode_M{m}_isolated_gbs": db_m[m] / (d_ms[m] * 1e-3) / 1e9
                       for m in DECODE_M}},

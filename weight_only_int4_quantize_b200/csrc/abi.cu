@@ -92,7 +92,7 @@ AwqWs awq_layout(int64_t M, int64_t N, int64_t K, int n_alpha, int n_shrink, int
   w.partials = w.e + round256(sizeof(uint16_t) * static_cast<size_t>(n_shrink) * N * K);
   const size_t tiles = static_cast<size_t>(sumsq_tiles(static_cast<int>(M), static_cast<int>(N)));
   w.list = w.partials + round256(sizeof(double) * n_alpha * n_shrink * n_seg * tiles);
-  w.rowsum = w.list + round256(sizeof(int) * (kExactCap + 1));
+  w.rowsum = w.list + round256(sizeof(int) * (2 * kExactCap + 1));  // list, count, masks
   w.total = w.rowsum + round256(sizeof(double) * kExactCap *
                                 static_cast<size_t>(exact_token_chunks(static_cast<int>(M))) * N);
   return w;
@@ -616,20 +616,21 @@ w4_status awq_score_grid(const void* x_bf16, int64_t M, const void* w_bf16, int6
   }
   e = launch_awq_reduce(partials, n_alpha * n_shrink, n_seg, tiles, n_shrink, fe, sse_out, s);
   if (e != cudaSuccess) return cuda_status(e, "awq reduce");
+  SegOffsets so{};
+  for (int i = 0; i <= n_seg; ++i) so.off[i] = static_cast<int>(seg[i]);
   // Near ties of any selection: those candidates' SSE again in binary64.
   int* list = reinterpret_cast<int*>(ws + L.list);
   int* count = list + kExactCap;
+  uint32_t* masks = reinterpret_cast<uint32_t*>(count + 1);
   double* rowsum = reinterpret_cast<double*>(ws + L.rowsum);
   e = launch_awq_flag(sse_out, n_seg, n_alpha, n_shrink, c1, kGridTieTol, kExactCap, list, count,
-                      s);
+                      masks, s);
   if (e != cudaSuccess) return cuda_status(e, "awq near-tie flags");
   e = launch_exact_rowsse(x_bf16, static_cast<int>(M), w_bf16, static_cast<int>(N),
                           static_cast<int>(K), s_all, sl, n_shrink, symmetric != 0, list, count,
-                          kExactCap, nullptr, nullptr, rowsum, s);
+                          kExactCap, nullptr, nullptr, masks, so, n_seg, rowsum, s);
   if (e != cudaSuccess) return cuda_status(e, "awq binary64 near-tie scores");
-  SegOffsets so;
-  for (int i = 0; i <= n_seg; ++i) so.off[i] = seg[i];
-  e = launch_awq_exact_merge(rowsum, static_cast<int>(M), static_cast<int>(N), list, count,
+  e = launch_awq_exact_merge(rowsum, static_cast<int>(M), static_cast<int>(N), list, count, masks,
                              kExactCap, n_seg, so, n_alpha * n_shrink, sse_out, s);
   if (e != cudaSuccess) return cuda_status(e, "awq binary64 merge");
   return cuda_status(launch_awq_argmin(sse_out, n_seg, n_alpha, n_shrink, c1, argmin_out, s),

@@ -417,6 +417,7 @@ __global__ void __launch_bounds__(256, 2)
                         const float* __restrict__ s_all, ShrinkList shrinks, int n_r,
                         const int* __restrict__ list, const int* __restrict__ count, int cap,
                         const int* __restrict__ rowlist, const int* __restrict__ rowcount,
+                        const uint32_t* __restrict__ cmask, SegOffsets seg, int n_seg,
                         double* __restrict__ partial) {
   extern __shared__ __align__(16) double esm[];
   double* Es = esm;                                // [64 rows][kExactLd]
@@ -433,6 +434,13 @@ __global__ void __launch_bounds__(256, 2)
   // Row i of the tile: n0 + i, or entry n0 + i of the ratio's row list.
   const int nrows = rowlist ? rowcount[jr] : N;
   if (n0 >= nrows) return;
+  if (cmask) {  // only the segments whose selections listed this candidate
+    const uint32_t m = cmask[ci];
+    bool need = false;
+    for (int q = 0; q < n_seg; ++q)
+      need = need || (((m >> q) & 1u) && seg.off[q] < n0 + kExactRows && seg.off[q + 1] > n0);
+    if (!need) return;
+  }
   auto row_of = [&](int i) {
     if (n0 + i >= nrows) return -1;
     return rowlist ? rowlist[static_cast<size_t>(jr) * N + n0 + i] : n0 + i;
@@ -587,8 +595,9 @@ __global__ void __launch_bounds__(256, 2)
 // alpha* after the decision.  One block.
 __global__ void __launch_bounds__(256)
     awq_flag_kernel(const double* __restrict__ sse, int n_seg, int n_a, int n_r, int c1,
-                    double tol, int cap, int* __restrict__ list, int* __restrict__ count) {
-  __shared__ unsigned char flag[kMaxGrid * kMaxGrid];
+                    double tol, int cap, int* __restrict__ list, int* __restrict__ count,
+                    uint32_t* __restrict__ masks) {
+  __shared__ uint32_t flag[kMaxGrid * kMaxGrid];  // per candidate: segments that need it
   __shared__ unsigned char near_a[17][kMaxGrid];  // per segment, and the group at n_seg
   __shared__ double dred[8];
   __shared__ int ired[8];
@@ -628,8 +637,11 @@ __global__ void __launch_bounds__(256)
     return r;
   };
   // One selection: candidates pick(0 .. n-1) of table s_.  Its near-minimum
-  // set is marked in `mark` (if given) and flagged when it has >= 2 members.
+  // set is marked in `mark` (if given) and flagged when it has >= 2 members,
+  // for segment s_ (the summed table: every segment).
+  const uint32_t all_seg = n_seg >= 32 ? 0xFFFFFFFFu : (1u << n_seg) - 1u;
   auto decide = [&](auto pick, int n, int s_, unsigned char* mark) {
+    const uint32_t bits = s_ < n_seg ? 1u << s_ : all_seg;
     double m = INFINITY;
     for (int u = t; u < n; u += blockDim.x) m = fmin(m, val(s_, pick(u)));
     const double lim = block_min(m) * (1.0 + tol);
@@ -639,7 +651,7 @@ __global__ void __launch_bounds__(256)
     for (int u = t; u < n; u += blockDim.x)
       if (val(s_, pick(u)) <= lim) {
         if (mark) mark[u] = 1;
-        if (tie) flag[pick(u)] = 1;
+        if (tie) flag[pick(u)] |= bits;
       }
     __syncthreads();
   };
@@ -656,7 +668,10 @@ __global__ void __launch_bounds__(256)
   for (int c = t; c < n_c; c += blockDim.x)
     if (flag[c]) {
       const int slot = atomicAdd(&nflag, 1);
-      if (slot < cap) list[slot] = c;
+      if (slot < cap) {
+        list[slot] = c;
+        masks[slot] = flag[c];
+      }
     }
   __syncthreads();
   if (t == 0) *count = nflag;
@@ -666,13 +681,13 @@ __global__ void __launch_bounds__(256)
 // sse[seg][c] = sum over the segment's rows, in order, of rowsum.
 __global__ void awq_exact_merge_kernel(const double* __restrict__ partial, int chunks, int N,
                                        const int* __restrict__ list, const int* __restrict__ count,
-                                       int cap, int n_seg, SegOffsets seg, int n_c,
-                                       double* __restrict__ sse) {
+                                       const uint32_t* __restrict__ masks, int cap, int n_seg,
+                                       SegOffsets seg, int n_c, double* __restrict__ sse) {
   const int ci = blockIdx.x;
   const int n = *count < cap ? *count : cap;
   if (ci >= n) return;
   const int s_ = threadIdx.x;
-  if (s_ >= n_seg) return;
+  if (s_ >= n_seg || !((masks[ci] >> s_) & 1u)) return;  // a segment not recomputed
   double sum = 0.0;
   for (int row = seg.off[s_]; row < seg.off[s_ + 1]; ++row) {
     double rsum = 0.0;
@@ -814,7 +829,8 @@ int exact_token_chunks(int M) { return (M + kExactChunk - 1) / kExactChunk; }
 cudaError_t launch_exact_rowsse(const void* x, int M, const void* w, int N, int K,
                                 const float* s_all, const ShrinkList& shrinks, int n_r,
                                 bool symmetric, const int* list, const int* count, int cap,
-                                const int* rowlist, const int* rowcount, double* rowsum,
+                                const int* rowlist, const int* rowcount, const uint32_t* cmask,
+                                const SegOffsets& seg, int n_seg, double* rowsum,
                                 cudaStream_t stream) {
   const dim3 grid(static_cast<unsigned>((N + kExactRows - 1) / kExactRows),
                   static_cast<unsigned>(exact_token_chunks(M)), static_cast<unsigned>(cap));
@@ -825,27 +841,30 @@ cudaError_t launch_exact_rowsse(const void* x, int M, const void* w, int N, int 
     e = exact_smem_attr<exact_rowsse_kernel<true>>();
     if (e != cudaSuccess) return e;
     exact_rowsse_kernel<true><<<grid, 256, kExactSmem, stream>>>(
-        xb, M, wb, N, K, s_all, shrinks, n_r, list, count, cap, rowlist, rowcount, rowsum);
+        xb, M, wb, N, K, s_all, shrinks, n_r, list, count, cap, rowlist, rowcount, cmask, seg,
+        n_seg, rowsum);
   } else {
     e = exact_smem_attr<exact_rowsse_kernel<false>>();
     if (e != cudaSuccess) return e;
     exact_rowsse_kernel<false><<<grid, 256, kExactSmem, stream>>>(
-        xb, M, wb, N, K, s_all, shrinks, n_r, list, count, cap, rowlist, rowcount, rowsum);
+        xb, M, wb, N, K, s_all, shrinks, n_r, list, count, cap, rowlist, rowcount, cmask, seg,
+        n_seg, rowsum);
   }
   return cudaGetLastError();
 }
 
 cudaError_t launch_awq_flag(const double* sse, int n_seg, int n_a, int n_r, int c1, double tol,
-                            int cap, int* list, int* count, cudaStream_t stream) {
-  awq_flag_kernel<<<1, 256, 0, stream>>>(sse, n_seg, n_a, n_r, c1, tol, cap, list, count);
+                            int cap, int* list, int* count, uint32_t* masks, cudaStream_t stream) {
+  awq_flag_kernel<<<1, 256, 0, stream>>>(sse, n_seg, n_a, n_r, c1, tol, cap, list, count, masks);
   return cudaGetLastError();
 }
 
 cudaError_t launch_awq_exact_merge(const double* rowsum, int M, int N, const int* list,
-                                   const int* count, int cap, int n_seg, const SegOffsets& seg,
-                                   int n_c, double* sse, cudaStream_t stream) {
+                                   const int* count, const uint32_t* masks, int cap, int n_seg,
+                                   const SegOffsets& seg, int n_c, double* sse,
+                                   cudaStream_t stream) {
   awq_exact_merge_kernel<<<cap, 32, 0, stream>>>(rowsum, exact_token_chunks(M), N, list, count,
-                                                 cap, n_seg, seg, n_c, sse);
+                                                 masks, cap, n_seg, seg, n_c, sse);
   return cudaGetLastError();
 }
 
@@ -861,7 +880,7 @@ cudaError_t launch_clip_exact(const void* x, int M, const void* w, int N, int K,
   clip_list_kernel<<<1, 32, 0, stream>>>(mask, shrinks.n, list, count);
   clip_compact_kernel<<<shrinks.n, 1024, 0, stream>>>(flags, N, rows, row_counts);
   e = launch_exact_rowsse(x, M, w, N, K, s, shrinks, shrinks.n, symmetric, list, count, shrinks.n,
-                          rows, row_counts, rowsum, stream);
+                          rows, row_counts, nullptr, SegOffsets{}, 0, rowsum, stream);
   if (e != cudaSuccess) return e;
   clip_exact_merge_kernel<<<blocks, 128, 0, stream>>>(rowsum, exact_token_chunks(M), flags, list,
                                                       count, N, shrinks.n, shrinks, sse_rows,

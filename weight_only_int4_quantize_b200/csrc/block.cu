@@ -41,18 +41,32 @@ namespace {
 
 // ---------------------------------------------------------------------------
 // Batched fp64 GEMM: C[b] (+)= A[b] B[b / bdiv]^T (+ R) with arbitrary
-// strides.  CTA tile 64 (M) x 128 (N), 64-deep k steps staged in shared
-// memory; warp w owns rows 32 (w & 1) .. +31 and columns 32 (w >> 1) .. +31
-// as 4 x 4 MMA tiles of 8 x 8.
+// strides.  CTA tile 64 (M) x 128 (N); 32-deep k steps staged in shared
+// memory by asynchronous copies, two stages (the next step's copies are in
+// flight while this one's MMAs run); warp w owns rows 32 (w & 1) .. +31 and
+// columns 32 (w >> 1) .. +31 as 4 x 4 MMA tiles of 8 x 8.  A and a binary64
+// B are staged as doubles; a bf16 B (k contiguous) is staged as raw bf16 and
+// widened when its fragments are loaded (exact).
 // ---------------------------------------------------------------------------
-constexpr int kGM = 64, kGN = 128, kGK = 64;
-constexpr int kGLd = 68;  // doubles per staged row (64 + 4: conflict-free fragment loads)
-constexpr size_t kGemmSmem = static_cast<size_t>(kGM + kGN) * kGLd * sizeof(double);
+constexpr int kGM = 64, kGN = 128, kGK = 32;
+constexpr int kGLd = 36;   // doubles per staged row (32 + 4: conflict-free fragment loads)
+constexpr int kGLdH = 40;  // bf16 per staged row (32 + 8: conflict-free fragment loads)
+constexpr uint32_t kStageA = kGM * kGLd * 8;
+constexpr uint32_t kStageBd = kGN * kGLd * 8;
+constexpr uint32_t kStageBh = kGN * kGLdH * 2;
+template <typename TB>
+__host__ __device__ constexpr uint32_t gemm_stage_bytes() {
+  return kStageA + (sizeof(TB) == 8 ? kStageBd : kStageBh);
+}
+template <typename TB>
+constexpr size_t gemm_smem_bytes() {
+  return 2 * static_cast<size_t>(gemm_stage_bytes<TB>());
+}
 
 struct GemmArgs {
   const double* A;
   int64_t sAm, sAk, bA;
-  const void* B;  // double or bf16 bits
+  const void* B;  // double, or bf16 bits with sBk == 1
   int64_t sBn, sBk, bB;
   int bdiv;  // batch b reads B batch b / bdiv
   double* C;
@@ -68,78 +82,140 @@ __device__ __forceinline__ void dmma_m8n8k4(double (&d)[2], double a, double b) 
                : "d"(a), "d"(b));
 }
 
-__device__ __forceinline__ double load_b(const double* p, int64_t i) { return __ldg(p + i); }
-__device__ __forceinline__ double load_b(const uint16_t* p, int64_t i) {
-  return static_cast<double>(__uint_as_float(static_cast<uint32_t>(__ldg(p + i)) << 16));
+// Asynchronous copies global -> shared of 8 / 4 bytes; nothing is read (the
+// destination is zero-filled) when `valid` is false.
+__device__ __forceinline__ void cpa8(uint32_t dst, const void* src, bool valid) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;" ::"r"(dst), "l"(src),
+               "r"(valid ? 8 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void cpa4(uint32_t dst, const void* src, bool valid) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst), "l"(src),
+               "r"(valid ? 4 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void cpa_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cpa_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
-// Stages rows [r0, r0 + ROWS) x channels [k0, k0 + 64) of a strided operand
-// (zero outside [0, nrows) x [0, kend)) as dst[row][kGLd].
-template <int ROWS, typename T>
-__device__ __forceinline__ void stage_tile(double* dst, const T* src, int64_t s_row, int64_t s_k,
-                                           int r0, int nrows, int k0, int kend) {
+// Stages rows [r0, r0 + ROWS) x channels [k0, k0 + 32) of a strided binary64
+// operand (zero outside [0, nrows) x [0, kend)) as dst[row][kGLd].
+template <int ROWS>
+__device__ __forceinline__ void stage_f64(uint32_t dst, const double* src, int64_t s_row,
+                                          int64_t s_k, int r0, int nrows, int k0, int kend) {
   const int t = threadIdx.x;
   constexpr int kPer = ROWS * kGK / 256;
-  if (s_k == 1) {  // lanes along k
-    const int kk = t & 63;
+  if (s_k == 1) {  // lanes along k: a warp copies 256 contiguous bytes
+    const int kk = t & 31;
     const int k = k0 + kk;
-#pragma unroll 8
+#pragma unroll
     for (int j = 0; j < kPer; ++j) {
-      const int r = (t >> 6) + 4 * j;
+      const int r = (t >> 5) + 8 * j;
       const int row = r0 + r;
-      dst[r * kGLd + kk] = (row < nrows && k < kend) ? load_b(src, row * s_row + k) : 0.0;
+      const bool v = row < nrows && k < kend;
+      cpa8(dst + static_cast<uint32_t>(r * kGLd + kk) * 8u, v ? src + row * s_row + k : src, v);
     }
   } else {  // lanes along rows
     constexpr int kStep = 256 / ROWS;
     const int r = t % ROWS;
     const int row = r0 + r;
-#pragma unroll 8
+#pragma unroll
     for (int j = 0; j < kPer; ++j) {
       const int kk = t / ROWS + kStep * j;
       const int k = k0 + kk;
-      dst[r * kGLd + kk] = (row < nrows && k < kend) ? load_b(src, row * s_row + k * s_k) : 0.0;
+      const bool v = row < nrows && k < kend;
+      cpa8(dst + static_cast<uint32_t>(r * kGLd + kk) * 8u,
+           v ? src + row * s_row + k * s_k : src, v);
     }
   }
 }
 
+// Stages 128 rows x 32 channels of a bf16 operand with k contiguous (K and
+// k0 even) as raw bf16 pairs, dst[row][kGLdH].
+__device__ __forceinline__ void stage_bf16(uint32_t dst, const uint16_t* src, int64_t s_row,
+                                           int r0, int nrows, int k0, int kend) {
+  const int t = threadIdx.x;
+  const int pr = t & 15;
+  const int k = k0 + 2 * pr;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const int r = (t >> 4) + 16 * j;
+    const int row = r0 + r;
+    const bool v = row < nrows && k < kend;
+    cpa4(dst + static_cast<uint32_t>(r * kGLdH + 2 * pr) * 2u, v ? src + row * s_row + k : src, v);
+  }
+}
+
+__device__ __forceinline__ double bf16_bits_to_double(uint16_t h) {
+  return static_cast<double>(__uint_as_float(static_cast<uint32_t>(h) << 16));
+}
+
 template <typename TB>
 __global__ void __launch_bounds__(256, 2) gemm_f64_kernel(GemmArgs g) {
-  extern __shared__ __align__(16) double gsm[];
-  double* As = gsm;               // [64][kGLd]
-  double* Bs = gsm + kGM * kGLd;  // [128][kGLd]
+  constexpr bool kBf16 = sizeof(TB) == 2;
+  extern __shared__ __align__(16) uint8_t gsm[];
+  const uint32_t sbase = smem_u32(gsm);
   const int m0 = blockIdx.y * kGM, n0 = blockIdx.x * kGN;
   if (g.causal == 1 && n0 >= m0 + kGM) return;  // every key after every query
   const int b = blockIdx.z;
   const double* A = g.A + b * g.bA;
   const TB* B = static_cast<const TB*>(g.B) + (b / g.bdiv) * g.bB;
   const int kend = g.causal == 2 ? min(g.K, m0 + kGM) : g.K;
+  const int nk = (kend + kGK - 1) / kGK;
   const int t = threadIdx.x, lane = t & 31, wid = t >> 5;
   const int wr = wid & 1, wc = wid >> 1;
   const int fr = lane >> 2, fq = lane & 3;
+  auto stage = [&](int buf, int k0) {
+    const uint32_t st = sbase + buf * gemm_stage_bytes<TB>();
+    stage_f64<kGM>(st, A, g.sAm, g.sAk, m0, g.M, k0, kend);
+    if constexpr (kBf16)
+      stage_bf16(st + kStageA, reinterpret_cast<const uint16_t*>(B), g.sBn, n0, g.N, k0, kend);
+    else
+      stage_f64<kGN>(st + kStageA, reinterpret_cast<const double*>(B), g.sBn, g.sBk, n0, g.N, k0,
+                     kend);
+  };
   double acc[4][4][2];
 #pragma unroll
   for (int i = 0; i < 4; ++i)
 #pragma unroll
     for (int j = 0; j < 4; ++j) acc[i][j][0] = acc[i][j][1] = 0.0;
-  for (int k0 = 0; k0 < kend; k0 += kGK) {
-    __syncthreads();  // the previous step's tiles are consumed
-    stage_tile<kGM>(As, A, g.sAm, g.sAk, m0, g.M, k0, kend);
-    stage_tile<kGN>(Bs, B, g.sBn, g.sBk, n0, g.N, k0, kend);
-    __syncthreads();
-    const double* ea = As + (32 * wr + fr) * kGLd + fq;
-    const double* eb = Bs + (32 * wc + fr) * kGLd + fq;
-#pragma unroll 4
+  if (nk > 0) stage(0, 0);
+  cpa_commit();
+  for (int kt = 0; kt < nk; ++kt) {
+    if (kt + 1 < nk) {
+      stage((kt + 1) & 1, (kt + 1) * kGK);  // its buffer was consumed at step kt - 1
+      cpa_commit();
+      cpa_wait<1>();
+    } else {
+      cpa_wait<0>();
+    }
+    __syncthreads();  // every thread's copies of step kt have landed
+    const uint8_t* st = gsm + (kt & 1) * gemm_stage_bytes<TB>();
+    const double* ea = reinterpret_cast<const double*>(st) + (32 * wr + fr) * kGLd + fq;
+#pragma unroll
     for (int k4 = 0; k4 < kGK; k4 += 4) {
       double af[4], bf[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i) af[i] = ea[8 * i * kGLd + k4];
+      if constexpr (kBf16) {
+        const uint16_t* eb =
+            reinterpret_cast<const uint16_t*>(st + kStageA) + (32 * wc + fr) * kGLdH + fq;
 #pragma unroll
-      for (int j = 0; j < 4; ++j) bf[j] = eb[8 * j * kGLd + k4];
+        for (int j = 0; j < 4; ++j) bf[j] = bf16_bits_to_double(eb[8 * j * kGLdH + k4]);
+      } else {
+        const double* eb =
+            reinterpret_cast<const double*>(st + kStageA) + (32 * wc + fr) * kGLd + fq;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) bf[j] = eb[8 * j * kGLd + k4];
+      }
 #pragma unroll
       for (int i = 0; i < 4; ++i)
 #pragma unroll
         for (int j = 0; j < 4; ++j) dmma_m8n8k4(acc[i][j], af[i], bf[j]);
     }
+    __syncthreads();  // step kt's buffer is consumed before step kt + 2 refills it
   }
   double* C = g.C + b * g.bC;
   const double* R = g.R ? g.R + b * g.bC : nullptr;
@@ -361,7 +437,7 @@ __global__ void argmin_first_kernel(const double* __restrict__ v, int n, int32_t
 // ---------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------
-template <auto kern>
+template <auto kern, size_t kBytes>
 cudaError_t gemm_smem_attr() {
   static unsigned long long done = 0;
   int dev = 0;
@@ -369,7 +445,7 @@ cudaError_t gemm_smem_attr() {
   if (e != cudaSuccess) return e;
   if (dev < 64 && (__atomic_load_n(&done, __ATOMIC_ACQUIRE) & (1ull << dev))) return cudaSuccess;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(kGemmSmem));
+                           static_cast<int>(kBytes));
   if (e == cudaSuccess && dev < 64) __atomic_fetch_or(&done, 1ull << dev, __ATOMIC_RELEASE);
   return e;
 }
@@ -379,13 +455,17 @@ cudaError_t gemm(const GemmArgs& g, bool b_f64, int batch, cudaStream_t st) {
                   static_cast<unsigned>((g.M + kGM - 1) / kGM), static_cast<unsigned>(batch));
   cudaError_t e;
   if (b_f64) {
-    e = gemm_smem_attr<gemm_f64_kernel<double>>();
+    constexpr size_t kBytes = gemm_smem_bytes<double>();
+    e = gemm_smem_attr<gemm_f64_kernel<double>, kBytes>();
     if (e != cudaSuccess) return e;
-    gemm_f64_kernel<double><<<grid, 256, kGemmSmem, st>>>(g);
+    gemm_f64_kernel<double><<<grid, 256, kBytes, st>>>(g);
   } else {
-    e = gemm_smem_attr<gemm_f64_kernel<uint16_t>>();
+    // bf16 operands are the linears' weights: k contiguous, K even.
+    if (g.sBk != 1 || (g.K & 1) || (g.sBn & 1)) return cudaErrorInvalidValue;
+    constexpr size_t kBytes = gemm_smem_bytes<uint16_t>();
+    e = gemm_smem_attr<gemm_f64_kernel<uint16_t>, kBytes>();
     if (e != cudaSuccess) return e;
-    gemm_f64_kernel<uint16_t><<<grid, 256, kGemmSmem, st>>>(g);
+    gemm_f64_kernel<uint16_t><<<grid, 256, kBytes, st>>>(g);
   }
   return cudaGetLastError();
 }

@@ -372,6 +372,7 @@ __global__ void __launch_bounds__(kStreamThreads, MIN_CTAS)
   if (cp.bundle < units) compute_enter();
 
   uint32_t slot = 0;
+  const float zadd = (!SYM && t >= 2) ? 128.0f : 0.0f;
 #pragma unroll 1
   while (cp.bundle < units) {
     uint4 xv[4];
@@ -395,15 +396,17 @@ __global__ void __launch_bounds__(kStreamThreads, MIN_CTAS)
     cp_async_wait<S - 1>();
     const uint32_t src = ring + slot * kSlotBytes;
     const int sh = 16 * cpar;
+    const uint32_t hsel = cpar ? 0x3232u : 0x3210u;  // the value's half into the low 16 bits
 #pragma unroll
     for (int rt = 0; rt < kTiles; ++rt) {
       const uint4 wa = lds128s(src + rt * 1024 + lane * 16);
       const uint4 wb = lds128s(src + rt * 1024 + 512 + lane * 16);
-      const uint32_t v = (lds32s(src + kSlotCodes + rt * 128 + lane * 4) >> sh) & 0xFFFFu;
+      const uint32_t wv = lds32s(src + kSlotCodes + rt * 128 + lane * 4);
       const int q0 = lane & ~3;
-      const float sa = half_bits_to_float(__shfl_sync(0xffffffffu, v, q0 + 0));
-      const float sb = half_bits_to_float(__shfl_sync(0xffffffffu, v, q0 + 1));
       if constexpr (A8) {
+        const uint32_t v = (wv >> sh) & 0xFFFFu;
+        const float sa = half_bits_to_float(__shfl_sync(0xffffffffu, v, q0 + 0));
+        const float sb = half_bits_to_float(__shfl_sync(0xffffffffu, v, q0 + 1));
         // D = sum (q - z) x8 = sum q x8 - z * S (exact int32), then scale.
         int c[4];
         const uint4 x8[2] = {xv[0], xv[1]};
@@ -419,12 +422,17 @@ __global__ void __launch_bounds__(kStreamThreads, MIN_CTAS)
         acc[rt][2] = fmaf(sb, __int2float_rn(c[2] - zb * s0), acc[rt][2]);
         acc[rt][3] = fmaf(sb, __int2float_rn(c[3] - zb * s1), acc[rt][3]);
       } else {
+        // Each lane widens its own value once (a zero lane adds 128); the
+        // shuffles then move finished floats.
+        const float fv = half_bits_to_float(__byte_perm(wv, 0u, hsel) & 0xFFFFu) + zadd;
+        const float sa = __shfl_sync(0xffffffffu, fv, q0 + 0);
+        const float sb = __shfl_sync(0xffffffffu, fv, q0 + 1);
         float c[4];
         tile_group_s(c, wa, wb, xv);
         float za = 136.0f, zb = 136.0f;  // 128 + zero (symmetric: zero 8)
         if (!SYM) {
-          za = 128.0f + half_bits_to_float(__shfl_sync(0xffffffffu, v, q0 + 2));
-          zb = 128.0f + half_bits_to_float(__shfl_sync(0xffffffffu, v, q0 + 3));
+          za = __shfl_sync(0xffffffffu, fv, q0 + 2);
+          zb = __shfl_sync(0xffffffffu, fv, q0 + 3);
         }
         acc[rt][0] = fmaf(sa, fmaf(-za, xs[0], c[0]), acc[rt][0]);
         acc[rt][1] = fmaf(sa, fmaf(-za, xs[1], c[1]), acc[rt][1]);

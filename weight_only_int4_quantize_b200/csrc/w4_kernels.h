@@ -158,15 +158,17 @@ struct SegOffsets {
 cudaError_t launch_exact_rowsse(const void* x, int M, const void* w, int N, int K,
                                 const float* s_all, const ShrinkList& shrinks, int n_r,
                                 bool symmetric, const int* list, const int* count, int cap,
-                                const int* rowlist, const int* rowcount, double* rowsum,
+                                const int* rowlist, const int* rowcount, const uint32_t* cmask,
+                                const SegOffsets& seg, int n_seg, double* rowsum,
                                 cudaStream_t stream);
 cudaError_t launch_awq_flag(const double* sse, int n_seg, int n_a, int n_r, int c1, double tol,
-                            int cap, int* list, int* count, cudaStream_t stream);
+                            int cap, int* list, int* count, uint32_t* masks, cudaStream_t stream);
 // Token chunks of the binary64 kernel: its row sums are [cap][chunks][N].
 int exact_token_chunks(int M);
 cudaError_t launch_awq_exact_merge(const double* rowsum, int M, int N, const int* list,
-                                   const int* count, int cap, int n_seg, const SegOffsets& seg,
-                                   int n_c, double* sse, cudaStream_t stream);
+                                   const int* count, const uint32_t* masks, int cap, int n_seg,
+                                   const SegOffsets& seg, int n_c, double* sse,
+                                   cudaStream_t stream);
 cudaError_t launch_clip_exact(const void* x, int M, const void* w, int N, int K, const float* s,
                               const ShrinkList& shrinks, bool symmetric, double tol,
                               double* sse_rows, int32_t* choice, float* shrink_rows,
