@@ -465,9 +465,10 @@ typedef struct {
   const double* k_norm;  /* device float64 [head_dim] */
 } w4_block_weights;
 
-/* Workspace of awq_block_scoring_losses and awq_block_search for T tokens
- * (about (2 heads T^2 + 24 T max(hidden, ffn)) * 8 bytes plus the largest
- * group's binary64 candidate weights); 0 if cfg is NULL or T < 1. */
+/* Workspace of awq_block_scoring_losses and awq_block_search for T tokens:
+ * six sets of block activations (each about (heads T^2 + 16 T max(hidden,
+ * ffn)) * 8 bytes), the largest group's binary64 candidate weights and the
+ * fp16 copies of both blocks' weights; 0 if cfg is NULL or T < 1. */
 size_t w4_block_workspace_bytes(const w4_block_config* cfg, int64_t T);
 
 /*
@@ -510,11 +511,23 @@ w4_status awq_block_scoring_losses(const w4_block_config* cfg, const double* x, 
  * linears unclipped.  Groups are scored one at a time with the rest of
  * block i unquantized.  Ties go to the lowest index.
  *
+ * Every selection is screened first: the reference paths run once in
+ * binary64 with their intermediates kept, and a candidate's path is the
+ * reference plus its change, each linear's change a tcgen05 product of fp16
+ * operands scaled by exact powers of two (attention, norms and SwiGLU in
+ * binary64 on the full values).  The candidates whose screening loss is
+ * within 3e-4 (relative) of the least are scored again on the binary64 path
+ * of awq_block_scoring_losses, and the selection takes the least of those
+ * binary64 losses: the choices are those of the binary64 definition.  The
+ * call synchronizes the stream once per selection (the near-tie sets are
+ * read on the host).
+ *
  * choice_out     device int32 [11] out: alpha index per group (4), then
  *                shrink index per linear (7).
  * losses_out     device float64 [4 * n_alpha + 7 * n_shrink] out (the alpha
- *                losses per group, then the shrink losses per linear), or
- *                NULL.
+ *                losses per group, then the shrink losses per linear: the
+ *                binary64 value for a candidate of a near-tie set, else its
+ *                screening value), or NULL.
  * Other arguments and errors as awq_block_scoring_losses.
  */
 w4_status awq_block_search(const w4_block_config* cfg, const double* x, int64_t T,

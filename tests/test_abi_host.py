@@ -209,3 +209,70 @@ def test_binding_refuses_missized_companion_tensors(monkeypatch):
                          awq_s=torch.zeros(128))
     with pytest.raises(ValueError):
         w4.awq_clip_search_rows(x, torch.zeros(8, 128, dtype=torch.bfloat16), [1.0], False)
+
+
+def _block_structs(align_off=0, missing=None):
+    cfg = w4.BlockConfig(**w4.QWEN3_1P7B_BLOCK)
+    fields = {f[0]: A + 0x1000 * i + align_off for i, f in enumerate(w4._BlockWeights._fields_)}
+    if missing:
+        fields[missing] = None
+    return cfg, w4._BlockWeights(**fields)
+
+
+def test_block_validation(L):
+    """awq_block_scoring_losses / awq_block_search / w4_block_workspace_bytes
+    reject bad arguments before any device call."""
+    import numpy as np
+    by = ctypes.byref
+    cfg, blk = _block_structs()
+    ws_need = L.w4_block_workspace_bytes(by(cfg), 256)
+    assert ws_need > 0
+    # the workspace grows with T (the attention scores are heads x T^2)
+    assert L.w4_block_workspace_bytes(by(cfg), 512) > ws_need
+    assert L.w4_block_workspace_bytes(by(cfg), 0) == 0
+    assert L.w4_block_workspace_bytes(None, 256) == 0
+    bad = w4.BlockConfig(**dict(w4.QWEN3_1P7B_BLOCK, head_dim=96))
+    assert L.w4_block_workspace_bytes(by(bad), 256) == 0
+    al = np.array([0.0, 0.5], np.float32)
+    sh = np.array([1.0, 0.9], np.float32)
+    pa, ps = al.ctypes.data, sh.ctypes.data
+
+    def score(cfg_=cfg, x=A, t=256, blk_=blk, nxt=None, group=0, alphas=pa, na=2, shrinks=ps,
+              nr=2, only=-1, out=B, ws=A, wsb=None):
+        return L.awq_block_scoring_losses(
+            None if cfg_ is None else by(cfg_), x, t, None if blk_ is None else by(blk_),
+            None if nxt is None else by(nxt), group, alphas, na, shrinks, nr, 0, only, out, ws,
+            ws_need if wsb is None else wsb, None)
+
+    assert score(out=None) == 1                 # no output
+    assert score(group=4) == 1                  # group out of range
+    assert score(group=0, only=3) == 1          # o is not in qkv
+    assert score(group=2, only=6) == 1          # down is not in gate_up
+    assert score(cfg_=None) == 1
+    assert score(blk_=None) == 1
+    _, blk_missing = _block_structs(missing="k_norm")
+    assert score(blk_=blk_missing) == 1         # a missing gain
+    assert score(nxt=blk_missing) == 1          # the next block checked too
+    assert score(cfg_=bad) == 2                 # head_dim
+    assert score(cfg_=w4.BlockConfig(**dict(w4.QWEN3_1P7B_BLOCK, kv_heads=3))) == 2
+    assert score(t=0) == 2
+    assert score(t=8193) == 2
+    assert score(na=0) == 4
+    assert score(na=65) == 4
+    assert score(shrinks=np.array([1.0, 1.5], np.float32).ctypes.data) == 1
+    assert score(alphas=np.array([0.0, np.nan], np.float32).ctypes.data) == 1
+    _, blk_mis = _block_structs(align_off=8)
+    assert score(blk_=blk_mis) == 3             # misaligned weights
+    assert score(x=A + 8) == 3                  # misaligned input
+    assert score(out=B + 8) == 3                # misaligned losses
+    assert score(wsb=ws_need - 1) == 5          # workspace too small
+    assert score(ws=A + 128) == 3               # workspace not 256-byte aligned
+
+    def search(choice=B, losses=None, **kw):
+        return L.awq_block_search(by(cfg), A, 256, by(blk), None, pa, 2, ps, 2, 0, choice, losses,
+                                  A, kw.get("wsb", ws_need), None)
+
+    assert search(choice=None) == 1
+    assert search(choice=B + 4) == 3
+    assert search(losses=B + 8) == 3
+    assert search(wsb=16) == 5

@@ -829,7 +829,7 @@ w4_status awq_block_search(const w4_block_config* cfg, const double* x, int64_t 
   if (st != W4_OK) return st;
   return cuda_status(block_search(&c, x, T, bi, next ? &bn : nullptr, alphas, n_alpha, shrinks,
                                   n_shrink, symmetric != 0, choice_out, losses_out, workspace,
-                                  static_cast<cudaStream_t>(stream)),
+                                  static_cast<cudaStream_t>(stream), err),
                      "block-level search");
 }
 

@@ -271,19 +271,20 @@ __global__ void __launch_bounds__(256)
 // d / 32 channels per lane (lane + 32 j).
 template <int E>
 __global__ void __launch_bounds__(256)
-    qknorm_rope_kernel(double* __restrict__ x, int64_t rows, int heads,
+    qknorm_rope_kernel(const double* xin, double* x, int64_t rows, int heads,
                        const double* __restrict__ gain, double eps, double theta) {
   constexpr int d = 32 * E;
   const int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
   if (row >= rows) return;
   const int lane = threadIdx.x & 31;
   const int64_t pos = row / heads;
+  const double* xi = xin + row * d;  // may be x itself
   double* xr = x + row * d;
   double v[E];
   double ss = 0.0;
 #pragma unroll
   for (int j = 0; j < E; ++j) {
-    v[j] = xr[lane + 32 * j];
+    v[j] = xi[lane + 32 * j];
     ss = fma(v[j], v[j], ss);
   }
 #pragma unroll
@@ -360,7 +361,8 @@ __global__ void block_scales_kernel(const double* __restrict__ stat, int K, Alph
 // The candidate weight Q_r(W diag(s)) diag(1/s) in binary64: one warp per
 // (row, group of 128), lane l holds channels 4l .. 4l + 3 of the group.
 // Codes and scales are those of quant_group.cuh (the deployed quantizer).
-template <bool SYM>
+// DELTA: out = that weight minus W (binary64), the change a candidate makes.
+template <bool SYM, bool DELTA = false>
 __global__ void __launch_bounds__(256)
     candidate_weight_kernel(const uint16_t* __restrict__ w, int N, int K,
                             const float* __restrict__ s, float shrink,
@@ -395,11 +397,22 @@ __global__ void __launch_bounds__(256)
   for (int i = 0; i < 4; ++i) {
     const float what =
         __fmul_rn(__fsub_rn(static_cast<float>(code_of(v[i], gq)), gq.zero), gq.sc);  // exact
-    out[n * K + k0 + i] = static_cast<double>(what) / static_cast<double>(sk[i]);
+    const double wc = static_cast<double>(what) / static_cast<double>(sk[i]);
+    out[n * K + k0 + i] = DELTA ? __dsub_rn(wc, static_cast<double>(wf[i])) : wc;
   }
 }
 
 constexpr int kLossBlocks = 296;
+
+// A selection of the search decides in binary64 among the candidates whose
+// screening loss is within this relative distance of the least.  The
+// screening losses differ from the binary64 ones by far less (the fp16
+// roundings touch only each linear's change, about 2^-11 of it, and the
+// loss averages them over every token and hidden unit): at most 4.3e-5 on
+// Qwen3-1.7B-shaped blocks at 256 and 2048 tokens, both arms.  Two
+// candidates whose order the screening could invert are then both within
+// the tolerance; the tests hold the difference below half of it.
+constexpr double kBlockTieTol = 3e-4;
 
 // Per-block partial sums of (a - b)^2 (grid of kLossBlocks blocks).
 __global__ void __launch_bounds__(256)
@@ -425,13 +438,96 @@ __global__ void loss_finish_kernel(const double* __restrict__ partial, int64_t n
   out[0] = s / static_cast<double>(n);
 }
 
-// out[0] = the first index of the least of v[0 .. n).
-__global__ void argmin_first_kernel(const double* __restrict__ v, int n, int32_t* __restrict__ out) {
-  if (threadIdx.x != 0) return;
-  int best = 0;
-  for (int i = 1; i < n; ++i)
-    if (v[i] < v[best]) best = i;
-  out[0] = best;
+// ---------------------------------------------------------------------------
+// Screening kernels: fp16 tensor-core operands with power-of-two scaling
+// ---------------------------------------------------------------------------
+// partial[b] = max |a - b| (b may be null) over block b's grid-stride part.
+__global__ void __launch_bounds__(256)
+    absmax_partial_kernel(const double* __restrict__ a, const double* __restrict__ b, int64_t n,
+                          double* __restrict__ partial) {
+  __shared__ double red[8];
+  double m = 0.0;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x; i < n;
+       i += static_cast<int64_t>(kLossBlocks) * 256)
+    m = fmax(m, fabs(b ? __dsub_rn(a[i], b[i]) : a[i]));
+#pragma unroll
+  for (int o = 16; o; o >>= 1) m = fmax(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double r = red[0];
+    for (int i = 1; i < 8; ++i) r = fmax(r, red[i]);
+    partial[blockIdx.x] = r;
+  }
+}
+
+__global__ void __launch_bounds__(256)
+    absmax_partial_bf16_kernel(const uint16_t* __restrict__ w, int64_t n,
+                               double* __restrict__ partial) {
+  __shared__ double red[8];
+  float m = 0.f;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x; i < n;
+       i += static_cast<int64_t>(kLossBlocks) * 256)
+    m = fmaxf(m, fabsf(__uint_as_float(static_cast<uint32_t>(w[i]) << 16)));
+#pragma unroll
+  for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double r = red[0];
+    for (int i = 1; i < 8; ++i) r = fmax(r, red[i]);
+    partial[blockIdx.x] = r;
+  }
+}
+
+// The exponent e that puts the largest magnitude in [2^14, 2^15) (0 for an
+// all-zero tensor), from the partial maxima.
+__device__ __forceinline__ int f16_exponent(const double* __restrict__ partial) {
+  double m = 0.0;
+  for (int i = 0; i < kLossBlocks; ++i) m = fmax(m, partial[i]);
+  return m > 0.0 ? 14 - ilogb(m) : 0;
+}
+
+// out = fp16((a - b) * 2^e) (b may be null); *e_out = e.
+__global__ void __launch_bounds__(256)
+    to_f16_kernel(const double* __restrict__ a, const double* __restrict__ b, int64_t n,
+                  const double* __restrict__ partial, int* __restrict__ e_out,
+                  __half* __restrict__ out) {
+  __shared__ int se;
+  if (threadIdx.x == 0) {
+    se = f16_exponent(partial);
+    if (blockIdx.x == 0) *e_out = se;
+  }
+  __syncthreads();
+  const int e = se;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * 256)
+    out[i] = __double2half(ldexp(b ? __dsub_rn(a[i], b[i]) : a[i], e));
+}
+
+__global__ void __launch_bounds__(256)
+    bf16_to_f16_kernel(const uint16_t* __restrict__ w, int64_t n,
+                       const double* __restrict__ partial, int* __restrict__ e_out,
+                       __half* __restrict__ out) {
+  __shared__ int se;
+  if (threadIdx.x == 0) {
+    se = f16_exponent(partial);
+    if (blockIdx.x == 0) *e_out = se;
+  }
+  __syncthreads();
+  const int e = se;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * 256)
+    out[i] = __double2half(
+        ldexp(static_cast<double>(__uint_as_float(static_cast<uint32_t>(w[i]) << 16)), e));
+}
+
+// out = a + b elementwise (binary64).
+__global__ void add_f64_kernel(const double* __restrict__ a, const double* __restrict__ b,
+                               double* __restrict__ out, int64_t n) {
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x)
+    out[i] = __dadd_rn(a[i], b[i]);
 }
 
 // ---------------------------------------------------------------------------
@@ -512,14 +608,16 @@ cudaError_t run_rmsnorm(const Ctx& cx, const double* x, const double* gamma, dou
   return cudaGetLastError();
 }
 
-cudaError_t run_qknorm_rope(const Ctx& cx, double* x, int heads, const double* gain) {
+// out = the per-head norm and rotary embedding of in (in == out allowed).
+cudaError_t run_qknorm_rope(const Ctx& cx, const double* in, double* out, int heads,
+                            const double* gain) {
   const int64_t rows = static_cast<int64_t>(cx.T) * heads;
   const unsigned blocks = static_cast<unsigned>((rows + 7) / 8);
   if (cx.c->head_dim == 128)
-    qknorm_rope_kernel<4><<<blocks, 256, 0, cx.st>>>(x, rows, heads, gain, cx.c->eps,
+    qknorm_rope_kernel<4><<<blocks, 256, 0, cx.st>>>(in, out, rows, heads, gain, cx.c->eps,
                                                      cx.c->rope_theta);
   else
-    qknorm_rope_kernel<2><<<blocks, 256, 0, cx.st>>>(x, rows, heads, gain, cx.c->eps,
+    qknorm_rope_kernel<2><<<blocks, 256, 0, cx.st>>>(in, out, rows, heads, gain, cx.c->eps,
                                                      cx.c->rope_theta);
   return cudaGetLastError();
 }
@@ -543,8 +641,8 @@ cudaError_t forward_from(const Ctx& cx, int stage, const double* x, const Lin* W
     W4_TRY(linear(b.h, T, H, W[0].p, W[0].f64, nq, b.q, nullptr, cx.st));
     W4_TRY(linear(b.h, T, H, W[1].p, W[1].f64, nkv, b.k, nullptr, cx.st));
     W4_TRY(linear(b.h, T, H, W[2].p, W[2].f64, nkv, b.v, nullptr, cx.st));
-    W4_TRY(run_qknorm_rope(cx, b.q, c.heads, nm.q_norm));
-    W4_TRY(run_qknorm_rope(cx, b.k, c.kv_heads, nm.k_norm));
+    W4_TRY(run_qknorm_rope(cx, b.q, b.q, c.heads, nm.q_norm));
+    W4_TRY(run_qknorm_rope(cx, b.k, b.k, c.kv_heads, nm.k_norm));
     // S[h] = q_h k_{h/g}^T, causal tiles only.
     GemmArgs g{};
     g.A = b.q;
@@ -638,8 +736,13 @@ void linear_shape(const BlockConfig& c, int lin, int* n, int* k) {
 
 size_t rup(size_t b) { return (b + 255) & ~size_t{255}; }
 
+constexpr int kFBufs = 16;  // buffers of a screening forward (FBufs)
+
 struct Layout {
-  size_t bufsA[11], bufsB[11], out_a, out_b, ref, stat, s, wc, partial, loss, total;
+  size_t bufsA[11], bufsB[11], out_a, out_b, ref, stat, s, wc, partial, loss;
+  // Screening: reference and candidate sets of block i and block i+1, the
+  // fp16 weights, a candidate's weight change, fp16 operands, exponents.
+  size_t fset[4][kFBufs], w16[14], dw64, dw16[3], in16, d16, fpart, exps, floss, total;
 };
 
 Layout layout(const BlockConfig& c, int64_t T) {
@@ -685,6 +788,38 @@ Layout layout(const BlockConfig& c, int64_t T) {
   off += rup(kLossBlocks * sizeof(double));
   L.loss = off;
   off += rup(2 * kMaxGrid * 11 * sizeof(double));
+  // h ql kl v qr kr S a ap x1 h2 g u act mlp out
+  const size_t fw[kFBufs] = {H, nq, nkv, nkv, nq, nkv, 0, nq, H, H, H, F, F, F, H, H};
+  for (int set = 0; set < 4; ++set)
+    for (int i = 0; i < kFBufs; ++i) {
+      L.fset[set][i] = off;
+      const size_t elems = i == 6 ? static_cast<size_t>(c.heads) * Tz * Tz : Tz * fw[i];
+      off += rup(elems * sizeof(double));
+    }
+  size_t lmax = 0;
+  for (int l = 0; l < 14; ++l) {
+    int n, k;
+    linear_shape(c, l % 7, &n, &k);
+    L.w16[l] = off;
+    off += rup(static_cast<size_t>(n) * k * 2);
+    lmax = std::max(lmax, static_cast<size_t>(n) * k);
+  }
+  L.dw64 = off;
+  off += rup(lmax * sizeof(double));
+  for (int i = 0; i < 3; ++i) {
+    L.dw16[i] = off;
+    off += rup(lmax * 2);
+  }
+  L.in16 = off;
+  off += rup(Tz * kmax * 2);
+  L.d16 = off;
+  off += rup(Tz * kmax * 2);
+  L.fpart = off;
+  off += rup(kLossBlocks * sizeof(double));
+  L.exps = off;
+  off += rup(64 * sizeof(int));
+  L.floss = off;
+  off += rup(kMaxGrid * sizeof(double));
   L.total = off;
   return L;
 }
@@ -708,6 +843,7 @@ struct Session {
   bool sym;
   AlphaList al;
   ShrinkList sl;
+  unsigned* err;  // device error word (tcgen05 waits)
 };
 
 Session make_session(const BlockConfig* c, const double* x, int64_t T, const BlockLinears& blk,
@@ -810,6 +946,342 @@ cudaError_t candidate(const Session& s, int group, int ia, const int32_t* ia_dev
   return cudaGetLastError();
 }
 
+// ---------------------------------------------------------------------------
+// Screening forward.  The reference path keeps every intermediate in
+// binary64.  A candidate's path is then the reference plus its change: each
+// linear after the group is y_ref + (x - x_ref) W^T and each linear of the
+// group y_ref + x_ref (W_c - W)^T, the products on the tcgen05 tensor cores
+// with fp16 operands scaled by exact powers of two and binary64 epilogues;
+// norms, rotary embedding, attention and SwiGLU run in binary64 on the full
+// values.  The products round only the changes (about 2^-11 of each), so the
+// losses are close to the binary64 ones; selections decide their near ties
+// on the binary64 path.
+// ---------------------------------------------------------------------------
+struct FBufs {
+  double *h, *ql, *kl, *v, *qr, *kr, *S, *a, *ap, *x1, *h2, *g, *u, *act, *mlp, *out;
+};
+
+FBufs fbufs_at(uint8_t* ws, const size_t* off) {
+  double* p[kFBufs];
+  for (int i = 0; i < kFBufs; ++i) p[i] = reinterpret_cast<double*>(ws + off[i]);
+  return FBufs{p[0], p[1], p[2], p[3], p[4], p[5], p[6], p[7],
+               p[8], p[9], p[10], p[11], p[12], p[13], p[14], p[15]};
+}
+
+// Exponent slots: 0..6 block i's weights, 7..13 block i+1's, 14..16 the
+// group's weight changes, 17 the group's input, 18 the current change.
+constexpr int kSlotDw = 14, kSlotIn = 17, kSlotD = 18;
+
+#define W4_TRY(call)               \
+  do {                             \
+    cudaError_t e_ = (call);       \
+    if (e_ != cudaSuccess) return e_; \
+  } while (0)
+
+cudaError_t run_add(const Ctx& cx, const double* a, const double* b, double* out, int64_t n) {
+  add_f64_kernel<<<592, 256, 0, cx.st>>>(a, b, out, n);
+  return cudaGetLastError();
+}
+
+// q, k (after their norms and rotary embedding) and v -> S -> P -> a.
+cudaError_t attention(const Ctx& cx, const double* q, const double* k, const double* v, double* S,
+                      double* a) {
+  const BlockConfig& c = *cx.c;
+  const int T = cx.T, d = c.head_dim;
+  const int nq = c.heads * d, nkv = c.kv_heads * d;
+  GemmArgs g{};
+  g.A = q;
+  g.sAm = nq;
+  g.sAk = 1;
+  g.bA = d;
+  g.B = k;
+  g.sBn = nkv;
+  g.sBk = 1;
+  g.bB = d;
+  g.bdiv = c.heads / c.kv_heads;
+  g.C = S;
+  g.sCm = T;
+  g.sCn = 1;
+  g.bC = static_cast<int64_t>(T) * T;
+  g.M = T;
+  g.N = T;
+  g.K = d;
+  g.causal = 1;
+  W4_TRY(gemm(g, true, c.heads, cx.st));
+  const int64_t rows = static_cast<int64_t>(c.heads) * T;
+  softmax_causal_kernel<<<static_cast<unsigned>((rows + 7) / 8), 256, 0, cx.st>>>(
+      S, rows, T, sqrt(static_cast<double>(d)));
+  W4_TRY(cudaGetLastError());
+  GemmArgs p{};
+  p.A = S;
+  p.sAm = T;
+  p.sAk = 1;
+  p.bA = static_cast<int64_t>(T) * T;
+  p.B = v;
+  p.sBn = 1;
+  p.sBk = nkv;
+  p.bB = d;
+  p.bdiv = c.heads / c.kv_heads;
+  p.C = a;
+  p.sCm = nq;
+  p.sCn = 1;
+  p.bC = d;
+  p.M = T;
+  p.N = d;
+  p.K = T;
+  p.causal = 2;
+  return gemm(p, true, c.heads, cx.st);
+}
+
+// The reference path of one block with every intermediate kept (binary64;
+// the same kernels and order as forward_from, so the values are those of
+// the binary64 path).
+cudaError_t fwd_ref(const Ctx& cx, const double* x, const Lin* W, const BlockNorms& nm,
+                    const FBufs& R) {
+  const BlockConfig& c = *cx.c;
+  const int T = cx.T, H = c.hidden, nq = c.heads * c.head_dim, nkv = c.kv_heads * c.head_dim;
+  const int F = c.ffn;
+  const int64_t th = static_cast<int64_t>(T) * H;
+  W4_TRY(run_rmsnorm(cx, x, nm.ln1, R.h));
+  W4_TRY(linear(R.h, T, H, W[0].p, W[0].f64, nq, R.ql, nullptr, cx.st));
+  W4_TRY(linear(R.h, T, H, W[1].p, W[1].f64, nkv, R.kl, nullptr, cx.st));
+  W4_TRY(linear(R.h, T, H, W[2].p, W[2].f64, nkv, R.v, nullptr, cx.st));
+  W4_TRY(run_qknorm_rope(cx, R.ql, R.qr, c.heads, nm.q_norm));
+  W4_TRY(run_qknorm_rope(cx, R.kl, R.kr, c.kv_heads, nm.k_norm));
+  W4_TRY(attention(cx, R.qr, R.kr, R.v, R.S, R.a));
+  W4_TRY(linear(R.a, T, nq, W[3].p, W[3].f64, H, R.ap, nullptr, cx.st));
+  W4_TRY(run_add(cx, x, R.ap, R.x1, th));
+  W4_TRY(run_rmsnorm(cx, R.x1, nm.ln2, R.h2));
+  W4_TRY(linear(R.h2, T, H, W[4].p, W[4].f64, F, R.g, nullptr, cx.st));
+  W4_TRY(linear(R.h2, T, H, W[5].p, W[5].f64, F, R.u, nullptr, cx.st));
+  swiglu_f64_kernel<<<592, 256, 0, cx.st>>>(R.g, R.u, R.act, static_cast<int64_t>(T) * F);
+  W4_TRY(cudaGetLastError());
+  W4_TRY(linear(R.act, T, F, W[6].p, W[6].f64, H, R.mlp, nullptr, cx.st));
+  return run_add(cx, R.x1, R.mlp, R.out, th);
+}
+
+struct Screen {
+  const Session* s;
+  FBufs Ri, Rn, Ci, Cn;
+  __half* w16[14];
+  __half* dw16[3];
+  double* dw64;
+  __half* in16;
+  __half* d16;
+  double* part;
+  int* exps;
+  double* floss;
+};
+
+Screen make_screen(const Session& s) {
+  Screen z{};
+  z.s = &s;
+  z.Ri = fbufs_at(s.ws, s.L.fset[0]);
+  z.Rn = fbufs_at(s.ws, s.L.fset[1]);
+  z.Ci = fbufs_at(s.ws, s.L.fset[2]);
+  z.Cn = fbufs_at(s.ws, s.L.fset[3]);
+  for (int l = 0; l < 14; ++l) z.w16[l] = reinterpret_cast<__half*>(s.ws + s.L.w16[l]);
+  for (int i = 0; i < 3; ++i) z.dw16[i] = reinterpret_cast<__half*>(s.ws + s.L.dw16[i]);
+  z.dw64 = reinterpret_cast<double*>(s.ws + s.L.dw64);
+  z.in16 = reinterpret_cast<__half*>(s.ws + s.L.in16);
+  z.d16 = reinterpret_cast<__half*>(s.ws + s.L.d16);
+  z.part = reinterpret_cast<double*>(s.ws + s.L.fpart);
+  z.exps = reinterpret_cast<int*>(s.ws + s.L.exps);
+  z.floss = reinterpret_cast<double*>(s.ws + s.L.floss);
+  return z;
+}
+
+// out = fp16((a - b) 2^e), exps[slot] = e (b may be null).
+cudaError_t to_f16(const Screen& z, const double* a, const double* b, int64_t n, int slot,
+                   __half* out) {
+  const cudaStream_t st = z.s->cx.st;
+  absmax_partial_kernel<<<kLossBlocks, 256, 0, st>>>(a, b, n, z.part);
+  to_f16_kernel<<<592, 256, 0, st>>>(a, b, n, z.part, z.exps + slot, out);
+  return cudaGetLastError();
+}
+
+// out[T, N] = r1 (+ r2) + A B^T with A = fp16 operand of slot sa, B of slot sb.
+cudaError_t add_gemm(const Screen& z, const __half* a16, int sa, const __half* b16, int sb, int N,
+                     int K, double* out, const double* r1, const double* r2) {
+  return launch_add_gemm_f16(a16, z.s->cx.T, b16, N, K, out, N, r1, r2, z.exps + sa, z.exps + sb,
+                             z.s->cx.st, z.s->err);
+}
+
+// The reference paths and the fp16 weights of both blocks.
+cudaError_t screen_prepare(const Screen& z) {
+  const Session& s = *z.s;
+  const cudaStream_t st = s.cx.st;
+  for (int l = 0; l < (s.ahead ? 14 : 7); ++l) {
+    int n, k;
+    linear_shape(*s.c, l % 7, &n, &k);
+    const int64_t nk = static_cast<int64_t>(n) * k;
+    const auto* w = static_cast<const uint16_t*>(l < 7 ? s.Wi[l].p : s.Wn[l - 7].p);
+    absmax_partial_bf16_kernel<<<kLossBlocks, 256, 0, st>>>(w, nk, z.part);
+    bf16_to_f16_kernel<<<592, 256, 0, st>>>(w, nk, z.part, z.exps + l, z.w16[l]);
+    W4_TRY(cudaGetLastError());
+  }
+  W4_TRY(fwd_ref(s.cx, s.x, s.Wi, s.ni, z.Ri));
+  if (s.ahead) W4_TRY(fwd_ref(s.cx, z.Ri.out, s.Wn, s.nn, z.Rn));
+  return cudaSuccess;
+}
+
+// A group's statistic and its input in fp16 (slot kSlotIn).
+cudaError_t screen_group(const Screen& z, int group) {
+  const Session& s = *z.s;
+  const double* in[4] = {z.Ri.h, z.Ri.a, z.Ri.h2, z.Ri.act};
+  const int K = group_in_width(*s.c, group);
+  colmean_abs_f64_kernel<<<(K + 127) / 128, 128, 0, s.cx.st>>>(in[group], s.cx.T, K,
+                                                               ws_d(s, s.L.stat));
+  W4_TRY(cudaGetLastError());
+  return to_f16(z, in[group], nullptr, static_cast<int64_t>(s.cx.T) * K, kSlotIn, z.in16);
+}
+
+// Screening loss of one candidate (alpha index ia, ratio on linear `only`
+// or on every linear of the group) into loss_out (device).
+cudaError_t screen_candidate(const Screen& z, int group, int ia, float ratio, int only,
+                             double* loss_out) {
+  const Session& s = *z.s;
+  const BlockConfig& c = *s.c;
+  const cudaStream_t st = s.cx.st;
+  const int T = s.cx.T, H = c.hidden, nq = c.heads * c.head_dim, nkv = c.kv_heads * c.head_dim;
+  const int F = c.ffn;
+  const int64_t th = static_cast<int64_t>(T) * H;
+  const int K = group_in_width(c, group);
+  float* sv = reinterpret_cast<float*>(s.ws + s.L.s);
+  block_scales_kernel<<<(K + 127) / 128, 128, 0, st>>>(ws_d(s, s.L.stat), K, s.al, ia, nullptr,
+                                                       sv);
+  W4_TRY(cudaGetLastError());
+  // The group's weight changes, fp16 (slots kSlotDw + i).
+  for (int l = kGroupFirst[group]; l < kGroupFirst[group + 1]; ++l) {
+    int n, k;
+    linear_shape(c, l, &n, &k);
+    const float r = (only < 0 || only == l) ? ratio : 1.0f;
+    const int64_t items = static_cast<int64_t>(n) * (k / 128);
+    const unsigned blocks = static_cast<unsigned>((items + 7) / 8);
+    const auto* wb = static_cast<const uint16_t*>(s.Wi[l].p);
+    if (s.sym)
+      candidate_weight_kernel<true, true><<<blocks, 256, 0, st>>>(wb, n, k, sv, r, z.dw64);
+    else
+      candidate_weight_kernel<false, true><<<blocks, 256, 0, st>>>(wb, n, k, sv, r, z.dw64);
+    W4_TRY(cudaGetLastError());
+    const int i = l - kGroupFirst[group];
+    W4_TRY(to_f16(z, z.dw64, nullptr, static_cast<int64_t>(n) * k, kSlotDw + i, z.dw16[i]));
+  }
+  const FBufs &R = z.Ri, &C = z.Ci;
+  // Block i from the group on.
+  if (group == 0) {
+    W4_TRY(add_gemm(z, z.in16, kSlotIn, z.dw16[0], kSlotDw + 0, nq, H, C.ql, R.ql, nullptr));
+    W4_TRY(add_gemm(z, z.in16, kSlotIn, z.dw16[1], kSlotDw + 1, nkv, H, C.kl, R.kl, nullptr));
+    W4_TRY(add_gemm(z, z.in16, kSlotIn, z.dw16[2], kSlotDw + 2, nkv, H, C.v, R.v, nullptr));
+    W4_TRY(run_qknorm_rope(s.cx, C.ql, C.qr, c.heads, s.ni.q_norm));
+    W4_TRY(run_qknorm_rope(s.cx, C.kl, C.kr, c.kv_heads, s.ni.k_norm));
+    W4_TRY(attention(s.cx, C.qr, C.kr, C.v, C.S, C.a));
+    W4_TRY(to_f16(z, C.a, R.a, static_cast<int64_t>(T) * nq, kSlotD, z.d16));
+    W4_TRY(add_gemm(z, z.d16, kSlotD, z.w16[3], 3, H, nq, C.x1, s.x, R.ap));
+  } else if (group == 1) {
+    W4_TRY(add_gemm(z, z.in16, kSlotIn, z.dw16[0], kSlotDw, H, nq, C.x1, R.x1, nullptr));
+  }
+  if (group <= 1) {
+    W4_TRY(run_rmsnorm(s.cx, C.x1, s.ni.ln2, C.h2));
+    W4_TRY(to_f16(z, C.h2, R.h2, th, kSlotD, z.d16));
+    W4_TRY(add_gemm(z, z.d16, kSlotD, z.w16[4], 4, F, H, C.g, R.g, nullptr));
+    W4_TRY(add_gemm(z, z.d16, kSlotD, z.w16[5], 5, F, H, C.u, R.u, nullptr));
+  } else if (group == 2) {
+    W4_TRY(add_gemm(z, z.in16, kSlotIn, z.dw16[0], kSlotDw + 0, F, H, C.g, R.g, nullptr));
+    W4_TRY(add_gemm(z, z.in16, kSlotIn, z.dw16[1], kSlotDw + 1, F, H, C.u, R.u, nullptr));
+  }
+  if (group <= 2) {
+    swiglu_f64_kernel<<<592, 256, 0, st>>>(C.g, C.u, C.act, static_cast<int64_t>(T) * F);
+    W4_TRY(cudaGetLastError());
+    W4_TRY(to_f16(z, C.act, R.act, static_cast<int64_t>(T) * F, kSlotD, z.d16));
+    W4_TRY(add_gemm(z, z.d16, kSlotD, z.w16[6], 6, H, F, C.out, group <= 1 ? C.x1 : R.x1,
+                    R.mlp));
+  } else {
+    W4_TRY(add_gemm(z, z.in16, kSlotIn, z.dw16[0], kSlotDw, H, F, C.out, R.out, nullptr));
+  }
+  const double* fin = C.out;
+  const double* ref = R.out;
+  if (s.ahead) {
+    // Block i+1 on the changed input: every linear is y_ref + change.
+    const FBufs &Rn = z.Rn, &Cn = z.Cn;
+    W4_TRY(run_rmsnorm(s.cx, C.out, s.nn.ln1, Cn.h));
+    W4_TRY(to_f16(z, Cn.h, Rn.h, th, kSlotD, z.d16));
+    W4_TRY(add_gemm(z, z.d16, kSlotD, z.w16[7], 7, nq, H, Cn.ql, Rn.ql, nullptr));
+    W4_TRY(add_gemm(z, z.d16, kSlotD, z.w16[8], 8, nkv, H, Cn.kl, Rn.kl, nullptr));
+    W4_TRY(add_gemm(z, z.d16, kSlotD, z.w16[9], 9, nkv, H, Cn.v, Rn.v, nullptr));
+    W4_TRY(run_qknorm_rope(s.cx, Cn.ql, Cn.qr, c.heads, s.nn.q_norm));
+    W4_TRY(run_qknorm_rope(s.cx, Cn.kl, Cn.kr, c.kv_heads, s.nn.k_norm));
+    W4_TRY(attention(s.cx, Cn.qr, Cn.kr, Cn.v, Cn.S, Cn.a));
+    W4_TRY(to_f16(z, Cn.a, Rn.a, static_cast<int64_t>(T) * nq, kSlotD, z.d16));
+    W4_TRY(add_gemm(z, z.d16, kSlotD, z.w16[10], 10, H, nq, Cn.x1, C.out, Rn.ap));
+    W4_TRY(run_rmsnorm(s.cx, Cn.x1, s.nn.ln2, Cn.h2));
+    W4_TRY(to_f16(z, Cn.h2, Rn.h2, th, kSlotD, z.d16));
+    W4_TRY(add_gemm(z, z.d16, kSlotD, z.w16[11], 11, F, H, Cn.g, Rn.g, nullptr));
+    W4_TRY(add_gemm(z, z.d16, kSlotD, z.w16[12], 12, F, H, Cn.u, Rn.u, nullptr));
+    swiglu_f64_kernel<<<592, 256, 0, st>>>(Cn.g, Cn.u, Cn.act, static_cast<int64_t>(T) * F);
+    W4_TRY(cudaGetLastError());
+    W4_TRY(to_f16(z, Cn.act, Rn.act, static_cast<int64_t>(T) * F, kSlotD, z.d16));
+    W4_TRY(add_gemm(z, z.d16, kSlotD, z.w16[13], 13, H, F, Cn.out, Cn.x1, Rn.mlp));
+    fin = Cn.out;
+    ref = Rn.out;
+  }
+  double* part = ws_d(s, s.L.partial);
+  sqdiff_partial_kernel<<<kLossBlocks, 256, 0, st>>>(fin, ref, th, part);
+  loss_finish_kernel<<<1, 32, 0, st>>>(part, th, loss_out);
+  return cudaGetLastError();
+}
+
+__global__ void set_int_kernel(int32_t* p, int v) {
+  if (threadIdx.x == 0) *p = v;
+}
+
+// One selection of the search: screening losses of n candidates (cand(i)
+// = alpha index, ratio), near ties decided on the binary64 path.  Returns
+// the chosen index in *pick; losses (device, n) receive the values used.
+template <typename CandFn>
+cudaError_t screened_select(const Screen& z, int group, int n, int only, CandFn cand,
+                            double* losses, int* pick) {
+  const Session& s = *z.s;
+  for (int i = 0; i < n; ++i) {
+    int ia;
+    float r;
+    cand(i, &ia, &r);
+    W4_TRY(screen_candidate(z, group, ia, r, only, losses + i));
+  }
+  double host[kMaxGrid];
+  W4_TRY(cudaMemcpyAsync(host, losses, sizeof(double) * n, cudaMemcpyDeviceToHost, s.cx.st));
+  W4_TRY(cudaStreamSynchronize(s.cx.st));
+  double mn = host[0];
+  for (int i = 1; i < n; ++i) mn = fmin(mn, host[i]);
+  int members = 0;
+  bool near[kMaxGrid];
+  for (int i = 0; i < n; ++i) {
+    near[i] = host[i] <= mn * (1.0 + kBlockTieTol);
+    members += near[i];
+  }
+  if (members >= 2) {
+    // Binary64 losses of the near set (the exact path recomputes its own
+    // reference into its buffers).
+    W4_TRY(reference(s, group));
+    for (int i = 0; i < n; ++i)
+      if (near[i]) {
+        int ia;
+        float r;
+        cand(i, &ia, &r);
+        W4_TRY(candidate(s, group, ia, nullptr, r, only, losses + i));
+      }
+    W4_TRY(cudaMemcpyAsync(host, losses, sizeof(double) * n, cudaMemcpyDeviceToHost, s.cx.st));
+    W4_TRY(cudaStreamSynchronize(s.cx.st));
+  }
+  int best = -1;
+  for (int i = 0; i < n; ++i)
+    if (near[i] && (best < 0 || host[i] < host[best])) best = i;
+  *pick = best;
+  return cudaSuccess;
+}
+
+#undef W4_TRY
+
 }  // namespace
 
 size_t block_workspace_bytes(const BlockConfig& c, int64_t T) { return layout(c, T).total; }
@@ -834,28 +1306,42 @@ cudaError_t block_scoring_losses(const BlockConfig* c, const double* x, int64_t 
 cudaError_t block_search(const BlockConfig* c, const double* x, int64_t T, const BlockLinears& blk,
                          const BlockLinears* next, const float* alphas, int n_alpha,
                          const float* shrinks, int n_shrink, bool sym, int32_t* choice,
-                         double* losses, void* workspace, cudaStream_t st) {
+                         double* losses, void* workspace, cudaStream_t st, unsigned* err) {
   Session s = make_session(c, x, T, blk, next, alphas, n_alpha, shrinks, n_shrink, sym,
                            workspace, st);
+  s.err = err;
+  const Screen z = make_screen(s);
   double* lbuf = losses ? losses : ws_d(s, s.L.loss);
-  double* alpha_l = lbuf;                       // [4][n_alpha]
-  double* shrink_l = lbuf + 4 * n_alpha;        // [7][n_shrink]
+  double* alpha_l = lbuf;                 // [4][n_alpha]
+  double* shrink_l = lbuf + 4 * n_alpha;  // [7][n_shrink]
+  cudaError_t e = screen_prepare(z);
+  if (e != cudaSuccess) return e;
   for (int group = 0; group < 4; ++group) {
-    cudaError_t e = reference(s, group);
+    e = screen_group(z, group);
     if (e != cudaSuccess) return e;
-    for (int a = 0; a < n_alpha; ++a) {
-      e = candidate(s, group, a, nullptr, 1.0f, -1, alpha_l + group * n_alpha + a);
-      if (e != cudaSuccess) return e;
-    }
-    argmin_first_kernel<<<1, 32, 0, st>>>(alpha_l + group * n_alpha, n_alpha, choice + group);
+    int a_star = 0;
+    e = screened_select(
+        z, group, n_alpha, -1,
+        [&](int i, int* ia, float* r) {
+          *ia = i;
+          *r = 1.0f;
+        },
+        alpha_l + group * n_alpha, &a_star);
+    if (e != cudaSuccess) return e;
+    set_int_kernel<<<1, 32, 0, st>>>(choice + group, a_star);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     for (int l = kGroupFirst[group]; l < kGroupFirst[group + 1]; ++l) {
-      for (int j = 0; j < n_shrink; ++j) {
-        e = candidate(s, group, 0, choice + group, shrinks[j], l, shrink_l + l * n_shrink + j);
-        if (e != cudaSuccess) return e;
-      }
-      argmin_first_kernel<<<1, 32, 0, st>>>(shrink_l + l * n_shrink, n_shrink, choice + 4 + l);
+      int r_star = 0;
+      e = screened_select(
+          z, group, n_shrink, l,
+          [&](int i, int* ia, float* r) {
+            *ia = a_star;
+            *r = shrinks[i];
+          },
+          shrink_l + l * n_shrink, &r_star);
+      if (e != cudaSuccess) return e;
+      set_int_kernel<<<1, 32, 0, st>>>(choice + 4 + l, r_star);
       e = cudaGetLastError();
       if (e != cudaSuccess) return e;
     }

@@ -60,7 +60,7 @@ struct Tile {
 };
 
 enum : int { kBDequant = 0, kBTma = 1 };
-enum : int { kEpiStoreBf16 = 0, kEpiSumSquares = 1, kEpiColSumSquares = 2 };
+enum : int { kEpiStoreBf16 = 0, kEpiSumSquares = 1, kEpiColSumSquares = 2, kEpiAddF64 = 3 };
 
 constexpr unsigned kKernelIdGemm = 2;
 
@@ -84,6 +84,14 @@ struct SumSqArgs {
   int n_seg;
   int seg_off[17];      // column (N) boundaries, multiples of 16 inside
   int tiles;            // m_tiles * n_tiles
+  // Binary64 accumulate epilogue: out = r1 (+ r2) + 2^-(*ea + *eb) * acc,
+  // row pitch ldc.
+  double* out;
+  const double* r1;
+  const double* r2;
+  const int* ea;
+  const int* eb;
+  int ldc;
 };
 
 // A prefill launch decodes a group of linears that share the token count:
@@ -466,6 +474,32 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         }
+      } else if (EPI == kEpiAddF64) {
+        // out = r1 (+ r2) + 2^-(ea + eb) acc in binary64: the operands were
+        // scaled by exact powers of two, which the epilogue removes exactly.
+        const double scale = ldexp(1.0, -(*ss.ea + *ss.eb));
+        for (int mt = 0; mt < MT; ++mt)
+          for (int c = 0; c < NB / 32; ++c) {
+            const int m = m0 + 128 * mt + 32 * q + lane;
+            const int col = (NB / 2) * ch + 16 * c;
+            uint32_t r[16];
+            tmem_ld_32x32b_x16(tmem_base + (static_cast<uint32_t>(32 * q) << 16) + NB * mt + col,
+                               r);
+            tmem_ld_wait();
+            const int n = n0 + col;
+            if (m < M) {
+              const size_t o = static_cast<size_t>(m) * ss.ldc + n;
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                if (n + i < N) {
+                  double v = ss.r1[o + i];
+                  if (ss.r2) v = __dadd_rn(v, ss.r2[o + i]);
+                  ss.out[o + i] =
+                      __dadd_rn(v, __dmul_rn(scale, static_cast<double>(__uint_as_float(r[i]))));
+                }
+              }
+            }
+          }
       } else if (EPI == kEpiColSumSquares) {
         // Column sums of y^2 over the tile's rows: per 16-column chunk each
         // thread squares its row's 16 values (its row of each 128-row half
@@ -861,6 +895,38 @@ cudaError_t launch_sumsq_gemm(const void* a_f16, int M, const void* b_f16, int N
                        SmemLayout<2, BN>::bytes>(grid, false, stream, ta, tb, kNoGroup, ss, M, N,
                                                  K, 0, err);
   return launch_gemm<gemm_tc_kernel<kBTma, kEpiSumSquares, false, 1, BN>, SmemLayout<1, BN>::bytes>(
+      grid, false, stream, ta, tb, kNoGroup, ss, M, N, K, 0, err);
+}
+
+cudaError_t launch_add_gemm_f16(const void* a_f16, int M, const void* b_f16, int N, int K,
+                                double* out, int ldc, const double* r1, const double* r2,
+                                const int* ea, const int* eb, cudaStream_t stream,
+                                unsigned* err) {
+  if (K % BK != 0) return cudaErrorInvalidValue;
+  CUtensorMap ta, tb;
+  const uint64_t da[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(M)};
+  const uint64_t sa[1] = {static_cast<uint64_t>(K) * 2};
+  const int mt = sumsq_mt(M);
+  const uint32_t ba[2] = {BK, static_cast<uint32_t>(mt * BM)};
+  if (encode_tmap(&ta, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, da, sa, ba, a_f16) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+  const uint64_t db[3] = {static_cast<uint64_t>(K), static_cast<uint64_t>(N), 1};
+  const uint64_t sb[2] = {static_cast<uint64_t>(K) * 2, static_cast<uint64_t>(K) * 2 * N};
+  const uint32_t bb[3] = {BK, BN, 1};
+  if (encode_tmap(&tb, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, db, sb, bb, b_f16) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+  SumSqArgs ss = {};
+  ss.out = out;
+  ss.r1 = r1;
+  ss.r2 = r2;
+  ss.ea = ea;
+  ss.eb = eb;
+  ss.ldc = ldc;
+  dim3 grid((N + BN - 1) / BN, (M + mt * BM - 1) / (mt * BM), 1);
+  if (mt == 2)
+    return launch_gemm<gemm_tc_kernel<kBTma, kEpiAddF64, false, 2, BN>, SmemLayout<2, BN>::bytes>(
+        grid, false, stream, ta, tb, kNoGroup, ss, M, N, K, 0, err);
+  return launch_gemm<gemm_tc_kernel<kBTma, kEpiAddF64, false, 1, BN>, SmemLayout<1, BN>::bytes>(
       grid, false, stream, ta, tb, kNoGroup, ss, M, N, K, 0, err);
 }
 

@@ -175,6 +175,14 @@ cudaError_t launch_clip_exact(const void* x, int M, const void* w, int N, int K,
                               uint8_t* flags, unsigned long long* mask, int* list, int* count,
                               int* rows, int* row_counts, double* rowsum, cudaStream_t stream);
 
+// C[M, N] (pitch ldc, binary64) = r1 (+ r2) + 2^-(*ea + *eb) * A B^T with A
+// fp16 [M, K] and B fp16 [N, K] row-major (K a multiple of 64), on the
+// tcgen05 tensor cores with TMA-fed operands (gemm_tc.cu).
+cudaError_t launch_add_gemm_f16(const void* a_f16, int M, const void* b_f16, int N, int K,
+                                double* out, int ldc, const double* r1, const double* r2,
+                                const int* ea, const int* eb, cudaStream_t stream,
+                                unsigned* err);
+
 // Block-level candidate scoring in binary64 (block.cu).  Linears in the
 // order q, k, v, o, gate, up, down (bf16 [out, in]); groups 0 qkv, 1 o,
 // 2 gate_up, 3 down.
@@ -201,7 +209,7 @@ cudaError_t block_scoring_losses(const BlockConfig* c, const double* x, int64_t 
 cudaError_t block_search(const BlockConfig* c, const double* x, int64_t T, const BlockLinears& blk,
                          const BlockLinears* next, const float* alphas, int n_alpha,
                          const float* shrinks, int n_shrink, bool sym, int32_t* choice,
-                         double* losses, void* workspace, cudaStream_t st);
+                         double* losses, void* workspace, cudaStream_t st, unsigned* err);
 
 // Device address of the fixed scratch behind awq_score_grid_static_scratch
 // on the current device (looked up once per device, then cached).
