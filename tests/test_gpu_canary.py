@@ -141,3 +141,45 @@ def test_scoring_outputs_guarded():
     assert st == 0
     for g, name in ((rows_sse, "row sse"), (choice, "choice"), (rows, "ratios"), (cws, "workspace")):
         g.check(name)
+
+
+@pytest.mark.parametrize("ahead", [True, False])
+def test_block_scoring_outputs_guarded(ahead):
+    """Block-level losses and search: the losses, the choices and the whole
+    workspace between guards, at a ragged token count (partial row tiles and
+    causal tiles cut mid-way) on a small block."""
+    cfg = {"hidden": 256, "heads": 4, "kv_heads": 2, "head_dim": 64, "ffn": 384, "eps": 1e-6,
+           "rope_theta": 1e4}
+    t = 70
+    blk = {k: v.to(DEV) for k, v in synth.block_of_shape(cfg, 900).items()}
+    nxt = {k: v.to(DEV) for k, v in synth.block_of_shape(cfg, 950).items()} if ahead else None
+    x = synth.block_input(t, cfg["hidden"], seed=901).to(DEV)
+    al = synth.alpha_grid(20)[[2, 9, 16]]
+    sh = synth.shrink_grid(10)[[0, 4]]
+    need = w4.block_workspace_bytes(t, cfg)
+    ws = Guarded((need,), torch.uint8)
+    losses = Guarded((3, 2), torch.float64)
+    c = w4.BlockConfig(**cfg)
+    import ctypes
+    bi = w4._block_weights(blk, x)
+    bn = w4._block_weights(nxt, x)
+    al32, sh32 = np.ascontiguousarray(al), np.ascontiguousarray(sh)
+    st = torch.cuda.current_stream().cuda_stream
+    assert w4.lib().awq_block_scoring_losses(
+        ctypes.byref(c), x.data_ptr(), t, ctypes.byref(bi),
+        None if bn is None else ctypes.byref(bn), 0, al32.ctypes.data, 3, sh32.ctypes.data, 2, 0,
+        -1, losses.t.data_ptr(), ws.t.data_ptr(), need, st) == 0
+    losses.check("block losses")
+    ws.check("block workspace (losses)")
+    assert bool(torch.isfinite(losses.t).all())
+    choice = Guarded((11,), torch.int32)
+    sl = Guarded((4 * 3 + 7 * 2,), torch.float64)
+    assert w4.lib().awq_block_search(
+        ctypes.byref(c), x.data_ptr(), t, ctypes.byref(bi),
+        None if bn is None else ctypes.byref(bn), al32.ctypes.data, 3, sh32.ctypes.data, 2, 1,
+        choice.t.data_ptr(), sl.t.data_ptr(), ws.t.data_ptr(), need, st) == 0
+    choice.check("block choices")
+    sl.check("block search losses")
+    ws.check("block workspace (search)")
+    ch = choice.t.cpu().numpy()
+    assert ((ch[:4] >= 0) & (ch[:4] < 3)).all() and ((ch[4:] >= 0) & (ch[4:] < 2)).all()
