@@ -52,11 +52,11 @@ FALLBACK_BF16_TFLOPS = 1590.0
 # summaries under profiles/ give the commands), with the digest of the kernel
 # source the capture was taken on.  A changed source reports traffic null.
 TRAFFIC_CAPTURES = {
-    # decode_batch --m 1 --blocks 4 (streaming kernel, 28 linears): 110.43 MB
-    # (107.27 read + 3.16 written back from the preceding quantize) over
+    # decode_batch --m 1 --blocks 4 (streaming kernel, 28 linears): 110.71 MB
+    # (107.27 read + 3.43 written back from the preceding quantize) over
     # 107.27 MB algorithmic
-    "gemv_w4a16": {"source": "gemv_stream.cu", "digest": "094c567067a0bb3b",
-                   "ratio": (107269888 + 3163904) / 107266048},
+    "gemv_w4a16": {"source": "gemv_stream.cu", "digest": "47877b2f04a984c7",
+                   "ratio": (107271424 + 3434240) / 107266048},
     # quantize 17408 x 5120: 202.47 MB over 225.67 MB (part of the written codes
     # is still in the write-back L2 when the kernel ends)
     "quantize_pack": {"source": "quantize.cu", "digest": "f3061dcc5ac9fd85", "ratio": 202.47 / 225.67},
@@ -575,16 +575,17 @@ def breakdown(torch, dev, hbm, bf16_peak, bf16_sus):
     del cws, wg, x
     torch.cuda.empty_cache()
 
-    # Block-level (look-ahead) search of one Qwen3-1.7B-shaped block in
-    # binary64: T = 2048 tokens entering block i, block i+1 unquantized, the
-    # 20 x 10 grid (alpha* per group: 4 x 20 candidates, then a ratio per
-    # linear: 7 x 10), every candidate two block forwards from the group on.
+    # Block-level (look-ahead) search of one Qwen3-1.7B-shaped block: T =
+    # 2048 tokens entering block i, block i+1 unquantized, the 20 x 10 grid
+    # (alpha* per group: 4 x 20 candidates, then a ratio per linear: 7 x 10),
+    # every candidate screened (tcgen05 fp16 products of each linear's change,
+    # binary64 epilogues and attention), near ties decided in binary64.
     gi = {k: v.to(dev) for k, v in synth.qwen_block(3).items()}
     gn = {k: v.to(dev) for k, v in synth.qwen_block(4).items()}
     xb = synth.block_input(2048, 2048, seed=77).to(dev)
     wsb = torch.empty(w4.block_workspace_bytes(2048), dtype=torch.uint8, device=dev)
     al, sh = synth.alpha_grid(20), synth.shrink_grid(10)
-    w4.awq_block_scoring_losses(xb, gi, gn, "down", al[:1], sh[:1], False, workspace=wsb)
+    w4.awq_block_search(xb, gi, gn, al[:1], sh[:1], False, workspace=wsb)  # warm
     torch.cuda.synchronize()
     a_ev, b_ev = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a_ev.record()
@@ -595,7 +596,8 @@ def breakdown(torch, dev, hbm, bf16_peak, bf16_sus):
     out["block_search_qwen_T2048_20x10_lookahead"] = {
         "ms": t, "candidates": 4 * 20 + 7 * 10, "candidates_per_s": 150 / (t * 1e-3),
         "workspace_gb": wsb.numel() / 1e9, "choice": choice.tolist(),
-        "precision": "binary64 (fp64 MMA GEMMs)"}
+        "precision": "screened: tcgen05 fp16 change products with binary64 epilogues; "
+                     "near ties (3e-4) decided on the binary64 path"}
     del gi, gn, xb, wsb
     torch.cuda.empty_cache()
     return out
