@@ -516,7 +516,7 @@ w4_status awq_block_scoring_losses(const w4_block_config* cfg, const double* x, 
  * reference plus its change, each linear's change a tcgen05 product of fp16
  * operands scaled by exact powers of two (attention, norms and SwiGLU in
  * binary64 on the full values).  The candidates whose screening loss is
- * within 3e-4 (relative) of the least are scored again on the binary64 path
+ * within 1e-3 (relative) of the least are scored again on the binary64 path
  * of awq_block_scoring_losses, and the selection takes the least of those
  * binary64 losses: the choices are those of the binary64 definition.  The
  * call synchronizes the stream once per selection (the near-tie sets are

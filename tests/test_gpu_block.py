@@ -24,10 +24,10 @@ pytestmark = pytest.mark.gpu
 
 LOSS_RTOL = 1e-9
 # awq_block_search reports screening losses for candidates outside every
-# near-tie set; they must stay within half of its tie tolerance (3e-4) of
+# near-tie set; they must stay within half of its tie tolerance (1e-3) of
 # the binary64 values for the screening to be sound (two candidates whose
 # errors have opposite signs still both fall within the tolerance).
-SCREEN_RTOL = 1.5e-4
+SCREEN_RTOL = 5e-4
 T = 256
 CFG = dict(B.QWEN3_1P7B)
 
@@ -134,11 +134,10 @@ SMALL = {"hidden": 256, "heads": 4, "kv_heads": 4, "head_dim": 64, "ffn": 512, "
          "rope_theta": 1e4}  # multi-head (no grouping), 64-wide heads
 
 
-def _small_blocks(cfg, t, seed):
-    torch = _torch()
+def _small_blocks(cfg, t, seed, n_out=0, scale=1.0):
     out = []
     for b in (0, 1):
-        cpu = synth.block_of_shape(cfg, seed + 50 * b)
+        cpu = synth.block_of_shape(cfg, seed + 50 * b, n_outliers=n_out, outlier_scale=scale)
         bits = {n: synth.bits(cpu[n]) for n in synth.BLOCK_LINEAR_NAMES}
         norms = {n: cpu[n].numpy() for n in ("ln1", "ln2", "q_norm", "k_norm")}
         out.append(({n: v.to("cuda") for n, v in cpu.items()}, bits, norms))
@@ -160,20 +159,26 @@ def test_block_losses_ragged_and_single_token(blocks, t):
     _check_losses(got, ref, f"T={t}")
 
 
-@pytest.mark.parametrize("ahead", [True, False], ids=["lookahead", "own_output"])
-def test_block_search_small_config_full_grid(ahead):
-    """64-wide heads without grouping, symmetric, the full 20 x 10 grid."""
+@pytest.mark.parametrize("ahead,n_out,sym", [(True, 0, True), (False, 0, True), (True, 4, False),
+                                              (False, 4, True)],
+                         ids=["lookahead", "own_output", "lookahead-outliers",
+                              "own_output-outliers"])
+def test_block_search_small_config_full_grid(ahead, n_out, sym):
+    """64-wide heads without grouping, the full 20 x 10 grid; with 4 input
+    channels x20 in every linear, the case that concentrates the screening's
+    fp16 rounding on a few terms."""
     import weight_only_int4_quantize_b200 as w4
-    (gi, bi, ni), (gn, bn, nn), x, xh = _small_blocks(SMALL, 96, seed=300)
+    (gi, bi, ni), (gn, bn, nn), x, xh = _small_blocks(SMALL, 96, seed=300, n_out=n_out,
+                                                      scale=20.0)
     al, sh = synth.alpha_grid(20), synth.shrink_grid(10)
-    choice, losses = w4.awq_block_search(x, gi, gn if ahead else None, al, sh, True, cfg=SMALL)
+    choice, losses = w4.awq_block_search(x, gi, gn if ahead else None, al, sh, sym, cfg=SMALL)
     choice = choice.cpu().numpy()
-    ref = B.search_block(xh, bi, ni, (bn, nn) if ahead else None, al, sh, True, SMALL)
+    ref = B.search_block(xh, bi, ni, (bn, nn) if ahead else None, al, sh, sym, SMALL)
     nxt = (bn, nn) if ahead else None
     one = np.array([1.0], np.float32)
     for gidx, group in enumerate(B.GROUPS):
         a_star, r_star = ref[group]
-        col = B.scoring_losses(xh, bi, ni, nxt, group, al, one, True, SMALL)[:, 0]
+        col = B.scoring_losses(xh, bi, ni, nxt, group, al, one, sym, SMALL)[:, 0]
         rel = np.abs(losses.cpu().numpy()[gidx * 20:(gidx + 1) * 20] - col) / col
         assert rel.max() <= SCREEN_RTOL, (group, float(rel.max()))
         _same_pick(int(choice[gidx]), col, f"{group} alpha*")
@@ -182,6 +187,6 @@ def test_block_search_small_config_full_grid(ahead):
         for name, r in r_star.items():
             li = B.LINEARS.index(name)
             if int(choice[4 + li]) != r:
-                row = B.scoring_losses(xh, bi, ni, nxt, group, al[a_star:a_star + 1], sh, True,
+                row = B.scoring_losses(xh, bi, ni, nxt, group, al[a_star:a_star + 1], sh, sym,
                                        SMALL, only=name)[0]
                 _same_pick(int(choice[4 + li]), row, f"{name} r*")

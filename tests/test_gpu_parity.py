@@ -25,7 +25,10 @@ pytestmark = [pytest.mark.gpu,
 
 DEV = "cuda:0"
 Y_RTOL = 5e-3           # linear: max-normalized error bound
-SSE_RTOL = 2e-4         # AWQ: fp16 tensor-core operands, binary64 sums
+# AWQ: fp16 tensor-core operands, binary64 sums.  Half the library's tie
+# tolerance for tables (5e-4): within it the fp16 values cannot invert the
+# order of two candidates that are not both decided again in binary64.
+SSE_RTOL = 2.5e-4
 GENUINE_TIE_RTOL = 1e-12  # oracle values this close are a tie of the definition itself
 
 
@@ -342,7 +345,8 @@ def test_awq_grid_qwen_k_proj_full_size():
 
 # Per-row errors: each row's sum has only M * K products (no averaging over
 # rows), so the fp16 operand rounding (2^-11 relative on each of x/s and the
-# error operand) can move one row's value by up to ~4 * 2^-11 ~ 2e-3.
+# error operand) can move one row's value by up to ~4 * 2^-11 ~ 2e-3; below
+# half the library's per-row tie tolerance (5e-3).
 ROW_SSE_RTOL = 2e-3
 
 

@@ -409,10 +409,12 @@ constexpr int kLossBlocks = 296;
 // screening losses differ from the binary64 ones by far less (the fp16
 // roundings touch only each linear's change, about 2^-11 of it, and the
 // loss averages them over every token and hidden unit): at most 4.3e-5 on
-// Qwen3-1.7B-shaped blocks at 256 and 2048 tokens, both arms.  Two
-// candidates whose order the screening could invert are then both within
-// the tolerance; the tests hold the difference below half of it.
-constexpr double kBlockTieTol = 3e-4;
+// Qwen3-1.7B-shaped blocks at 256 and 2048 tokens, both arms.  Outlier
+// input channels concentrate the rounding on a few terms (on the fp16 AWQ
+// grid they raised the error about 5x), so half of the tolerance keeps a
+// margin above that too; the tests hold the difference below half of it,
+// with and without outlier channels.
+constexpr double kBlockTieTol = 1e-3;
 
 // Per-block partial sums of (a - b)^2 (grid of kLossBlocks blocks).
 __global__ void __launch_bounds__(256)

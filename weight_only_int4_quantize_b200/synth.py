@@ -135,17 +135,19 @@ def block_input(t: int, hidden: int, seed: int, std: float = 1.0) -> torch.Tenso
     return torch.randn(t, hidden, generator=g, dtype=torch.float64) * std
 
 
-def block_of_shape(cfg: dict, seed: int, std: float = 0.05):
+def block_of_shape(cfg: dict, seed: int, std: float = 0.05, n_outliers: int = 0,
+                   outlier_scale: float = 1.0):
     """A decoder block of any shape (cfg: hidden, heads, kv_heads, head_dim,
     ffn) for the block-level scoring: bf16 linears N(0, std) keyed "q" ..
-    "down" ([out, in]) and float64 gains 1 + 0.1 N(0, 1)."""
+    "down" ([out, in]), each with n_outliers input channels scaled by
+    outlier_scale (normal_weight), and float64 gains 1 + 0.1 N(0, 1)."""
     h, hq, hkv, d, f = cfg["hidden"], cfg["heads"], cfg["kv_heads"], cfg["head_dim"], cfg["ffn"]
     shapes = {"q": (hq * d, h), "k": (hkv * d, h), "v": (hkv * d, h), "o": (h, hq * d),
               "gate": (f, h), "up": (f, h), "down": (h, f)}
     out = {}
     for i, name in enumerate(BLOCK_LINEAR_NAMES):
         n, k = shapes[name]
-        out[name] = normal_weight(n, k, std, seed + i)
+        out[name] = normal_weight(n, k, std, seed + i, n_outliers, outlier_scale)
     g = _gen(seed + 100)
     for name, width in (("ln1", h), ("ln2", h), ("q_norm", d), ("k_norm", d)):
         out[name] = 1.0 + 0.1 * torch.randn(width, generator=g, dtype=torch.float64)
