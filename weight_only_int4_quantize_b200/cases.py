@@ -7,6 +7,7 @@ timing.  Inputs are seeded and generated on the device.
     python -m weight_only_int4_quantize_b200.cases decode_batch --m 1 --blocks 4 [--a8]
     python -m weight_only_int4_quantize_b200.cases clip_rows --m 2048 --n 6144 --k 2048 --nr 10
     python -m weight_only_int4_quantize_b200.cases block --t 512 --na 2 [--group qkv] [--own]
+    python -m weight_only_int4_quantize_b200.cases block --search --t 2048 --na 20 --nr 10
 
 Each case captures --iters launches in one CUDA graph (so host launch
 overhead does not count), replays it once to warm up, times one replay with
@@ -68,6 +69,9 @@ def main():
     ap.add_argument("--group", default="qkv", help="block: linear group scored")
     ap.add_argument("--own", action="store_true",
                     help="block: loss at the block's own output (no look-ahead)")
+    ap.add_argument("--search", action="store_true",
+                    help="block: the screened search (na alphas x nr shrinks) instead of the "
+                         "binary64 losses of one group")
     ap.add_argument("--blocks", type=int, default=4,
                     help="decode_batch: Qwen3-1.7B-shaped blocks (7 linears each) in one batch")
     ap.add_argument("--m", type=int, default=8)
@@ -97,6 +101,14 @@ def main():
         ws = torch.empty(w4.block_workspace_bytes(a.t), dtype=torch.uint8, device="cuda")
         al = synth.alpha_grid(20)[: a.na]
         one = np.array([1.0], np.float32)
+        if a.search:
+            sh = synth.shrink_grid(10)[: a.nr]
+            ms = _time(lambda: w4.awq_block_search(x, gi, gn, al, sh, False, workspace=ws),
+                       a.iters, False)
+            n_c = 4 * a.na + 7 * a.nr
+            print(json.dumps({"case": "block_search", "t": a.t, "candidates": n_c,
+                              "lookahead": not a.own, "ms": ms, "ms_per_candidate": ms / n_c}))
+            return
         ms = _time(lambda: w4.awq_block_scoring_losses(x, gi, gn, a.group, al, one, False,
                                                        workspace=ws), a.iters, False)
         print(json.dumps({"case": "block", "t": a.t, "group": a.group, "candidates": a.na,

@@ -218,11 +218,20 @@ __global__ void __launch_bounds__(256, 2) gemm_f64_kernel(GemmArgs g) {
     __syncthreads();  // step kt's buffer is consumed before step kt + 2 refills it
   }
   double* C = g.C + b * g.bC;
-  const double* R = g.R ? g.R + b * g.bC : nullptr;
+  const double* R = g.R ? g.R + b * g.bC : nullptr;  // never the output itself
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const int m = m0 + 32 * wr + 8 * i + fr;
     if (m >= g.M) continue;
+    // The row's eight residual values are loaded before its stores.
+    double rv[4][2];
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int n = n0 + 32 * wc + 8 * j + 2 * fq + u;
+        rv[j][u] = (R && n < g.N) ? __ldg(R + m * g.sCm + n * g.sCn) : 0.0;
+      }
 #pragma unroll
     for (int j = 0; j < 4; ++j)
 #pragma unroll
@@ -230,7 +239,7 @@ __global__ void __launch_bounds__(256, 2) gemm_f64_kernel(GemmArgs g) {
         const int n = n0 + 32 * wc + 8 * j + 2 * fq + u;
         if (n >= g.N) continue;
         const int64_t o = m * g.sCm + n * g.sCn;
-        C[o] = R ? __dadd_rn(R[o], acc[i][j][u]) : acc[i][j][u];
+        C[o] = R ? __dadd_rn(rv[j][u], acc[i][j][u]) : acc[i][j][u];
       }
   }
 }
@@ -1233,6 +1242,71 @@ cudaError_t screen_candidate(const Screen& z, int group, int ia, float ratio, in
   return cudaGetLastError();
 }
 
+// The binary64 loss of one candidate for a screened selection: the same
+// path as candidate(), reading the group's inputs (and the residuals before
+// the group) from the screening's reference set, which holds the binary64
+// reference values (fwd_ref runs forward_from's kernels in its order), and
+// writing everything from the group on into set A / set B.
+cudaError_t exact_candidate(const Screen& z, int group, int ia, float ratio, int only,
+                            double* loss_out) {
+  const Session& s = *z.s;
+  const BlockConfig& c = *s.c;
+  const cudaStream_t st = s.cx.st;
+  const int K = group_in_width(c, group);
+  float* sv = reinterpret_cast<float*>(s.ws + s.L.s);
+  block_scales_kernel<<<(K + 127) / 128, 128, 0, st>>>(ws_d(s, s.L.stat), K, s.al, ia, nullptr,
+                                                       sv);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  Lin W[7];
+  for (int i = 0; i < 7; ++i) W[i] = s.Wi[i];
+  size_t off = s.L.wc;
+  for (int l = kGroupFirst[group]; l < kGroupFirst[group + 1]; ++l) {
+    int n, k;
+    linear_shape(c, l, &n, &k);
+    double* wc = ws_d(s, off);
+    off += rup(static_cast<size_t>(n) * k * sizeof(double));
+    const float r = (only < 0 || only == l) ? ratio : 1.0f;
+    const int64_t items = static_cast<int64_t>(n) * (k / 128);
+    const unsigned blocks = static_cast<unsigned>((items + 7) / 8);
+    const auto* wb = static_cast<const uint16_t*>(s.Wi[l].p);
+    if (s.sym)
+      candidate_weight_kernel<true><<<blocks, 256, 0, st>>>(wb, n, k, sv, r, wc);
+    else
+      candidate_weight_kernel<false><<<blocks, 256, 0, st>>>(wb, n, k, sv, r, wc);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    W[l] = Lin{wc, true};
+  }
+  // Inputs before the group from the reference set, the rest into set A.
+  const FBufs& R = z.Ri;
+  Bufs b = s.A;
+  b.h = R.h;
+  if (group >= 1) b.a = R.a;
+  if (group >= 2) {
+    b.x1 = R.x1;
+    b.h2 = R.h2;
+  }
+  if (group >= 3) b.act = R.act;
+  double* out_i = ws_d(s, s.L.out_b);
+  e = forward_from(s.cx, group, s.x, W, s.ni, b, out_i);
+  if (e != cudaSuccess) return e;
+  const double* fin = out_i;
+  const double* ref = R.out;
+  if (s.ahead) {
+    double* out_n = ws_d(s, s.L.out_a);
+    e = forward_full(s.cx, out_i, s.Wn, s.nn, s.B, out_n);
+    if (e != cudaSuccess) return e;
+    fin = out_n;
+    ref = z.Rn.out;
+  }
+  const int64_t n = static_cast<int64_t>(s.cx.T) * c.hidden;
+  double* part = ws_d(s, s.L.partial);
+  sqdiff_partial_kernel<<<kLossBlocks, 256, 0, st>>>(fin, ref, n, part);
+  loss_finish_kernel<<<1, 32, 0, st>>>(part, n, loss_out);
+  return cudaGetLastError();
+}
+
 __global__ void set_int_kernel(int32_t* p, int v) {
   if (threadIdx.x == 0) *p = v;
 }
@@ -1262,15 +1336,13 @@ cudaError_t screened_select(const Screen& z, int group, int n, int only, CandFn 
     members += near[i];
   }
   if (members >= 2) {
-    // Binary64 losses of the near set (the exact path recomputes its own
-    // reference into its buffers).
-    W4_TRY(reference(s, group));
+    // Binary64 losses of the near set.
     for (int i = 0; i < n; ++i)
       if (near[i]) {
         int ia;
         float r;
         cand(i, &ia, &r);
-        W4_TRY(candidate(s, group, ia, nullptr, r, only, losses + i));
+        W4_TRY(exact_candidate(z, group, ia, r, only, losses + i));
       }
     W4_TRY(cudaMemcpyAsync(host, losses, sizeof(double) * n, cudaMemcpyDeviceToHost, s.cx.st));
     W4_TRY(cudaStreamSynchronize(s.cx.st));

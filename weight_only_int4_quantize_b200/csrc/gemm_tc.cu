@@ -477,29 +477,71 @@ __global__ void __launch_bounds__(kThreads, 1)
       } else if (EPI == kEpiAddF64) {
         // out = r1 (+ r2) + 2^-(ea + eb) acc in binary64: the operands were
         // scaled by exact powers of two, which the epilogue removes exactly.
+        // Each warp stages its 32 rows x NB/2 columns of fp32 accumulators
+        // in the (now idle) stage buffers, rows 132 floats apart, then walks
+        // the rows with all 32 lanes on one row, so that r1, r2 and the
+        // output move as contiguous runs of the row (4 columns a lane).
+        static_assert(EPI != kEpiAddF64 || NB == 256, "binary64 epilogue uses 256-column tiles");
+        constexpr int kLd = 132;
+        float* stg = reinterpret_cast<float*>(base_ptr + SL::a) + (warp - 2) * (32 * kLd);
         const double scale = ldexp(1.0, -(*ss.ea + *ss.eb));
-        for (int mt = 0; mt < MT; ++mt)
+        const double* r1p = ss.r1;
+        const double* r2p = ss.r2;
+        double* outp = ss.out;
+        for (int mt = 0; mt < MT; ++mt) {
           for (int c = 0; c < NB / 32; ++c) {
-            const int m = m0 + 128 * mt + 32 * q + lane;
-            const int col = (NB / 2) * ch + 16 * c;
             uint32_t r[16];
-            tmem_ld_32x32b_x16(tmem_base + (static_cast<uint32_t>(32 * q) << 16) + NB * mt + col,
-                               r);
+            tmem_ld_32x32b_x16(
+                tmem_base + (static_cast<uint32_t>(32 * q) << 16) + NB * mt + 128 * ch + 16 * c, r);
             tmem_ld_wait();
-            const int n = n0 + col;
-            if (m < M) {
-              const size_t o = static_cast<size_t>(m) * ss.ldc + n;
+            float4* d4 = reinterpret_cast<float4*>(stg + lane * kLd + 16 * c);
 #pragma unroll
-              for (int i = 0; i < 16; ++i) {
-                if (n + i < N) {
-                  double v = ss.r1[o + i];
-                  if (ss.r2) v = __dadd_rn(v, ss.r2[o + i]);
-                  ss.out[o + i] =
-                      __dadd_rn(v, __dmul_rn(scale, static_cast<double>(__uint_as_float(r[i]))));
-                }
+            for (int i = 0; i < 4; ++i)
+              d4[i] = make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
+                                  __uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3]));
+          }
+          __syncwarp();
+          const int n = n0 + 128 * ch + 4 * lane;  // this lane's 4 columns
+          const bool whole = n + 4 <= N && (ss.ldc & 1) == 0;
+          for (int rr = 0; rr < 32; ++rr) {
+            const int m = m0 + 128 * mt + 32 * q + rr;
+            if (m >= M) break;
+            const float4 a = *reinterpret_cast<const float4*>(stg + rr * kLd + 4 * lane);
+            const float av[4] = {a.x, a.y, a.z, a.w};
+            const size_t o = static_cast<size_t>(m) * ss.ldc + n;
+            double v[4], w[4] = {0.0, 0.0, 0.0, 0.0};
+            if (whole) {
+              const double2 p0 = __ldg(reinterpret_cast<const double2*>(r1p + o));
+              const double2 p1 = __ldg(reinterpret_cast<const double2*>(r1p + o) + 1);
+              v[0] = p0.x; v[1] = p0.y; v[2] = p1.x; v[3] = p1.y;
+              if (r2p) {
+                const double2 q0 = __ldg(reinterpret_cast<const double2*>(r2p + o));
+                const double2 q1 = __ldg(reinterpret_cast<const double2*>(r2p + o) + 1);
+                w[0] = q0.x; w[1] = q0.y; w[2] = q1.x; w[3] = q1.y;
+              }
+            } else {
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                v[i] = n + i < N ? r1p[o + i] : 0.0;
+                if (r2p && n + i < N) w[i] = r2p[o + i];
               }
             }
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const double base = r2p ? __dadd_rn(v[i], w[i]) : v[i];
+              v[i] = __dadd_rn(base, __dmul_rn(scale, static_cast<double>(av[i])));
+            }
+            if (whole) {
+              reinterpret_cast<double2*>(outp + o)[0] = make_double2(v[0], v[1]);
+              reinterpret_cast<double2*>(outp + o)[1] = make_double2(v[2], v[3]);
+            } else {
+#pragma unroll
+              for (int i = 0; i < 4; ++i)
+                if (n + i < N) outp[o + i] = v[i];
+            }
           }
+          __syncwarp();  // the staging rows are rewritten for the next 128-row half
+        }
       } else if (EPI == kEpiColSumSquares) {
         // Column sums of y^2 over the tile's rows: per 16-column chunk each
         // thread squares its row's 16 values (its row of each 128-row half
@@ -906,7 +948,13 @@ cudaError_t launch_add_gemm_f16(const void* a_f16, int M, const void* b_f16, int
   CUtensorMap ta, tb;
   const uint64_t da[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(M)};
   const uint64_t sa[1] = {static_cast<uint64_t>(K) * 2};
-  const int mt = sumsq_mt(M);
+  // 256-row tiles share each B tile between two UMMAs, but only when their
+  // count still covers the SMs; otherwise 128-row tiles double the CTAs.
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const long tiles2 = static_cast<long>((N + BN - 1) / BN) * ((M + 2 * BM - 1) / (2 * BM));
+  const int mt = (M >= 2 * BM && tiles2 >= sms) ? 2 : 1;
   const uint32_t ba[2] = {BK, static_cast<uint32_t>(mt * BM)};
   if (encode_tmap(&ta, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, da, sa, ba, a_f16) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
