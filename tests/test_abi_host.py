@@ -276,3 +276,20 @@ def test_block_validation(L):
     assert search(choice=B + 4) == 3
     assert search(losses=B + 8) == 3
     assert search(wsb=16) == 5
+
+
+def test_bench_traffic_captures_match_sources():
+    """bench.py reports a kernel's DRAM traffic from an ncu capture only while
+    the kernel's source is the one captured (its digest); a kernel changed
+    without a new capture would report null."""
+    import importlib.util
+    spec = importlib.util.spec_from_file_location("bench", os.path.join(ROOT, "bench.py"))
+    bench = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(bench)
+    for kernel, cap in bench.TRAFFIC_CAPTURES.items():
+        assert bench.source_digest(cap["source"]) == cap["digest"], (
+            f"{kernel}: {cap['source']} changed since its traffic capture")
+        assert 0.3 < cap["ratio"] < 1.5, kernel
+    e = bench.roofline_entry("gemv_w4a16", "hbm", 4000.0, 6535.7, "GB/s", "measured", 1e9, 0.5)
+    assert e["frac"] == 4000.0 / 6535.7 and e["traffic"] == bench.TRAFFIC_CAPTURES[
+        "gemv_w4a16"]["ratio"] * 1e9
