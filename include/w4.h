@@ -412,7 +412,8 @@ w4_status awq_clip_search_rows(const void* x_bf16, int64_t M, const void* w_bf16
                                size_t workspace_bytes, void* stream);
 
 /*
- * Block-level candidate scoring (binary64).
+ * Block-level candidate scoring (binary64 losses; the search screened on
+ * tcgen05 tensor cores with binary64 decisions).
  *
  * [rebuttal] 'Model Details' table, row 'Search', and the paragraph under
  * it: a candidate (alpha, shrink) for a linear group of decoder block i is
@@ -432,8 +433,9 @@ w4_status awq_clip_search_rows(const void* x_bf16, int64_t M, const void* w_bf16
  * attention scaled by 1/sqrt(head_dim), query head h reading key/value head
  * h / (heads / kv_heads), SwiGLU MLP (silu(gate) * up), residual adds.
  *
- * Every step runs in binary64 (the contractions on the fp64 MMA); results
- * depend on nothing but the inputs (fixed order of every sum).
+ * awq_block_scoring_losses runs every step in binary64 (the contractions on
+ * the fp64 MMA); its results depend on nothing but the inputs (fixed order
+ * of every sum).  awq_block_search screens first (see there).
  *
  * Linears are numbered q 0, k 1, v 2, o 3, gate 4, up 5, down 6; groups are
  * qkv 0 (q, k, v), o 1, gate_up 2 (gate, up), down 3.
