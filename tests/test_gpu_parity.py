@@ -217,6 +217,14 @@ def test_prefill_split_k(m, n, k, sym):
     assert linear_case(m, n, k, sym, seed=160 + m + n) <= Y_RTOL
 
 
+@pytest.mark.parametrize("m,n,k", [(96, 8448, 4096), (1024, 5120, 17408)])
+def test_prefill_split_k_four_way(m, n, k):
+    """Four-way K splits of 128 x 256 and of 256 x 128 tiles, which the
+    launch's time model picks for these shapes on B200."""
+    rows = None if m <= 128 else np.sort(np.random.default_rng(m + n).choice(m, 128, replace=False))
+    assert linear_case(m, n, k, False, seed=170 + m, rows=rows) <= Y_RTOL
+
+
 def test_prefill_split_k_deterministic():
     w = synth.normal_weight(384, 8192, 0.02, seed=171)
     x = synth.normal_activations(48, 8192, seed=172).to(DEV)

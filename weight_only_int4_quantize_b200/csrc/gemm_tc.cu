@@ -745,12 +745,10 @@ CUresult encode_tmap(CUtensorMap* map, CUtensorMapDataType dt, int rank, const u
 // The scoring GEMMs carry no group.
 const GemmGroup kNoGroup = {};
 
+// The opt-in shared-memory size is a per-device function attribute; set it
+// once per device and kernel instantiation.
 template <auto kern, size_t kSmemBytes>
-cudaError_t launch_gemm(dim3 grid, bool pdl, cudaStream_t stream, const CUtensorMap& ta,
-                        const CUtensorMap& tb, const GemmGroup& grp, const SumSqArgs& ss, int M,
-                        int N, int K, int pdl_static, unsigned* err, int cluster = 1) {
-  // The opt-in shared-memory size is a per-device function attribute; set it
-  // once per device and kernel instantiation.
+cudaError_t set_smem_attr() {
   static unsigned long long attr_done = 0;  // bit d: device d
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -761,6 +759,56 @@ cudaError_t launch_gemm(dim3 grid, bool pdl, cudaStream_t stream, const CUtensor
     if (e != cudaSuccess) return e;
     if (dev < 64) __atomic_fetch_or(&attr_done, 1ull << dev, __ATOMIC_RELEASE);
   }
+  return cudaSuccess;
+}
+
+// CTAs of the kernel that run at once when launched in clusters of ks
+// (1 <= ks <= 4): clusters must fit inside one GPC, so for ks > 1 this can be
+// fewer than the SM count.  Queried from the runtime once per device and
+// cluster size; while `stream` is being captured into a graph nothing is
+// queried, and an unknown value is estimated as whole clusters over the SMs.
+template <auto kern, size_t kSmemBytes>
+int resident_ctas(int ks, int sms, cudaStream_t stream) {
+  if (ks <= 1) return sms;  // one CTA per SM (shared memory)
+  static int cache[64][5];  // 0: not known yet
+  int dev = 0;
+  const int guess = (sms / ks) * ks;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev >= 64 || ks > 4) return guess;
+  const int known = __atomic_load_n(&cache[dev][ks], __ATOMIC_ACQUIRE);
+  if (known > 0) return known;
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(stream, &cap) != cudaSuccess || cap != cudaStreamCaptureStatusNone)
+    return guess;
+  if (set_smem_attr<kern, kSmemBytes>() != cudaSuccess) return guess;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(ks, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cudaLaunchAttribute attr;
+  attr.id = cudaLaunchAttributeClusterDimension;
+  attr.val.clusterDim.x = ks;
+  attr.val.clusterDim.y = 1;
+  attr.val.clusterDim.z = 1;
+  cfg.attrs = &attr;
+  cfg.numAttrs = 1;
+  int clusters = 0;
+  if (cudaOccupancyMaxActiveClusters(&clusters, reinterpret_cast<const void*>(kern), &cfg) !=
+          cudaSuccess ||
+      clusters <= 0) {
+    (void)cudaGetLastError();  // not sticky: clear it, keep the estimate
+    return guess;
+  }
+  const int n = clusters * ks < sms ? clusters * ks : sms;
+  __atomic_store_n(&cache[dev][ks], n, __ATOMIC_RELEASE);
+  return n;
+}
+
+template <auto kern, size_t kSmemBytes>
+cudaError_t launch_gemm(dim3 grid, bool pdl, cudaStream_t stream, const CUtensorMap& ta,
+                        const CUtensorMap& tb, const GemmGroup& grp, const SumSqArgs& ss, int M,
+                        int N, int K, int pdl_static, unsigned* err, int cluster = 1) {
+  cudaError_t e = set_smem_attr<kern, kSmemBytes>();
+  if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = dim3(kThreads, 1, 1);
@@ -806,31 +854,41 @@ cudaError_t launch_prefill_gemm_group(const PrefillItem* items_in, int count, in
         items[j - 1] = t;
       }
     const bool sym = items[0].z == nullptr;
-    // Tile shape (MT x 128 rows, NB columns), one CTA per SM.  Measured time
-    // of one wave of CTAs relative to 128 x 256 tiles (same K): 256 x 256
-    // 1.32, 128 x 256 1.00, 256 x 128 0.80, 128 x 128 0.68 -- the B
-    // dequantization scales with NB and the MMAs with MT x NB.  The group's
-    // tiles count in units of its longest K; the shape with the smallest
-    // waves x wave time wins, on equal cost the earlier (larger) one.
-    //
-    // A group whose best unsplit launch fills less than half the SMs also
-    // considers splitting K over a cluster of ks CTAs (ks <= 4, at least 2
-    // k-blocks each, the fp32 partial tile fitting the stage buffers): ks x
-    // the CTAs, each 1/ks of the K loop, plus about 15 % for writing and
-    // adding the partials through distributed shared memory.
-    struct Shape { int mt, nb, cost; size_t stage_bytes; };
+    // Tile shape (MT x 128 rows by NB columns, one CTA per SM) and K split
+    // (clusters of ks <= 4 CTAs, each running 1/ks of the k-blocks, the fp32
+    // partial tiles added through distributed shared memory) from a time
+    // model fitted to B200 measurements of single and grouped launches
+    // (27B- and Llama-2-7B-shaped linears, M = 16 ... 4096; rms error 6 %):
+    //   waves x (a + b x k-blocks per CTA + (ks > 1 ? c : 0)) microseconds,
+    //   waves = ceil(tiles x ks / CTAs resident at once),
+    // the group's tiles counted in units of its longest K.  Per k-block the
+    // B dequantization of NB columns dominates (two 128-row UMMAs share one
+    // dequantized tile at about the cost of one); c is the partial-tile
+    // exchange.  A split needs at least 2 k-blocks per CTA and the partial
+    // tile must fit the stage buffers.
+    struct Shape { int mt, nb; double a, b, c; size_t stage_bytes; };
     const Shape shapes[4] = {
-        {2, 256, 132, SmemLayout<2, 256>::kStages * size_t(Tile<2, 256>::kTileABytes + Tile<2, 256>::kTileBBytes)},
-        {1, 256, 100, SmemLayout<1, 256>::kStages * size_t(Tile<1, 256>::kTileABytes + Tile<1, 256>::kTileBBytes)},
-        {2, 128, 80, SmemLayout<2, 128>::kStages * size_t(Tile<2, 128>::kTileABytes + Tile<2, 128>::kTileBBytes)},
-        {1, 128, 68, SmemLayout<1, 128>::kStages * size_t(Tile<1, 128>::kTileABytes + Tile<1, 128>::kTileBBytes)}};
+        {2, 256, 8.9, 0.923, 0.2, SmemLayout<2, 256>::kStages * size_t(Tile<2, 256>::kTileABytes + Tile<2, 256>::kTileBBytes)},
+        {1, 256, 2.5, 0.779, 4.5, SmemLayout<1, 256>::kStages * size_t(Tile<1, 256>::kTileABytes + Tile<1, 256>::kTileBBytes)},
+        {2, 128, 7.9, 0.495, 0.9, SmemLayout<2, 128>::kStages * size_t(Tile<2, 128>::kTileABytes + Tile<2, 128>::kTileBBytes)},
+        {1, 128, 4.7, 0.482, 1.7, SmemLayout<1, 128>::kStages * size_t(Tile<1, 128>::kTileABytes + Tile<1, 128>::kTileBBytes)}};
+    auto resident = [&](int si, int ks) {
+      switch (si) {
+        case 0: return resident_ctas<gemm_tc_kernel<kBDequant, kEpiStoreBf16, true, 2, 256>,
+                                     SmemLayout<2, 256>::bytes>(ks, sms, stream);
+        case 1: return resident_ctas<gemm_tc_kernel<kBDequant, kEpiStoreBf16, true, 1, 256>,
+                                     SmemLayout<1, 256>::bytes>(ks, sms, stream);
+        case 2: return resident_ctas<gemm_tc_kernel<kBDequant, kEpiStoreBf16, true, 2, 128>,
+                                     SmemLayout<2, 128>::bytes>(ks, sms, stream);
+        default: return resident_ctas<gemm_tc_kernel<kBDequant, kEpiStoreBf16, true, 1, 128>,
+                                      SmemLayout<1, 128>::bytes>(ks, sms, stream);
+      }
+    };
     const int k_max = items[0].K;
     int kb_min = 1 << 30;
     for (int i = 0; i < n; ++i) kb_min = items[i].K / BK < kb_min ? items[i].K / BK : kb_min;
     int best = -1, best_ks = 1;
     double best_cost = 0.0;
-    bool allow_split = false;
-    for (int pass = 0; pass < 2; ++pass) {
     for (int si = 0; si < 4; ++si) {
       const Shape sh = shapes[si];
       if (sh.mt == 2 && M < 2 * BM) continue;  // 256-row tiles only when rows fill them
@@ -839,17 +897,17 @@ cudaError_t launch_prefill_gemm_group(const PrefillItem* items_in, int count, in
         eq += static_cast<double>((items[i].N + sh.nb - 1) / sh.nb) *
               ((M + sh.mt * BM - 1) / (sh.mt * BM)) * items[i].K / k_max;
       const size_t part_bytes = static_cast<size_t>(sh.mt) * BM * (sh.nb + 4) * 4;
-      for (int ks = pass == 0 ? 1 : 2; ks <= (pass == 0 ? 1 : 4); ++ks) {
-        if (ks > 1 && (!allow_split || part_bytes > sh.stage_bytes || kb_min < 2 * ks)) break;
-        const double cost = std::ceil(eq * ks / sms - 1e-9) * sh.cost / ks * (ks > 1 ? 1.15 : 1.0);
+      for (int ks = 1; ks <= 4; ++ks) {
+        if (ks > 1 && (part_bytes > sh.stage_bytes || kb_min < 2 * ks)) break;
+        const double waves = std::ceil(eq * ks / resident(si, ks) - 1e-9);
+        const double cost =
+            waves * (sh.a + sh.b * (static_cast<double>(k_max) / BK) / ks + (ks > 1 ? sh.c : 0.0));
         if (best < 0 || cost < best_cost - 1e-9) {
           best = si;
           best_ks = ks;
           best_cost = cost;
-          if (pass == 0) allow_split = eq * 2 < sms;
         }
       }
-    }
     }
     if (best < 0) best = 1;
     const int mt = shapes[best].mt, nb = shapes[best].nb;
