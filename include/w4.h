@@ -162,9 +162,14 @@ w4_status w4_quantize_pack_batched(const w4_quant_item* items, int count, int gr
  * launches with at least two of its 4-warp bundles per SM, and a per-CTA
  * tensor-map kernel (K split over a thread-block cluster) for smaller
  * launches and 9 <= M <= 64.  W4_LINEAR_DECODE_STREAM / _TILED override the
- * choice; both meet the same error bound.  A prefill launch with few tiles
- * splits K over a thread-block cluster of up to 4 CTAs and adds the fp32
- * partial tiles through distributed shared memory in rank order.
+ * choice; both meet the same error bound.  A prefill launch picks its tile
+ * shape (128 or 256 rows x 128 or 256 columns) and a split of K over a
+ * thread-block cluster of up to 4 CTAs from a time model measured on B200 and
+ * the number of CTAs the device runs at once in clusters of each size (asked
+ * of the runtime once per device; a launch captured into a graph before any
+ * uncaptured one on its device estimates it).  The fp32 partial tiles are
+ * added through distributed shared memory in rank order, so a given launch
+ * configuration always gives the same bits.
  */
 #define W4_LINEAR_FORCE_GEMV 0x1u  /* decode kernel at any M <= 64 (K <= 81920) */
 #define W4_LINEAR_FORCE_GEMM 0x2u  /* prefill kernel at any M */
