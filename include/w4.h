@@ -217,6 +217,30 @@ w4_status w4a16_linear_batched(const w4_linear_item* items, int count, int64_t M
                                unsigned flags, void* stream);
 
 /*
+ * w4_prefill_plan -- the tile shape and K split that a prefill launch uses
+ * (w4a16_linear above 32 rows, or one launch of w4a16_linear_batched) for
+ * `count` linears of N[i] x K[i] weights that share the token count M.  For
+ * inspection and tuning: it computes the launch's own choice (the time model
+ * described at w4a16_linear) and launches nothing.
+ *
+ * N, K       host int64 [count]; N >= 1, K a positive multiple of 128.
+ * count      1 .. 16 (a launch takes at most 16 linears).
+ * M          >= 1.
+ * resident   NULL: the current device's counts (asks the runtime); else host
+ *            int [16]: for the tile shapes 256 x 256, 128 x 256, 256 x 128 and
+ *            128 x 128 (rows x columns) in that order, the CTAs that run at
+ *            once in clusters of 1, 2, 3 and 4 CTAs (each >= 1).  With
+ *            resident given no device is used.
+ * tile_rows, tile_cols, k_split  host int out: the CTA tile and the number
+ *            of CTAs that split K in a cluster (1: no split).
+ * Returns W4_ERR_INVALID_ARG (NULL pointer, count out of range, a resident
+ * count < 1) or W4_ERR_SHAPE; with resident NULL, W4_ERR_CUDA without a
+ * usable device.
+ */
+w4_status w4_prefill_plan(const int64_t* N, const int64_t* K, int count, int64_t M,
+                          const int* resident, int* tile_rows, int* tile_cols, int* k_split);
+
+/*
  * W4A8 decode -- the same stored int4 weights against int8 activations
  * ([qsrt] 'What is included': W4A8 decode execution; the storage paragraph:
  * W4A8 and W4A16 use the same stored weights; the runtime paragraph: W4A8

@@ -18,7 +18,7 @@ __all__ = [
     "W4Error", "lib", "quantize_pack", "quantize_pack_batched", "quantize_pack_rows",
     "awq_clip_search_rows", "clip_rows_workspace_bytes", "w4a16_linear",
     "quantize_act_int8", "w4a8_linear", "w4a8_linear_batched", "a8_items",
-    "w4a16_linear_batched", "awq_scales", "awq_score_grid", "awq_score_grid_static_scratch",
+    "w4a16_linear_batched", "prefill_plan", "awq_scales", "awq_score_grid", "awq_score_grid_static_scratch",
     "awq_workspace_bytes", "device_error", "selftest_bounded_wait",
     "LINEAR_FORCE_GEMV", "LINEAR_FORCE_GEMM", "LINEAR_PDL", "LINEAR_STATIC_WEIGHTS",
     "LINEAR_DECODE_STREAM", "LINEAR_DECODE_TILED", "STREAM_BATCH",
@@ -76,6 +76,8 @@ def _declare(L: ctypes.CDLL) -> None:
     L.w4_quantize_pack_batched.argtypes = [_p, ctypes.c_int, ctypes.c_int, ctypes.c_int, _p]
     L.w4a16_linear_batched.restype = ctypes.c_int
     L.w4a16_linear_batched.argtypes = [_p, ctypes.c_int, _i64, ctypes.c_int, ctypes.c_uint, _p]
+    L.w4_prefill_plan.restype = ctypes.c_int
+    L.w4_prefill_plan.argtypes = [_p, _p, ctypes.c_int, _i64, _p, _p, _p, _p]
     L.w4_awq_scales.restype = ctypes.c_int
     L.w4_awq_scales.argtypes = [_p, _i64, _i64, _p, ctypes.c_int, _p, _p]
     L.w4_awq_workspace_bytes.restype = ctypes.c_size_t
@@ -307,6 +309,26 @@ def linear_items(items, m=None):
         a.zeros_f16 = None if zr is None else zr.data_ptr()
         a.N, a.K, a.y_bf16 = qw.shape[0], x.shape[1], y.data_ptr()
     return arr
+
+
+def prefill_plan(shapes, m: int, resident=None):
+    """(tile_rows, tile_cols, k_split) of the prefill launch for linears of
+    shapes [(N, K), ...] (at most 16) sharing m rows.  resident: None (the
+    current device's counts) or 4 x 4 ints, the CTAs run at once per tile
+    shape (256x256, 128x256, 256x128, 128x128) and cluster size 1..4."""
+    n = len(shapes)
+    na = (ctypes.c_int64 * max(n, 1))(*[int(s[0]) for s in shapes])
+    ka = (ctypes.c_int64 * max(n, 1))(*[int(s[1]) for s in shapes])
+    res = None
+    if resident is not None:
+        flat = [int(v) for row in resident for v in row]
+        if len(flat) != 16:
+            raise ValueError("resident must be 4 x 4")
+        res = (ctypes.c_int * 16)(*flat)
+    rows, cols, ks = ctypes.c_int(), ctypes.c_int(), ctypes.c_int()
+    _check(lib().w4_prefill_plan(na, ka, n, int(m), res, ctypes.byref(rows), ctypes.byref(cols),
+                                 ctypes.byref(ks)), "w4_prefill_plan")
+    return rows.value, cols.value, ks.value
 
 
 def w4a16_linear_batched(items, m: int, flags: int = 0, group: int = 128, stream=None) -> None:

@@ -431,6 +431,37 @@ static w4_status decode_tiled(const w4_linear_item* items, const int* idx, int n
   return W4_OK;
 }
 
+w4_status w4_prefill_plan(const int64_t* N, const int64_t* K, int count, int64_t M,
+                          const int* resident, int* tile_rows, int* tile_cols, int* k_split) {
+  if (!N || !K || !tile_rows || !tile_cols || !k_split) return W4_ERR_INVALID_ARG;
+  if (count < 1 || count > 16) return W4_ERR_INVALID_ARG;
+  if (M < 1 || M > 0x7FFFFFFF) return W4_ERR_SHAPE;
+  int n32[16], k32[16];
+  for (int i = 0; i < count; ++i) {
+    if (N[i] < 1 || N[i] > 0x7FFFFFFF || !valid_k(K[i])) return W4_ERR_SHAPE;
+    n32[i] = static_cast<int>(N[i]);
+    k32[i] = static_cast<int>(K[i]);
+  }
+  int res[kPrefillShapes][kPrefillMaxSplit];
+  if (resident) {
+    for (int s = 0; s < kPrefillShapes; ++s)
+      for (int c = 0; c < kPrefillMaxSplit; ++c) {
+        res[s][c] = resident[s * kPrefillMaxSplit + c];
+        if (res[s][c] < 1) return W4_ERR_INVALID_ARG;
+      }
+  } else {
+    int sms = 0;
+    w4_status st = device_info(&sms, nullptr);
+    if (st != W4_OK) return st;
+    prefill_resident(sms, nullptr, res);
+  }
+  const PrefillPlan p = plan_prefill_group(n32, k32, count, static_cast<int>(M), res);
+  *tile_rows = p.rows;
+  *tile_cols = p.cols;
+  *k_split = p.ks;
+  return W4_OK;
+}
+
 w4_status w4a16_linear_batched(const w4_linear_item* items, int count, int64_t M, int group,
                                unsigned flags, void* stream) {
   if (!items || count < 1) return W4_ERR_INVALID_ARG;

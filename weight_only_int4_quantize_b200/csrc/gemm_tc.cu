@@ -835,6 +835,73 @@ cudaError_t launch_gemm(dim3 grid, bool pdl, cudaStream_t stream, const CUtensor
 
 }  // namespace
 
+void prefill_resident(int sms, cudaStream_t stream,
+                      int (&resident)[kPrefillShapes][kPrefillMaxSplit]) {
+  for (int ks = 1; ks <= kPrefillMaxSplit; ++ks) {
+    int* r = &resident[0][ks - 1];
+    r[0 * kPrefillMaxSplit] = resident_ctas<gemm_tc_kernel<kBDequant, kEpiStoreBf16, true, 2, 256>,
+                                            SmemLayout<2, 256>::bytes>(ks, sms, stream);
+    r[1 * kPrefillMaxSplit] = resident_ctas<gemm_tc_kernel<kBDequant, kEpiStoreBf16, true, 1, 256>,
+                                            SmemLayout<1, 256>::bytes>(ks, sms, stream);
+    r[2 * kPrefillMaxSplit] = resident_ctas<gemm_tc_kernel<kBDequant, kEpiStoreBf16, true, 2, 128>,
+                                            SmemLayout<2, 128>::bytes>(ks, sms, stream);
+    r[3 * kPrefillMaxSplit] = resident_ctas<gemm_tc_kernel<kBDequant, kEpiStoreBf16, true, 1, 128>,
+                                            SmemLayout<1, 128>::bytes>(ks, sms, stream);
+  }
+}
+
+// Tile shape (MT x 128 rows by NB columns, one CTA per SM) and K split
+// (clusters of ks <= 4 CTAs, each running 1/ks of the k-blocks, the fp32
+// partial tiles added through distributed shared memory) from a time model
+// fitted to B200 measurements of single and grouped launches (27B- and
+// Llama-2-7B-shaped linears, M = 16 ... 4096; rms error 6 %):
+//   waves x (a + b x k-blocks per CTA + (ks > 1 ? c : 0)) microseconds,
+//   waves = ceil(tiles x ks / CTAs resident at once),
+// the group's tiles counted in units of its longest K.  Per k-block the B
+// dequantization of NB columns dominates (two 128-row UMMAs share one
+// dequantized tile at about the cost of one); c is the partial-tile
+// exchange.  A split needs at least 2 k-blocks per CTA and the partial tile
+// must fit the stage buffers.  On equal modelled time the earlier shape and
+// the smaller split win.
+PrefillPlan plan_prefill_group(const int* N, const int* K, int n, int M,
+                               const int (&resident)[kPrefillShapes][kPrefillMaxSplit]) {
+  struct Shape { int mt, nb; double a, b, c; size_t stage_bytes; };
+  const Shape shapes[kPrefillShapes] = {
+      {2, 256, 8.9, 0.923, 0.2, SmemLayout<2, 256>::kStages * size_t(Tile<2, 256>::kTileABytes + Tile<2, 256>::kTileBBytes)},
+      {1, 256, 2.5, 0.779, 4.5, SmemLayout<1, 256>::kStages * size_t(Tile<1, 256>::kTileABytes + Tile<1, 256>::kTileBBytes)},
+      {2, 128, 7.9, 0.495, 0.9, SmemLayout<2, 128>::kStages * size_t(Tile<2, 128>::kTileABytes + Tile<2, 128>::kTileBBytes)},
+      {1, 128, 4.7, 0.482, 1.7, SmemLayout<1, 128>::kStages * size_t(Tile<1, 128>::kTileABytes + Tile<1, 128>::kTileBBytes)}};
+  int k_max = 0, kb_min = 1 << 30;
+  for (int i = 0; i < n; ++i) {
+    k_max = K[i] > k_max ? K[i] : k_max;
+    kb_min = K[i] / BK < kb_min ? K[i] / BK : kb_min;
+  }
+  int best = 1, best_ks = 1;
+  double best_cost = -1.0;
+  for (int si = 0; si < kPrefillShapes; ++si) {
+    const Shape sh = shapes[si];
+    if (sh.mt == 2 && M < 2 * BM) continue;  // 256-row tiles only when rows fill them
+    double eq = 0.0;  // tiles of the longest K
+    for (int i = 0; i < n; ++i)
+      eq += static_cast<double>((N[i] + sh.nb - 1) / sh.nb) *
+            ((M + sh.mt * BM - 1) / (sh.mt * BM)) * K[i] / k_max;
+    const size_t part_bytes = static_cast<size_t>(sh.mt) * BM * (sh.nb + 4) * 4;
+    for (int ks = 1; ks <= kPrefillMaxSplit; ++ks) {
+      if (ks > 1 && (part_bytes > sh.stage_bytes || kb_min < 2 * ks)) break;
+      const int res = resident[si][ks - 1] > 0 ? resident[si][ks - 1] : 1;
+      const double waves = std::ceil(eq * ks / res - 1e-9);
+      const double cost =
+          waves * (sh.a + sh.b * (static_cast<double>(k_max) / BK) / ks + (ks > 1 ? sh.c : 0.0));
+      if (best_cost < 0.0 || cost < best_cost - 1e-9) {
+        best = si;
+        best_ks = ks;
+        best_cost = cost;
+      }
+    }
+  }
+  return PrefillPlan{shapes[best].mt * BM, shapes[best].nb, best_ks};
+}
+
 cudaError_t launch_prefill_gemm_group(const PrefillItem* items_in, int count, int M,
                                       bool pdl, bool static_w, cudaStream_t stream,
                                       unsigned* err) {
@@ -842,6 +909,8 @@ cudaError_t launch_prefill_gemm_group(const PrefillItem* items_in, int count, in
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess)
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  int resident[kPrefillShapes][kPrefillMaxSplit];
+  prefill_resident(sms, stream, resident);
   // Longest K first: the long CTAs start first and the short ones fill in.
   PrefillItem items[kGemmGroup];
   for (int i0 = 0; i0 < count; i0 += kGemmGroup) {
@@ -854,64 +923,14 @@ cudaError_t launch_prefill_gemm_group(const PrefillItem* items_in, int count, in
         items[j - 1] = t;
       }
     const bool sym = items[0].z == nullptr;
-    // Tile shape (MT x 128 rows by NB columns, one CTA per SM) and K split
-    // (clusters of ks <= 4 CTAs, each running 1/ks of the k-blocks, the fp32
-    // partial tiles added through distributed shared memory) from a time
-    // model fitted to B200 measurements of single and grouped launches
-    // (27B- and Llama-2-7B-shaped linears, M = 16 ... 4096; rms error 6 %):
-    //   waves x (a + b x k-blocks per CTA + (ks > 1 ? c : 0)) microseconds,
-    //   waves = ceil(tiles x ks / CTAs resident at once),
-    // the group's tiles counted in units of its longest K.  Per k-block the
-    // B dequantization of NB columns dominates (two 128-row UMMAs share one
-    // dequantized tile at about the cost of one); c is the partial-tile
-    // exchange.  A split needs at least 2 k-blocks per CTA and the partial
-    // tile must fit the stage buffers.
-    struct Shape { int mt, nb; double a, b, c; size_t stage_bytes; };
-    const Shape shapes[4] = {
-        {2, 256, 8.9, 0.923, 0.2, SmemLayout<2, 256>::kStages * size_t(Tile<2, 256>::kTileABytes + Tile<2, 256>::kTileBBytes)},
-        {1, 256, 2.5, 0.779, 4.5, SmemLayout<1, 256>::kStages * size_t(Tile<1, 256>::kTileABytes + Tile<1, 256>::kTileBBytes)},
-        {2, 128, 7.9, 0.495, 0.9, SmemLayout<2, 128>::kStages * size_t(Tile<2, 128>::kTileABytes + Tile<2, 128>::kTileBBytes)},
-        {1, 128, 4.7, 0.482, 1.7, SmemLayout<1, 128>::kStages * size_t(Tile<1, 128>::kTileABytes + Tile<1, 128>::kTileBBytes)}};
-    auto resident = [&](int si, int ks) {
-      switch (si) {
-        case 0: return resident_ctas<gemm_tc_kernel<kBDequant, kEpiStoreBf16, true, 2, 256>,
-                                     SmemLayout<2, 256>::bytes>(ks, sms, stream);
-        case 1: return resident_ctas<gemm_tc_kernel<kBDequant, kEpiStoreBf16, true, 1, 256>,
-                                     SmemLayout<1, 256>::bytes>(ks, sms, stream);
-        case 2: return resident_ctas<gemm_tc_kernel<kBDequant, kEpiStoreBf16, true, 2, 128>,
-                                     SmemLayout<2, 128>::bytes>(ks, sms, stream);
-        default: return resident_ctas<gemm_tc_kernel<kBDequant, kEpiStoreBf16, true, 1, 128>,
-                                      SmemLayout<1, 128>::bytes>(ks, sms, stream);
-      }
-    };
-    const int k_max = items[0].K;
-    int kb_min = 1 << 30;
-    for (int i = 0; i < n; ++i) kb_min = items[i].K / BK < kb_min ? items[i].K / BK : kb_min;
-    int best = -1, best_ks = 1;
-    double best_cost = 0.0;
-    for (int si = 0; si < 4; ++si) {
-      const Shape sh = shapes[si];
-      if (sh.mt == 2 && M < 2 * BM) continue;  // 256-row tiles only when rows fill them
-      double eq = 0.0;  // tiles of the longest K
-      for (int i = 0; i < n; ++i)
-        eq += static_cast<double>((items[i].N + sh.nb - 1) / sh.nb) *
-              ((M + sh.mt * BM - 1) / (sh.mt * BM)) * items[i].K / k_max;
-      const size_t part_bytes = static_cast<size_t>(sh.mt) * BM * (sh.nb + 4) * 4;
-      for (int ks = 1; ks <= 4; ++ks) {
-        if (ks > 1 && (part_bytes > sh.stage_bytes || kb_min < 2 * ks)) break;
-        const double waves = std::ceil(eq * ks / resident(si, ks) - 1e-9);
-        const double cost =
-            waves * (sh.a + sh.b * (static_cast<double>(k_max) / BK) / ks + (ks > 1 ? sh.c : 0.0));
-        if (best < 0 || cost < best_cost - 1e-9) {
-          best = si;
-          best_ks = ks;
-          best_cost = cost;
-        }
-      }
+    int Ns[kGemmGroup], Ks[kGemmGroup];
+    for (int i = 0; i < n; ++i) {
+      Ns[i] = items[i].N;
+      Ks[i] = items[i].K;
     }
-    if (best < 0) best = 1;
-    const int mt = shapes[best].mt, nb = shapes[best].nb;
-    const int ks = best_ks;
+    const PrefillPlan plan = plan_prefill_group(Ns, Ks, n, M, resident);
+    const int mt = plan.rows / BM, nb = plan.cols;
+    const int ks = plan.ks;
     const int bm = mt * BM;
     GemmGroup grp;
     grp.count = n;

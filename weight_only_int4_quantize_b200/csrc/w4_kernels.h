@@ -101,6 +101,23 @@ struct PrefillItem {
   void* y;             // bf16 [M, N]
   int N, K;
 };
+// Tile shape (rows x cols) and K split (CTAs per cluster) of a prefill launch.
+struct PrefillPlan {
+  int rows, cols, ks;
+};
+// Tile shapes in the order of the `resident` tables: 256 x 256, 128 x 256,
+// 256 x 128, 128 x 128; K splits 1 .. 4.
+constexpr int kPrefillShapes = 4;
+constexpr int kPrefillMaxSplit = 4;
+// CTAs of each tile shape that the current device runs at once in clusters
+// of 1 .. 4 (asked of the runtime once per device; estimated while `stream`
+// is being captured and the counts are not known yet).
+void prefill_resident(int sms, cudaStream_t stream,
+                      int (&resident)[kPrefillShapes][kPrefillMaxSplit]);
+// The plan of one grouped launch of n <= 16 linears (N[i] x K[i], sharing M
+// rows) from the launch's time model; host arithmetic only.
+PrefillPlan plan_prefill_group(const int* N, const int* K, int n, int M,
+                               const int (&resident)[kPrefillShapes][kPrefillMaxSplit]);
 // Up to 16 linears per tcgen05 launch (more in further launches).
 cudaError_t launch_prefill_gemm_group(const PrefillItem* items, int count, int M, bool pdl,
                                       bool static_w, cudaStream_t stream, unsigned* err);
