@@ -123,3 +123,14 @@ def test_plan_validation(_lib):
     assert f(n1, k1, 1, 64, zero, *o) == 1
     with pytest.raises(ValueError):
         w4.prefill_plan([(4096, 4096)], 64, [[148] * 4] * 3)
+
+
+def test_device_counts_need_a_device(_lib):
+    """Without given counts the plan asks the current device; with no usable
+    device the call returns W4_ERR_CUDA and launches nothing."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a device is present")
+    n1 = (ctypes.c_int64 * 1)(4096)
+    out = [ctypes.c_int() for _ in range(3)]
+    assert _lib.w4_prefill_plan(n1, n1, 1, 64, None, *[ctypes.byref(v) for v in out]) == 6
