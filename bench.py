@@ -141,37 +141,66 @@ def step_bytes():
 # ----------------------------------------------------------- clocks --------
 
 class ClockSampler:
+    """nvidia-smi samples every 100 ms, each stamped with the host time it
+    arrived; the summary keeps those inside the window marked by start() and
+    stop() (the timed region), or all of them if none fell inside."""
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
               "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
               "clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index: int):
+    def __init__(self, gpu_index: int, cmd=None, first_wait_s: float = 3.0):
         self.proc = None
-        self.gpu = gpu_index
+        self.cmd = cmd or ["nvidia-smi", "-i", str(gpu_index), f"--query-gpu={self.FIELDS}",
+                           "--format=csv,noheader,nounits", "-lms", "100"]
+        self.first_wait_s = first_wait_s
+        self.samples = []  # (host monotonic time, line)
+        self.window = (None, None)
+        self._reader = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.samples.append((time.monotonic(), line))
 
     def __enter__(self):
+        import threading
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.proc = subprocess.Popen(self.cmd, stdout=subprocess.PIPE,
+                                         stderr=subprocess.DEVNULL, text=True)
         except Exception:
             self.proc = None
+            return self
+        self._reader = threading.Thread(target=self._read, daemon=True)
+        self._reader.start()
+        # Sampling is running before the timed region starts.
+        t_end = time.monotonic() + self.first_wait_s
+        while not self.samples and time.monotonic() < t_end and self.proc.poll() is None:
+            time.sleep(0.01)
         return self
 
+    def start(self):
+        self.window = (time.monotonic(), None)
+
+    def stop(self):
+        self.window = (self.window[0], time.monotonic())
+
     def __exit__(self, *a):
-        self.out = ""
         if self.proc is not None:
             self.proc.terminate()
             try:
-                self.out, _ = self.proc.communicate(timeout=5)
+                self.proc.wait(timeout=5)
             except Exception:
                 self.proc.kill()
+        if self._reader is not None:
+            self._reader.join(timeout=5)
 
     def summary(self):
+        t0, t1 = self.window
+        inside = [ln for t, ln in self.samples
+                  if t0 is not None and t1 is not None and t0 <= t <= t1]
+        lines = inside or [ln for _, ln in self.samples]
         sm, mx, reasons = [], [], set()
         names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
-        for line in (self.out or "").splitlines():
+        for line in lines:
             parts = [p.strip() for p in line.split(",")]
             if len(parts) < 7:
                 continue
@@ -186,7 +215,8 @@ class ClockSampler:
         if not sm:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
-                "samples": len(sm)}
+                "samples": len(sm),
+                "window": "timed region" if inside else "whole sampler run"}
 
 
 # ------------------------------------------------------------ CPU leg ------
@@ -606,7 +636,7 @@ def breakdown(torch, dev, hbm, bf16_peak, bf16_sus):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-breakdown", action="store_true")
@@ -662,6 +692,7 @@ def main():
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local) as clk:
         torch.cuda.synchronize()
+        clk.start()
         start.record()
         for i in range(args.steps):
             e = ev[i]
@@ -672,6 +703,7 @@ def main():
             e[2].record()
         end.record()
         torch.cuda.synchronize()
+        clk.stop()
     if pg:
         pg.barrier()
     total_ms = start.elapsed_time(end)
