@@ -1,6 +1,7 @@
 // tcgen05 GEMM core for sm_100a: D[M, N] = A[M, K] . B[N, K]^T with both
 // operands K-major in 128-byte-swizzled shared memory and the fp32
-// accumulator in tensor memory.  One CTA computes a 128 x 256 tile.
+// accumulator in tensor memory.  One CTA computes a tile of 128 or 256 rows
+// by 128 or 256 columns.
 //
 // Warp roles (10 warps):
 //   warp 0      TMA producer (A tiles; also B tiles when B comes from TMA)
@@ -217,7 +218,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __nv_bfloat16* __restrict__ y = nullptr;
   int N = N_arg, K = K_arg;
   int tile_n = blockIdx.x, tile_m = blockIdx.y;
-  // Split K over a thread-block cluster (prefill launches with few tiles):
+  // Split K over a thread-block cluster (prefill launches whose plan splits K):
   // CTA `rank` of the cluster takes its share of the k-blocks, and the
   // partial accumulators are added through distributed shared memory.
   int ks = 1, rank = 0;
